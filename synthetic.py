@@ -1,0 +1,122 @@
+"""Seeded synthetic inputs for the MoBA prefill workloads.
+
+This module is shared by the fp64 oracle's tests and by the CUDA path's
+tests and benchmark, and holds none of the method's arithmetic: it only
+draws numbers.
+
+Recipe (the same for every workload):
+  * q, k, v are bf16 roundings of standard normal draws, packed [T][H][d];
+  * every (sequence, block, kv head) gets an offset vector with i.i.d.
+    N(0, 0.5^2) entries, added to the keys of that block in fp32 before the
+    rounding, so that block means differ;
+  * draws come from one torch.Generator seeded with the workload's seed, on
+    the device the tensors are made on, in this order: offsets, q, k, v, each
+    in chunks of CHUNK tokens (so the numbers depend on the device, the seed
+    and nothing else).
+Varlen lengths come from numpy.random.default_rng(seed): uniform integers in
+[lo, hi], rounded down to a multiple of `round_to`.
+"""
+import dataclasses
+from typing import List, Optional
+
+import numpy as np
+import torch
+
+CHUNK = 65536
+
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    lengths: List[int]          # tokens of each sequence (batch = equal lengths)
+    Hq: int
+    Hkv: int
+    d: int
+    B: int                      # block size
+    k: int                      # top-k, counting the own block
+    seed: int
+    batch_mode: bool = True     # equal lengths passed as a [b, N, H, d] batch
+    note: str = ""
+
+    @property
+    def T(self) -> int:
+        return int(sum(self.lengths))
+
+    @property
+    def cu(self) -> np.ndarray:
+        cu = np.zeros(len(self.lengths) + 1, dtype=np.int64)
+        cu[1:] = np.cumsum(np.asarray(self.lengths, dtype=np.int64))
+        return cu
+
+    def with_k(self, k: int) -> "Workload":
+        return dataclasses.replace(self, k=k, name="%s_k%d" % (self.name, k))
+
+
+def varlen_lengths(seed: int, n: int, lo: int, hi: int, round_to: int) -> List[int]:
+    rng = np.random.default_rng(seed)
+    raw = rng.integers(lo, hi, size=n, endpoint=True)
+    return [int(max(round_to, (x // round_to) * round_to)) for x in raw]
+
+
+# The five benchmark workloads.
+TINY = Workload("tiny_2k", [2048], 1, 1, 64, 256, 3, seed=0,
+                note="batch 1, 1 head, d=64, N=2048, B=256 (n=8), k=3")
+FINE_32K = Workload("fine_32k", [32768], 32, 8, 128, 256, 32, seed=1,
+                    note="32 q / 8 kv heads, d=128, N=32768, B=256 (128 blocks), k=32")
+LONG_128K = Workload("long_128k", [131072], 32, 8, 128, 4096, 12, seed=2,
+                     note="32 q / 8 kv heads, d=128, N=131072, B=4096 (32 blocks), k=12")
+MILLION = Workload("prefill_1m", [1048576], 32, 8, 128, 4096, 12, seed=3,
+                   note="32 q / 8 kv heads, d=128, N=1048576, B=4096 (256 blocks), k=12")
+VARLEN = Workload("varlen_8seq", varlen_lengths(4, 8, 4096, 65536, 256), 32, 8, 128, 512, 8,
+                  seed=4, batch_mode=False,
+                  note="8 packed sequences, lengths U[4096,65536] rounded to 256, B=512, k=8")
+
+WORKLOADS = {w.name: w for w in (TINY, FINE_32K, LONG_128K, MILLION, VARLEN)}
+
+
+def block_ids(lengths: List[int], B: int) -> np.ndarray:
+    """Global block id (sequence by sequence) of every token."""
+    out = []
+    base = 0
+    for L in lengths:
+        j = np.arange(L, dtype=np.int64) // B
+        out.append(j + base)
+        base += (L + B - 1) // B
+    return np.concatenate(out) if out else np.zeros(0, dtype=np.int64)
+
+
+def make_qkv(w: Workload, device="cpu", seed: Optional[int] = None, need_v: bool = True):
+    """q [T,Hq,d], k [T,Hkv,d], v [T,Hkv,d] as bf16 tensors on `device`."""
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed if seed is None else seed)
+    T = w.T
+    bid = block_ids(w.lengths, w.B)
+    nb = int(bid[-1]) + 1 if T else 0
+    offs = torch.randn(nb, w.Hkv, w.d, generator=g, device=dev, dtype=torch.float32) * 0.5
+    bid_t = torch.from_numpy(bid).to(dev)
+
+    def draw(H, offsets=None):
+        out = torch.empty(T, H, w.d, device=dev, dtype=torch.bfloat16)
+        for a in range(0, T, CHUNK):
+            e = min(T, a + CHUNK)
+            x = torch.randn(e - a, H, w.d, generator=g, device=dev, dtype=torch.float32)
+            if offsets is not None:
+                x += offsets[bid_t[a:e]]
+            out[a:e] = x.to(torch.bfloat16)
+            del x
+        return out
+
+    q = draw(w.Hq)
+    k = draw(w.Hkv, offs)
+    v = draw(w.Hkv) if need_v else None
+    return q, k, v
+
+
+def sample_rows(w: Workload, per_head_rows: int, seed: int = 1234) -> np.ndarray:
+    """Seeded sample of distinct global query rows, sorted (all rows if fewer)."""
+    T = w.T
+    if per_head_rows >= T:
+        return np.arange(T, dtype=np.int64)
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(T, size=per_head_rows, replace=False)).astype(np.int64)
