@@ -1,0 +1,295 @@
+"""Python binding of libmoba (C ABI in include/moba.h): argument marshalling only.
+
+Every step of the MoBA prefill forward runs in libmoba's CUDA kernels; this
+module only passes torch tensors' device pointers, sizes and the current
+stream through ctypes.  There is no fallback: if libmoba.so is missing or no
+CUDA device is present the calls raise.
+
+    import block_sparse_long_07_b200 as moba
+    o, lse = moba.forward(q, k, v, block_size=4096, top_k=12)          # [b,N,H,d]
+    o, lse = moba.forward_varlen(q, k, v, cu_seqlens, block_size=512, top_k=8)
+    o, lse = moba.full_causal(q, k, v)
+    sel = moba.gate(q, k, block_size=..., top_k=...)
+"""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoba.so")
+
+MOBA_OK = 0
+_STATUS = {0: "MOBA_OK", 1: "MOBA_ERR_INVALID_ARG", 2: "MOBA_ERR_UNSUPPORTED",
+           3: "MOBA_ERR_WORKSPACE", 4: "MOBA_ERR_CUDA", 5: "MOBA_ERR_TIMEOUT",
+           6: "MOBA_ERR_DEVICE_CHECK"}
+
+EXPORTS = ("moba_workspace_size", "moba_workspace_size_varlen", "moba_gate", "moba_gate_varlen",
+           "moba_forward", "moba_forward_varlen", "moba_full_causal_workspace_size",
+           "moba_full_causal", "moba_full_causal_varlen", "moba_last_device_status",
+           "moba_status_string", "moba_version", "moba_profile_enable", "moba_profile_reset",
+           "moba_profile_read")
+
+
+class MobaError(RuntimeError):
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__("%s failed: %s" % (what, _STATUS.get(code, str(code))))
+
+
+class MobaParams(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("seqlen", ctypes.c_int),
+                ("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("block_size", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("softmax_scale", ctypes.c_float)]
+
+
+class KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 24), ("launches", ctypes.c_int),
+                ("total_ms", ctypes.c_double)]
+
+
+_lib = None
+
+
+def load_library(path=None):
+    """Load libmoba.so (raises OSError if it is missing: no fallback exists)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise OSError("libmoba.so not built at %s (run python -m block_sparse_long_07_b200.build)" % p)
+    lib = ctypes.CDLL(p)
+    vp, sz, i32, i64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_int64
+    pp = ctypes.POINTER(MobaParams)
+    lib.moba_workspace_size.restype = sz
+    lib.moba_workspace_size.argtypes = [pp, i32]
+    lib.moba_workspace_size_varlen.restype = sz
+    lib.moba_workspace_size_varlen.argtypes = [pp, i64, i32, i32]
+    lib.moba_gate.restype = i32
+    lib.moba_gate.argtypes = [vp, vp, vp, pp, vp, sz, vp]
+    lib.moba_gate_varlen.restype = i32
+    lib.moba_gate_varlen.argtypes = [vp, vp, vp, i32, i64, vp, pp, vp, sz, vp]
+    lib.moba_forward.restype = i32
+    lib.moba_forward.argtypes = [vp, vp, vp, vp, vp, vp, pp, vp, sz, vp]
+    lib.moba_forward_varlen.restype = i32
+    lib.moba_forward_varlen.argtypes = [vp, vp, vp, vp, i32, i64, vp, vp, vp, pp, vp, sz, vp]
+    lib.moba_full_causal_workspace_size.restype = sz
+    lib.moba_full_causal_workspace_size.argtypes = [i64, i32]
+    lib.moba_full_causal.restype = i32
+    lib.moba_full_causal.argtypes = [vp, vp, vp, vp, vp, pp, vp, sz, vp]
+    lib.moba_full_causal_varlen.restype = i32
+    lib.moba_full_causal_varlen.argtypes = [vp, vp, vp, vp, i32, i64, vp, vp, pp, vp, sz, vp]
+    lib.moba_last_device_status.restype = i32
+    lib.moba_last_device_status.argtypes = [vp, vp]
+    lib.moba_status_string.restype = ctypes.c_char_p
+    lib.moba_status_string.argtypes = [i32]
+    lib.moba_version.restype = i32
+    lib.moba_version.argtypes = []
+    lib.moba_profile_enable.restype = None
+    lib.moba_profile_enable.argtypes = [i32]
+    lib.moba_profile_reset.restype = None
+    lib.moba_profile_reset.argtypes = []
+    lib.moba_profile_read.restype = i32
+    lib.moba_profile_read.argtypes = [ctypes.POINTER(KernelTime), i32]
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _check(code, what):
+    if code != MOBA_OK:
+        raise MobaError(code, what)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_params(batch, seqlen, Hq, Hkv, d, block_size=128, top_k=1, softmax_scale=0.0):
+    return MobaParams(int(batch), int(seqlen), int(Hq), int(Hkv), int(d), int(block_size),
+                      int(top_k), float(softmax_scale))
+
+
+def _require_cuda_bf16(*ts):
+    torch = _torch()
+    for t in ts:
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+            raise ValueError("expected contiguous bf16 CUDA tensors")
+
+
+def workspace_size(params, heads_per_pass=0):
+    return int(load_library().moba_workspace_size(ctypes.byref(params), int(heads_per_pass)))
+
+
+def workspace_size_varlen(params, total_tokens, num_seqs, heads_per_pass=0):
+    return int(load_library().moba_workspace_size_varlen(ctypes.byref(params), int(total_tokens),
+                                                         int(num_seqs), int(heads_per_pass)))
+
+
+def full_causal_workspace_size(total_tokens, num_seqs):
+    return int(load_library().moba_full_causal_workspace_size(int(total_tokens), int(num_seqs)))
+
+
+DEFAULT_WS_BUDGET = 32 << 30  # bytes a forward call may take for its workspace by default
+
+
+def pick_heads_per_pass(size_fn, num_kv_heads, budget=DEFAULT_WS_BUDGET):
+    """Largest number of kv heads per pass whose workspace fits `budget` (at least 1)."""
+    for hp in range(num_kv_heads, 0, -1):
+        if size_fn(hp) <= budget:
+            return hp
+    return 1
+
+
+def alloc_workspace(nbytes, device=None):
+    torch = _torch()
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def profile_enable(on=True):
+    """Bracket every library kernel launch with CUDA events (see moba.h)."""
+    lib = load_library()
+    lib.moba_profile_reset()
+    lib.moba_profile_enable(1 if on else 0)
+
+
+def profile_read():
+    """{kernel class: (launches, total device ms)} since profile_enable."""
+    arr = (KernelTime * 16)()
+    n = load_library().moba_profile_read(arr, 16)
+    return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n)}
+
+
+def last_device_status(ws, stream=None):
+    """Synchronises and returns the device status latched in `ws` (0 = ok)."""
+    return int(load_library().moba_last_device_status(_ptr(ws), _stream(stream)))
+
+
+def gate(q, k, block_size, top_k, softmax_scale=0.0, ws=None, sel=None, stream=None):
+    """Selection sel [b, Hq, N, top_k] int32 for q [b,N,Hq,d], k [b,N,Hkv,d]."""
+    torch = _torch()
+    _require_cuda_bf16(q, k)
+    b, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    p = make_params(b, N, Hq, Hkv, d, block_size, top_k, softmax_scale)
+    if sel is None:
+        sel = torch.empty(b, Hq, N, top_k, dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(workspace_size(p, 1), q.device)
+    _check(load_library().moba_gate(_ptr(q), _ptr(k), _ptr(sel), ctypes.byref(p), _ptr(ws),
+                                    ws.numel(), _stream(stream)), "moba_gate")
+    return sel
+
+
+def gate_varlen(q, k, cu_seqlens, block_size, top_k, softmax_scale=0.0, ws=None, sel=None,
+                stream=None):
+    """Selection sel [Hq, T, top_k] for packed q [T,Hq,d], k [T,Hkv,d]."""
+    torch = _torch()
+    _require_cuda_bf16(q, k)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    nseq = cu_seqlens.numel() - 1
+    p = make_params(1, 0, Hq, Hkv, d, block_size, top_k, softmax_scale)
+    if sel is None:
+        sel = torch.empty(Hq, T, top_k, dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(workspace_size_varlen(p, T, nseq, 1), q.device)
+    _check(load_library().moba_gate_varlen(_ptr(q), _ptr(k), _ptr(cu_seqlens), nseq, T,
+                                           _ptr(sel), ctypes.byref(p), _ptr(ws), ws.numel(),
+                                           _stream(stream)), "moba_gate_varlen")
+    return sel
+
+
+def forward(q, k, v, block_size, top_k, softmax_scale=0.0, ws=None, out=None, lse=None,
+            sel_out=None, stream=None):
+    """MoBA prefill forward for q [b,N,Hq,d], k/v [b,N,Hkv,d]: (o, lse)."""
+    torch = _torch()
+    _require_cuda_bf16(q, k, v)
+    b, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    p = make_params(b, N, Hq, Hkv, d, block_size, top_k, softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(b, Hq, N, dtype=torch.float32, device=q.device)
+    if ws is None:
+        hp = pick_heads_per_pass(lambda n: workspace_size(p, n), Hkv)
+        ws = alloc_workspace(workspace_size(p, hp), q.device)
+    _check(load_library().moba_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                       _ptr(sel_out), ctypes.byref(p), _ptr(ws), ws.numel(),
+                                       _stream(stream)), "moba_forward")
+    return out, lse
+
+
+def forward_varlen(q, k, v, cu_seqlens, block_size, top_k, softmax_scale=0.0, ws=None,
+                   out=None, lse=None, sel_out=None, stream=None):
+    """MoBA prefill forward on packed sequences q [T,Hq,d], k/v [T,Hkv,d]: (o, lse [Hq,T])."""
+    torch = _torch()
+    _require_cuda_bf16(q, k, v)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    nseq = cu_seqlens.numel() - 1
+    p = make_params(1, 0, Hq, Hkv, d, block_size, top_k, softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(Hq, T, dtype=torch.float32, device=q.device)
+    if ws is None:
+        hp = pick_heads_per_pass(lambda n: workspace_size_varlen(p, T, nseq, n), Hkv)
+        ws = alloc_workspace(workspace_size_varlen(p, T, nseq, hp), q.device)
+    _check(load_library().moba_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq,
+                                              T, _ptr(out), _ptr(lse), _ptr(sel_out),
+                                              ctypes.byref(p), _ptr(ws), ws.numel(),
+                                              _stream(stream)), "moba_forward_varlen")
+    return out, lse
+
+
+def full_causal(q, k, v, softmax_scale=0.0, ws=None, out=None, lse=None, stream=None):
+    """Dense causal attention (the k = n comparator) for q [b,N,Hq,d]: (o, lse)."""
+    torch = _torch()
+    _require_cuda_bf16(q, k, v)
+    b, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    p = make_params(b, N, Hq, Hkv, d, 128, 1, softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(b, Hq, N, dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(full_causal_workspace_size(b * N, b), q.device)
+    _check(load_library().moba_full_causal(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                           ctypes.byref(p), _ptr(ws), ws.numel(),
+                                           _stream(stream)), "moba_full_causal")
+    return out, lse
+
+
+def full_causal_varlen(q, k, v, cu_seqlens, softmax_scale=0.0, ws=None, out=None, lse=None,
+                       stream=None):
+    torch = _torch()
+    _require_cuda_bf16(q, k, v)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    nseq = cu_seqlens.numel() - 1
+    p = make_params(1, 0, Hq, Hkv, d, 128, 1, softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(Hq, T, dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(full_causal_workspace_size(T, nseq), q.device)
+    _check(load_library().moba_full_causal_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                                                  nseq, T, _ptr(out), _ptr(lse), ctypes.byref(p),
+                                                  _ptr(ws), ws.numel(), _stream(stream)),
+           "moba_full_causal_varlen")
+    return out, lse

@@ -1,0 +1,687 @@
+// moba_api.cu -- the C ABI of libmoba (declared in include/moba.h): argument
+// checks, workspace carving, TMA descriptor encoding and the launch sequence
+// of the MoBA causal prefill forward on one sm_100a GPU.
+//
+// Launch sequence of moba_forward (one stream, no host synchronisation):
+//   plan -> pool -> gate -> for each pass of kv heads:
+//     bucket scan -> bucket scatter -> routed attention -> own-block
+//     attention -> merge
+// The routed/own split and the online-softmax merge follow the method's
+// implementation outline (MoBA: Mixture of Block Attention, wispaper.ai
+// blog, "Efficiency and Implementation"; sherconan.github.io step 5):
+// queries are arranged by their selected past blocks (bucketing), attention
+// runs per block, and the per-block results are recombined by online
+// softmax.  Each step is a kernel of this library.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "moba.h"
+#include "aux_kernels.cuh"
+#include "attn_tc.cuh"
+#include "common.cuh"
+#include "layout.cuh"
+
+using namespace moba;
+
+namespace {
+
+// ------------------------------------------------------------ kernel timer
+enum KernelClass {
+  kKPlan, kKPool, kKGate, kKScan, kKScatter, kKRouted, kKOwn, kKMerge, kKDense, kKNum
+};
+const char* const kKernelNames[kKNum] = {"plan", "pool", "gate", "bucket_scan", "bucket_scatter",
+                                         "attn_routed", "attn_own", "merge", "attn_dense"};
+struct TimedLaunch {
+  int cls;
+  cudaEvent_t a, b;
+};
+struct KernelTimer {
+  bool on = false;
+  std::vector<TimedLaunch> pending;
+  int launches[kKNum] = {};
+  double ms[kKNum] = {};
+};
+KernelTimer& timer() {
+  static KernelTimer t;
+  return t;
+}
+// RAII bracket around one launch: events on the launch stream when enabled.
+struct Timed {
+  int cls;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr, b = nullptr;
+  Timed(int c, cudaStream_t s) : cls(c), st(s) {
+    if (!timer().on) return;
+    if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) {
+      a = b = nullptr;
+      return;
+    }
+    cudaEventRecord(a, st);
+  }
+  ~Timed() {
+    if (!a) return;
+    cudaEventRecord(b, st);
+    timer().pending.push_back(TimedLaunch{cls, a, b});
+  }
+};
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Problem {
+  bool varlen;
+  int nseq;
+  int N;          // batch: seqlen
+  int64_t T;
+  const int32_t* cu;
+  int Hq, Hkv, G, D, B, topk;
+  float scale;
+  int64_t NBmax, NQTmax;
+  int64_t max_blocks_per_seq;  // upper bound
+  RowLayout R;
+};
+
+struct Ws {
+  uint32_t* status;
+  Plan P;
+  float* kbar;
+  uint32_t* counts;
+  int32_t* entry_off;
+  int32_t* tile_off;
+  uint32_t* cursor;
+  uint2* entries;
+  __nv_bfloat16* part_O;
+  float* part_lse;
+  float* own_O;
+  float* own_lse;
+  int32_t* sel;
+  size_t bytes;
+};
+
+// Carve (or only measure, base == nullptr) the workspace for `nu` kv heads per pass.
+Ws carve(const Problem& pr, int nu, char* base) {
+  Ws w;
+  memset(&w, 0, sizeof w);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + bytes);
+    return p;
+  };
+  const int64_t NB = pr.NBmax, NQ = pr.NQTmax;
+  const int64_t np = pr.topk > 1 ? pr.topk - 1 : 0;
+  (void)NQ;
+  w.status = reinterpret_cast<uint32_t*>(take(kAlign));
+  w.P.totals = reinterpret_cast<int32_t*>(take(4 * sizeof(int32_t)));
+  w.P.blk_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (pr.nseq + 1)));
+  w.P.qt_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (pr.nseq + 1)));
+  w.P.blk_tok = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * NB));
+  w.P.blk_len = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * NB));
+  w.kbar = reinterpret_cast<float*>(take(sizeof(float) * (size_t)pr.Hkv * NB * pr.D));
+  w.counts = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * (size_t)pr.Hkv * NB));
+  w.sel = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)pr.Hq * pr.T * pr.topk));
+  w.entry_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * ((size_t)nu * NB + 1)));
+  w.tile_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * ((size_t)nu * NB + 1)));
+  w.cursor = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * (size_t)nu * NB));
+  const size_t prow = (size_t)nu * pr.T * pr.G;  // partial rows per pass
+  w.entries = reinterpret_cast<uint2*>(take(sizeof(uint2) * prow * np));
+  w.part_O = reinterpret_cast<__nv_bfloat16*>(take(2 * prow * np * pr.D));
+  w.part_lse = reinterpret_cast<float*>(take(sizeof(float) * prow * np));
+  w.own_O = reinterpret_cast<float*>(take(sizeof(float) * prow * pr.D));
+  w.own_lse = reinterpret_cast<float*>(take(sizeof(float) * prow));
+  w.bytes = off;
+  return w;
+}
+
+moba_status make_problem(const moba_params* p, bool varlen, const int32_t* cu, int num_seqs,
+                         int64_t total_tokens, bool need_blocks, Problem* out) {
+  if (!p) return MOBA_ERR_INVALID_ARG;
+  Problem pr;
+  memset(&pr, 0, sizeof pr);
+  pr.varlen = varlen;
+  if (varlen) {
+    if (!cu || num_seqs <= 0 || total_tokens < 0) return MOBA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(cu) % 4) return MOBA_ERR_INVALID_ARG;
+    pr.nseq = num_seqs;
+    pr.N = 0;
+    pr.T = total_tokens;
+    pr.cu = cu;
+  } else {
+    if (p->batch <= 0 || p->seqlen < 0) return MOBA_ERR_INVALID_ARG;
+    pr.nseq = p->batch;
+    pr.N = p->seqlen;
+    pr.T = (int64_t)p->batch * p->seqlen;
+    pr.cu = nullptr;
+  }
+  if (pr.T >= (int64_t(1) << 31) - 256) return MOBA_ERR_UNSUPPORTED;
+  if (p->num_q_heads <= 0 || p->num_kv_heads <= 0 || p->num_q_heads % p->num_kv_heads)
+    return MOBA_ERR_INVALID_ARG;
+  pr.Hq = p->num_q_heads;
+  pr.Hkv = p->num_kv_heads;
+  pr.G = pr.Hq / pr.Hkv;
+  if (p->head_dim != 64 && p->head_dim != 128) return MOBA_ERR_UNSUPPORTED;
+  pr.D = p->head_dim;
+  if (need_blocks) {
+    if (p->block_size <= 0 || p->top_k <= 0) return MOBA_ERR_INVALID_ARG;
+    if (p->block_size % kTileM) return MOBA_ERR_UNSUPPORTED;
+    pr.B = p->block_size;
+    pr.topk = p->top_k;
+  } else {
+    pr.B = kTileM;  // block numbering unused by the dense kernel
+    pr.topk = 1;
+  }
+  if (pr.G > 65535 || pr.topk > 65536) return MOBA_ERR_UNSUPPORTED;
+  pr.scale = (p->softmax_scale > 0.f) ? p->softmax_scale : 1.0f / sqrtf((float)pr.D);
+  if (!(pr.scale < INFINITY)) return MOBA_ERR_INVALID_ARG;
+  if (varlen) {
+    pr.NBmax = pr.T / pr.B + pr.nseq;
+    pr.NQTmax = pr.T / kTileM + pr.nseq;
+    pr.max_blocks_per_seq = (pr.T + pr.B - 1) / pr.B;
+  } else {
+    const int64_t nb = ((int64_t)pr.N + pr.B - 1) / pr.B;
+    pr.NBmax = (int64_t)pr.nseq * nb;
+    pr.NQTmax = (int64_t)pr.nseq * (((int64_t)pr.N + kTileM - 1) / kTileM);
+    pr.max_blocks_per_seq = nb;
+    if (nb > kMaxBlocksPerSeq) return MOBA_ERR_UNSUPPORTED;
+  }
+  if (pr.NBmax < 1) pr.NBmax = 1;
+  if (pr.NQTmax < 1) pr.NQTmax = 1;
+  if (pr.NBmax > INT32_MAX / 4 || pr.NQTmax > INT32_MAX / 4) return MOBA_ERR_UNSUPPORTED;
+  if (varlen) {
+    pr.R.seq_stride = 0;
+    pr.R.head_stride = pr.T;
+    pr.R.use_token = 1;
+  } else {
+    pr.R.seq_stride = (int64_t)pr.Hq * pr.N;
+    pr.R.head_stride = pr.N;
+    pr.R.use_token = 0;
+  }
+  *out = pr;
+  return MOBA_OK;
+}
+
+int pow2_at_least(int64_t x) {
+  int v = 1;
+  while (v < x) v <<= 1;
+  return v;
+}
+
+// ---------------------------------------------------------------- TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [T][H][D] bf16 viewed as (x = D, y = H, z = T), box 64 x 1 x 128, 128-B swizzle.
+bool make_tmap(CUtensorMap* m, const void* ptr, int H, int64_t T, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)(T > 0 ? T : 1)};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kTileM};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+template <int D, int MODE>
+moba_status launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const AttnArgs& a, cudaStream_t stream) {
+  using C = AttnCfg<D>;
+  auto kern = attn_tc_kernel<D, MODE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+      cudaSuccess)
+    return MOBA_ERR_CUDA;
+  const int grid = num_sms();
+  if (grid <= 0) return MOBA_ERR_CUDA;
+  Timed tm(MODE == kRouted ? kKRouted : (MODE == kOwn ? kKOwn : kKDense), stream);
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA;
+}
+
+template <int D, int KM>
+moba_status launch_gate_km(const Problem& pr, const void* q, const Ws& w, int32_t* sel,
+                           uint32_t* counts, cudaStream_t st) {
+  const size_t smem = sizeof(float) * kGateChunk * D + sizeof(uint32_t) * kMaxBlocksPerSeq;
+  auto kern = gate_kernel<D, KM>;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess)
+    return MOBA_ERR_CUDA;
+  SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
+  dim3 grid((unsigned)pr.NQTmax, (unsigned)pr.Hq);
+  Timed tm(kKGate, st);
+  kern<<<grid, 128, smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(q), pr.Hq, pr.G, pr.B,
+                                pr.topk, L, w.P, (int)pr.NBmax, w.kbar, sel, pr.R, counts,
+                                w.status);
+  return cudaGetLastError() == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA;
+}
+
+template <int D>
+moba_status launch_gate(const Problem& pr, const void* q, const Ws& w, int32_t* sel,
+                        uint32_t* counts, cudaStream_t st) {
+  const int64_t npast = pr.topk - 1;
+  const int64_t need = (npast >= pr.max_blocks_per_seq - 1) ? 1 : npast;
+  switch (pow2_at_least(need)) {
+    case 1: return launch_gate_km<D, 1>(pr, q, w, sel, counts, st);
+    case 2: return launch_gate_km<D, 2>(pr, q, w, sel, counts, st);
+    case 4: return launch_gate_km<D, 4>(pr, q, w, sel, counts, st);
+    case 8: return launch_gate_km<D, 8>(pr, q, w, sel, counts, st);
+    case 16: return launch_gate_km<D, 16>(pr, q, w, sel, counts, st);
+    case 32: return launch_gate_km<D, 32>(pr, q, w, sel, counts, st);
+    case 64: return launch_gate_km<D, 64>(pr, q, w, sel, counts, st);
+    default: return MOBA_ERR_UNSUPPORTED;
+  }
+}
+
+template <int KS>
+moba_status launch_scatter_ks(const Problem& pr, const Ws& w, const int32_t* sel, int u0, int nu,
+                              cudaStream_t st) {
+  SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
+  dim3 grid((unsigned)pr.NQTmax, (unsigned)(nu * pr.G));
+  Timed tm(kKScatter, st);
+  bucket_scatter_kernel<KS><<<grid, 128, sizeof(uint32_t) * kMaxBlocksPerSeq, st>>>(
+      sel, pr.R, pr.topk, pr.B, pr.G, u0, nu, L, w.P, w.entry_off, w.cursor, w.entries,
+      w.status);
+  return cudaGetLastError() == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA;
+}
+
+moba_status launch_scatter(const Problem& pr, const Ws& w, const int32_t* sel, int u0, int nu,
+                           cudaStream_t st) {
+  int64_t need = pr.topk - 1;
+  if (need > pr.max_blocks_per_seq - 1) need = pr.max_blocks_per_seq - 1;
+  if (need < 1) need = 1;
+  switch (pow2_at_least(need)) {
+    case 1: return launch_scatter_ks<1>(pr, w, sel, u0, nu, st);
+    case 2: return launch_scatter_ks<2>(pr, w, sel, u0, nu, st);
+    case 4: return launch_scatter_ks<4>(pr, w, sel, u0, nu, st);
+    case 8: return launch_scatter_ks<8>(pr, w, sel, u0, nu, st);
+    case 16: return launch_scatter_ks<16>(pr, w, sel, u0, nu, st);
+    case 32: return launch_scatter_ks<32>(pr, w, sel, u0, nu, st);
+    case 64: return launch_scatter_ks<64>(pr, w, sel, u0, nu, st);
+    default: return MOBA_ERR_UNSUPPORTED;
+  }
+}
+
+bool topk_supported(const Problem& pr) {
+  const int64_t npast = pr.topk - 1;
+  return npast <= 64 || npast >= pr.max_blocks_per_seq - 1;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moba_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign)) return MOBA_ERR_WORKSPACE;
+  if (ws_bytes < need) return MOBA_ERR_WORKSPACE;
+  return MOBA_OK;
+}
+
+#define MOBA_TRY(x)                      \
+  do {                                   \
+    moba_status _s = (x);                \
+    if (_s != MOBA_OK) return _s;        \
+  } while (0)
+#define MOBA_CUDA(x)                                   \
+  do {                                                 \
+    if ((x) != cudaSuccess) return MOBA_ERR_CUDA;      \
+  } while (0)
+
+moba_status run_plan_pool(const Problem& pr, const void* k, const Ws& w, cudaStream_t st) {
+  SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
+  {
+    Timed tm(kKPlan, st);
+    plan_kernel<<<1, 1024, 0, st>>>(L, pr.B, w.P, (int)pr.NBmax, (int)pr.NQTmax, w.status);
+  }
+  MOBA_CUDA(cudaGetLastError());
+  dim3 grid((unsigned)pr.NBmax, (unsigned)pr.Hkv);
+  Timed tm(kKPool, st);
+  if (pr.D == 128)
+    pool_kernel<128><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(k), pr.Hkv,
+                                           w.P, (int)pr.NBmax, w.kbar);
+  else
+    pool_kernel<64><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(k), pr.Hkv,
+                                          w.P, (int)pr.NBmax, w.kbar);
+  MOBA_CUDA(cudaGetLastError());
+  return MOBA_OK;
+}
+
+moba_status gate_impl(const Problem& pr, const void* q, const void* k, int32_t* sel, void* ws,
+                      size_t ws_bytes, cudaStream_t st) {
+  if (!q || !k || !sel || !aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(sel) & 3))
+    return MOBA_ERR_INVALID_ARG;
+  if (!topk_supported(pr)) return MOBA_ERR_UNSUPPORTED;
+  const Ws need = carve(pr, 1, nullptr);
+  MOBA_TRY(check_ws(ws, ws_bytes, need.bytes));
+  if (pr.T == 0) return MOBA_OK;
+  const Ws w = carve(pr, 1, static_cast<char*>(ws));
+  MOBA_TRY(run_plan_pool(pr, k, w, st));
+  return pr.D == 128 ? launch_gate<128>(pr, q, w, sel, nullptr, st)
+                     : launch_gate<64>(pr, q, w, sel, nullptr, st);
+}
+
+template <int D>
+moba_status forward_passes(const Problem& pr, const void* q, const void* k, const void* v,
+                           void* o, float* lse, const Ws& w, int32_t* sel, int nu_max,
+                           cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, pr.Hq, pr.T, D) || !make_tmap(&tk, k, pr.Hkv, pr.T, D) ||
+      !make_tmap(&tv, v, pr.Hkv, pr.T, D))
+    return MOBA_ERR_CUDA;
+  SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
+  MOBA_CUDA(cudaMemsetAsync(w.counts, 0, sizeof(uint32_t) * (size_t)pr.Hkv * pr.NBmax, st));
+  MOBA_TRY(launch_gate<D>(pr, q, w, sel, w.counts, st));
+  AttnArgs a;
+  memset(&a, 0, sizeof a);
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.Hq = pr.Hq;
+  a.Hkv = pr.Hkv;
+  a.G = pr.G;
+  a.B = pr.B;
+  a.topk = pr.topk;
+  a.scale_log2 = pr.scale * 1.4426950408889634f;
+  a.L = L;
+  a.P = w.P;
+  a.R = pr.R;
+  a.tile_off = w.tile_off;
+  a.entry_off = w.entry_off;
+  a.entries = w.entries;
+  a.part_O = w.part_O;
+  a.part_lse = w.part_lse;
+  a.own_O = w.own_O;
+  a.own_lse = w.own_lse;
+  a.o = reinterpret_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.status = w.status;
+  for (int u0 = 0; u0 < pr.Hkv; u0 += nu_max) {
+    const int nu = (pr.Hkv - u0) < nu_max ? (pr.Hkv - u0) : nu_max;
+    a.u0 = u0;
+    a.nu = nu;
+    if (pr.topk > 1) {
+      {
+        Timed tm(kKScan, st);
+        bucket_scan_kernel<<<1, 1024, 0, st>>>(w.counts, u0, nu, w.P, (int)pr.NBmax,
+                                               w.entry_off, w.tile_off, w.cursor);
+      }
+      MOBA_CUDA(cudaGetLastError());
+      MOBA_TRY(launch_scatter(pr, w, sel, u0, nu, st));
+      MOBA_TRY((launch_attn<D, kRouted>(tq, tk, tv, a, st)));
+    }
+    MOBA_TRY((launch_attn<D, kOwn>(tq, tk, tv, a, st)));
+    if (pr.topk > 1) {
+      const int64_t warps = pr.T * nu * pr.G;
+      const unsigned blocks = (unsigned)((warps + 7) / 8);
+      Timed tm(kKMerge, st);
+      merge_kernel<D><<<blocks, 256, 0, st>>>(w.part_O, w.part_lse, w.own_O, w.own_lse, pr.topk,
+                                              pr.B, pr.G, pr.Hq, u0, nu, L,
+                                              reinterpret_cast<__nv_bfloat16*>(o), lse, pr.R);
+      MOBA_CUDA(cudaGetLastError());
+    }
+  }
+  return MOBA_OK;
+}
+
+moba_status forward_impl(const Problem& pr, const void* q, const void* k, const void* v, void* o,
+                         float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,
+                         cudaStream_t st) {
+  if (!q || !k || !v || !o || !lse) return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3) || (reinterpret_cast<uintptr_t>(sel_out) & 3))
+    return MOBA_ERR_INVALID_ARG;
+  if (!topk_supported(pr)) return MOBA_ERR_UNSUPPORTED;
+  // per-pass entry indices are int32
+  if ((int64_t)pr.T * pr.G * (pr.topk > 1 ? pr.topk - 1 : 1) >= INT32_MAX)
+    return MOBA_ERR_UNSUPPORTED;
+  const Ws need = carve(pr, 1, nullptr);
+  MOBA_TRY(check_ws(ws, ws_bytes, need.bytes));
+  if (pr.T == 0) return MOBA_OK;
+  int nu = 1;
+  while (nu < pr.Hkv && carve(pr, nu + 1, nullptr).bytes <= ws_bytes &&
+         (int64_t)(nu + 1) * pr.T * pr.G * (pr.topk > 1 ? pr.topk - 1 : 1) < INT32_MAX)
+    ++nu;
+  const Ws w = carve(pr, nu, static_cast<char*>(ws));
+  int32_t* sel = sel_out ? sel_out : w.sel;
+  MOBA_TRY(run_plan_pool(pr, k, w, st));
+  return pr.D == 128 ? forward_passes<128>(pr, q, k, v, o, lse, w, sel, nu, st)
+                     : forward_passes<64>(pr, q, k, v, o, lse, w, sel, nu, st);
+}
+
+size_t dense_ws_bytes(int64_t T, int nseq) {
+  Problem pr;
+  memset(&pr, 0, sizeof pr);
+  pr.nseq = nseq;
+  pr.T = 0;
+  pr.NBmax = T / kTileM + nseq;
+  pr.NQTmax = pr.NBmax;
+  pr.Hkv = 1;
+  pr.Hq = 1;
+  pr.G = 1;
+  pr.D = 64;
+  pr.topk = 1;
+  // status + plan arrays only: kbar/sel/partials are sized by T = 0 and Hkv = 1
+  return carve(pr, 1, nullptr).bytes + align_up(sizeof(float) * 64 * (size_t)pr.NBmax);
+}
+
+moba_status dense_impl(const Problem& pr, const void* q, const void* k, const void* v, void* o,
+                       float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (!q || !k || !v || !o || !lse) return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3))
+    return MOBA_ERR_INVALID_ARG;
+  MOBA_TRY(check_ws(ws, ws_bytes, dense_ws_bytes(pr.T, pr.nseq)));
+  if (pr.T == 0) return MOBA_OK;
+  // plan only needs status + plan arrays; carve them from a T = 0 view
+  Problem pv = pr;
+  pv.T = 0;
+  pv.Hkv = 1;
+  pv.Hq = 1;
+  pv.G = 1;
+  pv.D = 64;
+  pv.topk = 1;
+  const Ws w = carve(pv, 1, static_cast<char*>(ws));
+  SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
+  {
+    Timed tm(kKPlan, st);
+    plan_kernel<<<1, 1024, 0, st>>>(L, pr.B, w.P, (int)pr.NBmax, (int)pr.NQTmax, w.status);
+  }
+  MOBA_CUDA(cudaGetLastError());
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, pr.Hq, pr.T, pr.D) || !make_tmap(&tk, k, pr.Hkv, pr.T, pr.D) ||
+      !make_tmap(&tv, v, pr.Hkv, pr.T, pr.D))
+    return MOBA_ERR_CUDA;
+  AttnArgs a;
+  memset(&a, 0, sizeof a);
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.Hq = pr.Hq;
+  a.Hkv = pr.Hkv;
+  a.G = pr.G;
+  a.B = pr.B;
+  a.topk = 1;
+  a.scale_log2 = pr.scale * 1.4426950408889634f;
+  a.L = L;
+  a.P = w.P;
+  a.R = pr.R;
+  a.o = reinterpret_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.status = w.status;
+  a.u0 = 0;
+  a.nu = pr.Hkv;
+  return pr.D == 128 ? launch_attn<128, kDense>(tq, tk, tv, a, st)
+                     : launch_attn<64, kDense>(tq, tk, tv, a, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moba_workspace_size(const moba_params* p, int heads_per_pass) {
+  Problem pr;
+  if (make_problem(p, false, nullptr, 0, 0, true, &pr) != MOBA_OK) return 0;
+  int nu = (heads_per_pass <= 0 || heads_per_pass > pr.Hkv) ? pr.Hkv : heads_per_pass;
+  return carve(pr, nu, nullptr).bytes;
+}
+
+size_t moba_workspace_size_varlen(const moba_params* p, int64_t total_tokens, int num_seqs,
+                                  int heads_per_pass) {
+  Problem pr;
+  static const int32_t dummy = 0;
+  if (make_problem(p, true, &dummy, num_seqs, total_tokens, true, &pr) != MOBA_OK) return 0;
+  int nu = (heads_per_pass <= 0 || heads_per_pass > pr.Hkv) ? pr.Hkv : heads_per_pass;
+  return carve(pr, nu, nullptr).bytes;
+}
+
+moba_status moba_gate(const void* q, const void* k, int32_t* sel, const moba_params* p, void* ws,
+                      size_t ws_bytes, moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  return gate_impl(pr, q, k, sel, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moba_status moba_gate_varlen(const void* q, const void* k, const int32_t* cu_seqlens,
+                             int num_seqs, int64_t total_tokens, int32_t* sel,
+                             const moba_params* p, void* ws, size_t ws_bytes,
+                             moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, true, cu_seqlens, num_seqs, total_tokens, true, &pr));
+  return gate_impl(pr, q, k, sel, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moba_status moba_forward(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int32_t* sel_out, const moba_params* p, void* ws, size_t ws_bytes,
+                         moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  return forward_impl(pr, q, k, v, o, lse, sel_out, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+moba_status moba_forward_varlen(const void* q, const void* k, const void* v,
+                                const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens,
+                                void* o, float* lse, int32_t* sel_out, const moba_params* p,
+                                void* ws, size_t ws_bytes, moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, true, cu_seqlens, num_seqs, total_tokens, true, &pr));
+  return forward_impl(pr, q, k, v, o, lse, sel_out, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moba_full_causal_workspace_size(int64_t total_tokens, int num_seqs) {
+  if (total_tokens < 0 || num_seqs <= 0) return 0;
+  return dense_ws_bytes(total_tokens, num_seqs);
+}
+
+moba_status moba_full_causal(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const moba_params* p, void* ws, size_t ws_bytes,
+                             moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, false, nullptr, 0, 0, false, &pr));
+  return dense_impl(pr, q, k, v, o, lse, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moba_status moba_full_causal_varlen(const void* q, const void* k, const void* v,
+                                    const int32_t* cu_seqlens, int num_seqs,
+                                    int64_t total_tokens, void* o, float* lse,
+                                    const moba_params* p, void* ws, size_t ws_bytes,
+                                    moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, true, cu_seqlens, num_seqs, total_tokens, false, &pr));
+  return dense_impl(pr, q, k, v, o, lse, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moba_status moba_last_device_status(void* ws, moba_stream_t stream) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign)) return MOBA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, ws, sizeof word, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MOBA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOBA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof word, st) != cudaSuccess) return MOBA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOBA_ERR_CUDA;
+  if (word & MOBA_DEV_TIMEOUT) return MOBA_ERR_TIMEOUT;
+  if (word) return MOBA_ERR_DEVICE_CHECK;
+  return MOBA_OK;
+}
+
+const char* moba_status_string(moba_status s) {
+  switch (s) {
+    case MOBA_OK: return "MOBA_OK";
+    case MOBA_ERR_INVALID_ARG: return "MOBA_ERR_INVALID_ARG";
+    case MOBA_ERR_UNSUPPORTED: return "MOBA_ERR_UNSUPPORTED";
+    case MOBA_ERR_WORKSPACE: return "MOBA_ERR_WORKSPACE";
+    case MOBA_ERR_CUDA: return "MOBA_ERR_CUDA";
+    case MOBA_ERR_TIMEOUT: return "MOBA_ERR_TIMEOUT";
+    case MOBA_ERR_DEVICE_CHECK: return "MOBA_ERR_DEVICE_CHECK";
+  }
+  return "MOBA_ERR_UNKNOWN";
+}
+
+int moba_version(void) { return 100; }
+
+void moba_profile_enable(int on) { timer().on = (on != 0); }
+
+void moba_profile_reset(void) {
+  KernelTimer& t = timer();
+  for (auto& p : t.pending) {
+    cudaEventDestroy(p.a);
+    cudaEventDestroy(p.b);
+  }
+  t.pending.clear();
+  for (int c = 0; c < kKNum; ++c) {
+    t.launches[c] = 0;
+    t.ms[c] = 0.0;
+  }
+}
+
+int moba_profile_read(moba_kernel_time* out, int max_entries) {
+  KernelTimer& t = timer();
+  for (auto& p : t.pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(p.b) == cudaSuccess && cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
+      t.launches[p.cls] += 1;
+      t.ms[p.cls] += ms;
+    }
+    cudaEventDestroy(p.a);
+    cudaEventDestroy(p.b);
+  }
+  t.pending.clear();
+  int n = 0;
+  for (int c = 0; c < kKNum && n < max_entries; ++c) {
+    if (!out) break;
+    strncpy(out[n].name, kKernelNames[c], sizeof(out[n].name) - 1);
+    out[n].name[sizeof(out[n].name) - 1] = 0;
+    out[n].launches = t.launches[c];
+    out[n].total_ms = t.ms[c];
+    ++n;
+  }
+  return n;
+}
+
+}  // extern "C"

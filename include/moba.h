@@ -1,0 +1,154 @@
+/*
+ * moba.h -- C ABI of libmoba: the causal prefill forward of MoBA (Mixture of
+ * Block Attention) on one NVIDIA B200 (sm_100a).
+ *
+ * The operation (MoBA: Mixture of Block Attention for Long-Context LLMs):
+ *   - the keys of each sequence are split into contiguous blocks of B tokens,
+ *     the last block possibly short (wispaper.ai blog, "The Change", block
+ *     partition; sherconan.github.io step 1);
+ *   - each block is represented by the mean of its keys, and every query q
+ *     scores every block before its own as s_j = <q, mean(K_j)> (same
+ *     section, affinity equation; sherconan.github.io step 2);
+ *   - the query keeps its own block plus the k-1 past blocks of highest
+ *     score; future blocks are never chosen, ties go to the lower block
+ *     index, and when fewer than k blocks exist all of them are kept (same
+ *     section, routing and causality rules; sherconan.github.io steps 3-4);
+ *   - exact softmax attention with scale 1/sqrt(d) runs over the chosen
+ *     blocks only, causal inside the own block, and the per-block partial
+ *     results are combined by online softmax into O and its log-sum-exp
+ *     (wispaper.ai blog, "Efficiency and Implementation";
+ *     globaladvisors.biz, "Underlying computational mechanism").
+ *
+ * Tensor layouts (all row-major, contiguous, device memory):
+ *   batch calls : q, o  [batch][seqlen][num_q_heads][head_dim]  bf16
+ *                 k, v  [batch][seqlen][num_kv_heads][head_dim] bf16
+ *                 lse   [batch][num_q_heads][seqlen]            fp32 (natural log)
+ *                 sel   [batch][num_q_heads][seqlen][top_k]     int32
+ *   varlen calls: the same with the batch and seqlen axes replaced by the
+ *                 packed token axis T: q, o [T][Hq][d], k, v [T][Hkv][d],
+ *                 lse [Hq][T], sel [Hq][T][top_k]; sequence s covers tokens
+ *                 [cu_seqlens[s], cu_seqlens[s+1]) (int32, device, length
+ *                 num_seqs + 1, cu_seqlens[0] = 0, cu_seqlens[num_seqs] = T).
+ *   Query head h reads kv head h / (num_q_heads / num_kv_heads).
+ *   sel lists a row's chosen blocks (block ids within the sequence),
+ *   ascending, the own block last, -1 padded to top_k.
+ *
+ * Ownership: the caller owns every pointer, including the workspace; the
+ * library allocates no device memory.  Every call is asynchronous on
+ * `stream` (a cudaStream_t; NULL = legacy default stream).  The workspace
+ * must not be shared by calls that can run at the same time.
+ *
+ * Errors: invalid arguments are reported before anything is launched.
+ * Errors found on the device (a stuck pipeline wait, malformed cu_seqlens,
+ * an out-of-range selection) are latched in the workspace's status word and
+ * reported by moba_last_device_status().  Nothing crosses the ABI as an
+ * exception.
+ */
+#ifndef MOBA_H
+#define MOBA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moba_stream_t; /* same type as cudaStream_t */
+
+typedef enum moba_status {
+  MOBA_OK = 0,
+  MOBA_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad size or shape */
+  MOBA_ERR_UNSUPPORTED = 2,  /* head_dim not 64/128, block_size not a multiple of 128,
+                                top_k beyond 65, too many blocks per sequence */
+  MOBA_ERR_WORKSPACE = 3,    /* ws null, misaligned (256 B) or smaller than required */
+  MOBA_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, attribute, device) */
+  MOBA_ERR_TIMEOUT = 5,      /* device: a pipeline wait ran out of time */
+  MOBA_ERR_DEVICE_CHECK = 6  /* device: malformed cu_seqlens or selection, capacity */
+} moba_status;
+
+typedef struct moba_params {
+  int batch;           /* sequences in a batch call (ignored by varlen calls) */
+  int seqlen;          /* tokens per sequence in a batch call (ignored by varlen calls) */
+  int num_q_heads;     /* Hq */
+  int num_kv_heads;    /* Hkv, divides Hq */
+  int head_dim;        /* d: 64 or 128 */
+  int block_size;      /* B: multiple of 128 */
+  int top_k;           /* k >= 1, the own block included */
+  float softmax_scale; /* <= 0 selects 1/sqrt(head_dim) */
+} moba_params;
+
+/* Workspace bytes for moba_gate / moba_forward on a batch of
+ * params->batch sequences of params->seqlen tokens.  The forward processes
+ * the kv heads in passes; `heads_per_pass` (1..num_kv_heads, <= 0 = all)
+ * sets how many kv heads one pass holds, which is what the size grows with.
+ * moba_forward picks the largest pass the given workspace holds. */
+size_t moba_workspace_size(const moba_params *p, int heads_per_pass);
+
+/* The same for varlen calls over `total_tokens` tokens in `num_seqs`
+ * sequences (an upper bound covering any split of the tokens). */
+size_t moba_workspace_size_varlen(const moba_params *p, int64_t total_tokens, int num_seqs,
+                                  int heads_per_pass);
+
+/* Gate only: block means, scores, top-k; writes sel.  Follows the routing
+ * and causality rules cited above. */
+moba_status moba_gate(const void *q, const void *k, int32_t *sel, const moba_params *p,
+                      void *ws, size_t ws_bytes, moba_stream_t stream);
+moba_status moba_gate_varlen(const void *q, const void *k, const int32_t *cu_seqlens,
+                             int num_seqs, int64_t total_tokens, int32_t *sel,
+                             const moba_params *p, void *ws, size_t ws_bytes,
+                             moba_stream_t stream);
+
+/* Full MoBA prefill forward: o and lse; sel_out (nullable) receives the
+ * selection. */
+moba_status moba_forward(const void *q, const void *k, const void *v, void *o, float *lse,
+                         int32_t *sel_out, const moba_params *p, void *ws, size_t ws_bytes,
+                         moba_stream_t stream);
+moba_status moba_forward_varlen(const void *q, const void *k, const void *v,
+                                const int32_t *cu_seqlens, int num_seqs, int64_t total_tokens,
+                                void *o, float *lse, int32_t *sel_out, const moba_params *p,
+                                void *ws, size_t ws_bytes, moba_stream_t stream);
+
+/* Dense causal attention over every earlier token of each sequence: the
+ * k = n limit of the method (wispaper.ai blog, "The Change": k = n
+ * recovers full attention).  block_size and top_k are not used. */
+size_t moba_full_causal_workspace_size(int64_t total_tokens, int num_seqs);
+moba_status moba_full_causal(const void *q, const void *k, const void *v, void *o, float *lse,
+                             const moba_params *p, void *ws, size_t ws_bytes,
+                             moba_stream_t stream);
+moba_status moba_full_causal_varlen(const void *q, const void *k, const void *v,
+                                    const int32_t *cu_seqlens, int num_seqs,
+                                    int64_t total_tokens, void *o, float *lse,
+                                    const moba_params *p, void *ws, size_t ws_bytes,
+                                    moba_stream_t stream);
+
+/* Synchronises `stream`, returns and clears the device status latched in
+ * `ws` by earlier calls (MOBA_OK, MOBA_ERR_TIMEOUT or MOBA_ERR_DEVICE_CHECK). */
+moba_status moba_last_device_status(void *ws, moba_stream_t stream);
+
+/* Per-kernel timing, for benchmarks: while enabled, every kernel launch the
+ * library makes is bracketed by CUDA events recorded on the launch stream.
+ * moba_profile_read synchronises those events and returns, per kernel class
+ * (plan, pool, gate, bucket_scan, bucket_scatter, attn_routed, attn_own,
+ * merge, attn_dense), the launch count and summed device milliseconds since
+ * the last reset.  Returns the number of classes written (<= max_entries).
+ * Not thread safe; meant for one benchmarking thread. */
+typedef struct moba_kernel_time {
+  char name[24];
+  int launches;
+  double total_ms;
+} moba_kernel_time;
+void moba_profile_enable(int on);
+void moba_profile_reset(void);
+int moba_profile_read(moba_kernel_time *out, int max_entries);
+
+/* Static, human-readable name of a status code. */
+const char *moba_status_string(moba_status s);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int moba_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOBA_H */

@@ -18,7 +18,7 @@ def build(force: bool = False) -> str:
             and os.path.getmtime(LIB) >= os.path.getmtime(SRC)):
         return LIB
     tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+    cmd = ["gcc", "-O3", "-fopenmp", "-fPIC", "-shared", "-std=c11",
            "-Wall", "-Wextra", "-o", tmp, SRC, "-lm"]
     subprocess.check_call(cmd)
     os.replace(tmp, LIB)

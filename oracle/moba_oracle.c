@@ -207,13 +207,14 @@ int oracle_select(const uint16_t *Q, const double *Kbar, const int64_t *cu, int 
     {
         scored_block *buf = (scored_block *)malloc(sizeof(scored_block) * (size_t)(NB + 1));
         int32_t *tmp = (int32_t *)malloc(sizeof(int32_t) * (size_t)(k + 1));
-        if (!buf || !tmp) {
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!buf || !tmp || !qd) {
 #pragma omp atomic write
             err = ORC_ENOMEM;
         }
 #pragma omp for schedule(dynamic)
         for (int64_t rh = 0; rh < nrows * Hq; ++rh) {
-            if (!buf || !tmp)
+            if (!buf || !tmp || !qd)
                 continue;
             int64_t r = rh / Hq;
             int h = (int)(rh % Hq);
@@ -230,12 +231,14 @@ int oracle_select(const uint16_t *Q, const double *Kbar, const int64_t *cu, int 
             int64_t i = (t - cu[s]) / B; /* own block */
             int g = h / G;
             const uint16_t *qr = Q + ((size_t)t * Hq + h) * d;
+            for (int c = 0; c < d; ++c)
+                qd[c] = bf16_bits_to_double(qr[c]);
             double mx = 0.0;
             for (int64_t j = 0; j < i; ++j) {
                 const double *kb = Kbar + ((size_t)g * NB + first + j) * d;
                 double acc = 0.0;
                 for (int c = 0; c < d; ++c)
-                    acc += bf16_bits_to_double(qr[c]) * kb[c];
+                    acc += qd[c] * kb[c];
                 buf[j].s = acc;
                 buf[j].j = j;
                 if (fabs(acc) > mx)
@@ -266,6 +269,7 @@ int oracle_select(const uint16_t *Q, const double *Kbar, const int64_t *cu, int 
         }
         free(buf);
         free(tmp);
+        free(qd);
     }
     return err;
 }
@@ -296,6 +300,7 @@ int oracle_attend(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const
         size_t cap = 0;
         double *z = NULL;
         int64_t *idx = NULL;
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
 #pragma omp for schedule(dynamic)
         for (int64_t rh = 0; rh < nrows * Hq; ++rh) {
             int64_t r = rh / Hq;
@@ -318,7 +323,7 @@ int oracle_attend(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const
                 z = (double *)malloc(sizeof(double) * cap);
                 idx = (int64_t *)malloc(sizeof(int64_t) * cap);
             }
-            if (!z || !idx) {
+            if (!z || !idx || !qd) {
 #pragma omp atomic write
                 err = ORC_ENOMEM;
                 cap = 0;
@@ -347,13 +352,15 @@ int oracle_attend(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const
                 continue;
             }
             const uint16_t *qr = Q + ((size_t)t * Hq + h) * d;
+            for (int c = 0; c < d; ++c)
+                qd[c] = bf16_bits_to_double(qr[c]);
             int g = h / G;
             double zmax = -INFINITY;
             for (size_t u = 0; u < m; ++u) {
                 const uint16_t *kr = K + ((size_t)idx[u] * Hkv + g) * d;
                 double acc = 0.0;
                 for (int c = 0; c < d; ++c)
-                    acc += bf16_bits_to_double(qr[c]) * bf16_bits_to_double(kr[c]);
+                    acc += qd[c] * bf16_bits_to_double(kr[c]);
                 z[u] = acc * scale;
                 if (z[u] > zmax)
                     zmax = z[u];
@@ -378,6 +385,7 @@ int oracle_attend(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const
         }
         free(z);
         free(idx);
+        free(qd);
     }
     return err;
 }
@@ -400,6 +408,7 @@ int oracle_dense_causal(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
     {
         size_t cap = 0;
         double *z = NULL;
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
 #pragma omp for schedule(dynamic)
         for (int64_t rh = 0; rh < nrows * Hq; ++rh) {
             int64_t r = rh / Hq;
@@ -418,20 +427,22 @@ int oracle_dense_causal(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                 cap = m;
                 z = (double *)malloc(sizeof(double) * cap);
             }
-            if (!z) {
+            if (!z || !qd) {
 #pragma omp atomic write
                 err = ORC_ENOMEM;
                 cap = 0;
                 continue;
             }
             const uint16_t *qr = Q + ((size_t)t * Hq + h) * d;
+            for (int c = 0; c < d; ++c)
+                qd[c] = bf16_bits_to_double(qr[c]);
             int g = h / G;
             double zmax = -INFINITY;
             for (size_t u = 0; u < m; ++u) {
                 const uint16_t *kr = K + ((size_t)(a + u) * Hkv + g) * d;
                 double acc = 0.0;
                 for (int c = 0; c < d; ++c)
-                    acc += bf16_bits_to_double(qr[c]) * bf16_bits_to_double(kr[c]);
+                    acc += qd[c] * bf16_bits_to_double(kr[c]);
                 z[u] = acc * scale;
                 if (z[u] > zmax)
                     zmax = z[u];
@@ -453,6 +464,7 @@ int oracle_dense_causal(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
             lse[(size_t)r * Hq + h] = zmax + log(den);
         }
         free(z);
+        free(qd);
     }
     return err;
 }

@@ -1,0 +1,101 @@
+"""Comparison of the CUDA path's results with the fp64 oracle.
+
+Criteria (fixed by the task's parity bar):
+  * selection: bit-exact per (row, head), except rows whose oracle margin
+    between the last kept and the first dropped past score is below
+    1e-3 * max|s|; those are counted, and where the GPU chose differently the
+    oracle attention is recomputed with the GPU's own selection;
+  * O: max |err| <= 1e-2 and mean |err| <= 1e-3 (GPU bf16 vs oracle fp64);
+  * lse: max |err| <= 1e-3.
+"""
+import numpy as np
+import torch
+
+from oracle import Oracle, bf16_bits
+from oracle.oracle import bits_to_f64
+
+O_MAX_ABS = 1e-2
+O_MEAN_ABS = 1e-3
+LSE_MAX_ABS = 1e-3
+FLAG_REL = 1e-3
+
+
+def to_host_bits(t):
+    return bf16_bits(t)
+
+
+def check_selection_invariants(sel, own, k):
+    """sel [R, H, k] int32 numpy, own [R] own block: structural rules of the gate."""
+    R, H, K = sel.shape
+    assert K == k
+    cnt = np.minimum(k, own + 1)
+    valid = sel >= 0
+    assert np.all(valid.sum(axis=2) == cnt[:, None]), "wrong number of chosen blocks"
+    # valid entries first, ascending, unique; own block last
+    idx = np.arange(k)[None, None, :]
+    assert np.all(valid == (idx < cnt[:, None, None])), "padding not at the end"
+    last = np.take_along_axis(sel, (cnt - 1)[:, None, None].repeat(H, 1), axis=2)[..., 0]
+    assert np.all(last == own[:, None]), "own block not chosen"
+    d = np.diff(sel, axis=2)
+    inner = (idx[..., 1:] < cnt[:, None, None])
+    assert np.all(d[inner] > 0), "not strictly ascending"
+    assert np.all(sel[valid] >= 0) and np.all(sel.max(axis=2) <= own[:, None]), "future block"
+
+
+def compare(orc: Oracle, rows, gpu_O, gpu_lse, gpu_sel, label=""):
+    """gpu_O [R,H,d] float, gpu_lse [R,H], gpu_sel [R,H,k] or None.  Returns stats."""
+    O, lse, sel, margin, maxabs = orc.forward(rows)
+    stats = {"rows": int(len(rows)), "heads": int(orc.Hq)}
+    use_sel = sel
+    if gpu_sel is not None:
+        flagged = margin < FLAG_REL * maxabs
+        differ = np.any(gpu_sel != sel, axis=2)
+        bad = differ & ~flagged
+        stats["flagged"] = int(flagged.sum())
+        stats["flagged_and_differ"] = int((differ & flagged).sum())
+        assert not bad.any(), "%s: %d unflagged selection mismatches (first at %s)" % (
+            label, int(bad.sum()), np.argwhere(bad)[:3].tolist())
+        if (differ & flagged).any():
+            # re-check those rows against the oracle run on the GPU's own choice
+            O2, lse2, _ = orc.attend(rows, gpu_sel)
+            O = np.where(differ[..., None], O2, O)
+            lse = np.where(differ, lse2, lse)
+            use_sel = np.where(differ[..., None], gpu_sel, sel)
+    err = np.abs(gpu_O.astype(np.float64) - O)
+    lerr = np.abs(gpu_lse.astype(np.float64) - lse)
+    stats.update(o_max=float(err.max()), o_mean=float(err.mean()), lse_max=float(lerr.max()))
+    assert stats["o_max"] <= O_MAX_ABS, (label, stats)
+    assert stats["o_mean"] <= O_MEAN_ABS, (label, stats)
+    assert stats["lse_max"] <= LSE_MAX_ABS, (label, stats)
+    del use_sel
+    return stats
+
+
+def compare_dense(orc: Oracle, rows, gpu_O, gpu_lse, label=""):
+    O, lse = orc.dense(rows)
+    err = np.abs(gpu_O.astype(np.float64) - O)
+    lerr = np.abs(gpu_lse.astype(np.float64) - lse)
+    stats = dict(o_max=float(err.max()), o_mean=float(err.mean()), lse_max=float(lerr.max()))
+    assert stats["o_max"] <= O_MAX_ABS, (label, stats)
+    assert stats["o_mean"] <= O_MEAN_ABS, (label, stats)
+    assert stats["lse_max"] <= LSE_MAX_ABS, (label, stats)
+    return stats
+
+
+def gather_rows_packed(o, lse, sel, rows, Hq, varlen, N=None):
+    """Pull sampled rows out of GPU outputs.
+
+    batch layout: o [b,N,H,d], lse [b,H,N], sel [b,H,N,k]; varlen: o [T,H,d],
+    lse [H,T], sel [H,T,k].  rows are global token indices (b*N + t)."""
+    r = torch.as_tensor(rows, device=o.device, dtype=torch.long)
+    if varlen:
+        Og = o[r].float().cpu().numpy()
+        Lg = lse[:, r].t().contiguous().cpu().numpy()
+        Sg = sel[:, r, :].permute(1, 0, 2).contiguous().cpu().numpy() if sel is not None else None
+    else:
+        b = r // N
+        t = r % N
+        Og = o.view(-1, o.shape[2], o.shape[3])[r].float().cpu().numpy()
+        Lg = lse[b, :, t].cpu().numpy()
+        Sg = sel[b, :, t, :].cpu().numpy() if sel is not None else None
+    return Og, Lg, Sg

@@ -1,0 +1,221 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Small cases compare every row; the five benchmark workloads compare the
+seeded sample of query rows (all heads of each sampled row) in the launch
+configuration the benchmark uses (binding defaults: workspace picked by
+pick_heads_per_pass).  Tolerances and the flagged-row rule live in
+parity_util.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import synthetic as S
+from oracle import Oracle, bf16_bits, local_block_info
+from parity_util import (check_selection_invariants, compare, compare_dense,
+                         gather_rows_packed)
+
+pytestmark = pytest.mark.gpu
+
+PARITY_ROWS = int(os.environ.get("MOBA_PARITY_ROWS", "4096"))
+
+
+@pytest.fixture(scope="module")
+def moba():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from block_sparse_long_07_b200 import build
+    build.build()
+    import block_sparse_long_07_b200 as m
+    return m
+
+
+def _run_forward(m, w, q, k, v):
+    """Run the forward the way a user would; returns (o, lse, sel, ws)."""
+    dev = q.device
+    T = w.T
+    varlen = not w.batch_mode or len(set(w.lengths)) > 1
+    if varlen:
+        cu = torch.tensor(w.cu, dtype=torch.int32, device=dev)
+        p = m.make_params(1, 0, w.Hq, w.Hkv, w.d, w.B, w.k)
+        hp = m.pick_heads_per_pass(lambda n: m.workspace_size_varlen(p, T, len(w.lengths), n),
+                                   w.Hkv)
+        ws = m.alloc_workspace(m.workspace_size_varlen(p, T, len(w.lengths), hp), dev)
+        ws.zero_()
+        sel = torch.full((w.Hq, T, w.k), -7, dtype=torch.int32, device=dev)
+        o, lse = m.forward_varlen(q, k, v, cu, w.B, w.k, ws=ws, sel_out=sel)
+    else:
+        b, N = len(w.lengths), w.lengths[0]
+        q4, k4, v4 = (x.view(b, N, x.shape[1], x.shape[2]) for x in (q, k, v))
+        p = m.make_params(b, N, w.Hq, w.Hkv, w.d, w.B, w.k)
+        hp = m.pick_heads_per_pass(lambda n: m.workspace_size(p, n), w.Hkv)
+        ws = m.alloc_workspace(m.workspace_size(p, hp), dev)
+        ws.zero_()
+        sel = torch.full((b, w.Hq, N, w.k), -7, dtype=torch.int32, device=dev)
+        o, lse = m.forward(q4, k4, v4, w.B, w.k, ws=ws, sel_out=sel)
+    torch.cuda.synchronize()
+    assert m.last_device_status(ws) == 0
+    return o, lse, sel, varlen
+
+
+def _check_forward(m, w, rows=None, label=""):
+    q, k, v = S.make_qkv(w, "cuda")
+    o, lse, sel, varlen = _run_forward(m, w, q, k, v)
+    orc = Oracle(bf16_bits(q), bf16_bits(k), bf16_bits(v), w.cu, w.Hq, w.Hkv, w.d, w.B, w.k)
+    if rows is None:
+        rows = np.arange(w.T, dtype=np.int64)
+    N = None if varlen else w.lengths[0]
+    Og, Lg, Sg = gather_rows_packed(o, lse, sel, rows, w.Hq, varlen, N)
+    _, _, own = local_block_info(w.cu, rows, w.B)
+    check_selection_invariants(Sg, own, w.k)
+    stats = compare(orc, rows, Og, Lg, Sg, label=label or w.name)
+    return stats
+
+
+SMALL = [
+    # lengths, Hq, Hkv, d, B, k
+    ([2048], 1, 1, 64, 256, 3),
+    ([1000], 4, 1, 128, 128, 3),      # ragged N, GQA 4
+    ([777], 8, 1, 64, 256, 2),        # GQA 8, d = 64, partial last block
+    ([1536], 2, 2, 128, 512, 2),      # B = 512
+    ([640], 4, 2, 128, 128, 1),       # k = 1: own block only
+    ([900], 4, 2, 128, 128, 20),      # k > n: every block
+    ([1280, 1280], 4, 2, 128, 256, 3),  # batch of 2
+    ([129], 2, 1, 128, 128, 2),       # one row past the first block
+    ([4096], 8, 2, 128, 128, 5),      # many blocks, top-k ranking
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "x".join(map(str, c[0])) + "_%d_%d_%d_%d_%d" % c[1:])
+def test_forward_small(moba, case):
+    lengths, Hq, Hkv, d, B, k = case
+    w = S.Workload("small", lengths, Hq, Hkv, d, B, k, seed=101)
+    _check_forward(moba, w)
+
+
+VARLEN_SMALL = [
+    ([300, 1, 1024, 129, 640], 4, 2, 128, 128, 3),
+    ([0, 513, 0, 1], 2, 1, 64, 256, 2),   # empty and one-token sequences
+    ([2000, 700, 1500], 8, 2, 128, 256, 4),
+]
+
+
+@pytest.mark.parametrize("case", VARLEN_SMALL, ids=lambda c: "v" + "_".join(map(str, c[0])))
+def test_forward_varlen_small(moba, case):
+    lengths, Hq, Hkv, d, B, k = case
+    w = S.Workload("varlen_small", lengths, Hq, Hkv, d, B, k, seed=202, batch_mode=False)
+    _check_forward(moba, w)
+
+
+DENSE_SMALL = [
+    ([1], 1, 1, 64), ([127], 2, 1, 128), ([128], 1, 1, 128), ([300], 4, 2, 128),
+    ([2000], 8, 2, 64), ([700, 700], 4, 1, 128),
+]
+
+
+@pytest.mark.parametrize("case", DENSE_SMALL, ids=lambda c: "d" + "_".join(map(str, c[0])) + "_%d_%d_%d" % c[1:])
+def test_full_causal_small(moba, case):
+    lengths, Hq, Hkv, d = case
+    w = S.Workload("dense_small", lengths, Hq, Hkv, d, 128, 1, seed=303)
+    q, k, v = S.make_qkv(w, "cuda")
+    b, N = len(lengths), lengths[0]
+    o, lse = moba.full_causal(*(x.view(b, N, x.shape[1], x.shape[2]) for x in (q, k, v)))
+    torch.cuda.synchronize()
+    orc = Oracle(bf16_bits(q), bf16_bits(k), bf16_bits(v), w.cu, Hq, Hkv, d, 128, 1)
+    rows = np.arange(w.T)
+    Og, Lg, _ = gather_rows_packed(o, lse, None, rows, Hq, False, N)
+    compare_dense(orc, rows, Og, Lg, label=str(case))
+
+
+def test_full_causal_varlen_small(moba):
+    w = S.Workload("dense_varlen", [5, 300, 1000, 0, 17], 4, 2, 128, 128, 1, seed=304,
+                   batch_mode=False)
+    q, k, v = S.make_qkv(w, "cuda")
+    cu = torch.tensor(w.cu, dtype=torch.int32, device="cuda")
+    o, lse = moba.full_causal_varlen(q, k, v, cu)
+    torch.cuda.synchronize()
+    orc = Oracle(bf16_bits(q), bf16_bits(k), bf16_bits(v), w.cu, 4, 2, 128, 128, 1)
+    rows = np.arange(w.T)
+    Og, Lg, _ = gather_rows_packed(o, lse, None, rows, 4, True)
+    compare_dense(orc, rows, Og, Lg, label="dense varlen")
+
+
+def test_k_equal_n_matches_full_causal_kernel(moba):
+    # the method with every block selected is full attention: both CUDA paths agree
+    w = S.Workload("kn", [2048], 8, 2, 128, 256, 8, seed=404)
+    q, k, v = S.make_qkv(w, "cuda")
+    q4, k4, v4 = (x.view(1, 2048, x.shape[1], 128) for x in (q, k, v))
+    o1, l1 = moba.forward(q4, k4, v4, 256, 8)
+    o2, l2 = moba.full_causal(q4, k4, v4)
+    torch.cuda.synchronize()
+    assert (o1.float() - o2.float()).abs().max().item() <= 1e-2
+    assert (l1 - l2).abs().max().item() <= 1e-3
+
+
+def test_heads_per_pass_does_not_change_results(moba):
+    w = S.Workload("passes", [3000], 8, 4, 128, 256, 4, seed=505)
+    q, k, v = S.make_qkv(w, "cuda")
+    q4, k4, v4 = (x.view(1, 3000, x.shape[1], 128) for x in (q, k, v))
+    p = moba.make_params(1, 3000, 8, 4, 128, 256, 4)
+    outs = []
+    for hp in (1, 3, 4):
+        ws = moba.alloc_workspace(moba.workspace_size(p, hp))
+        outs.append(moba.forward(q4, k4, v4, 256, 4, ws=ws))
+    torch.cuda.synchronize()
+    for o, l in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(l, outs[0][1])
+
+
+def test_deterministic(moba):
+    w = S.Workload("det", [4096], 8, 2, 128, 256, 4, seed=606)
+    q, k, v = S.make_qkv(w, "cuda")
+    q4, k4, v4 = (x.view(1, 4096, x.shape[1], 128) for x in (q, k, v))
+    a = moba.forward(q4, k4, v4, 256, 4)
+    b = moba.forward(q4, k4, v4, 256, 4)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_gate_only_matches_forward_selection(moba):
+    w = S.Workload("gate", [4096], 8, 2, 128, 256, 5, seed=707)
+    q, k, v = S.make_qkv(w, "cuda")
+    q4, k4, v4 = (x.view(1, 4096, x.shape[1], 128) for x in (q, k, v))
+    sel_f = torch.empty(1, 8, 4096, 5, dtype=torch.int32, device="cuda")
+    moba.forward(q4, k4, v4, 256, 5, sel_out=sel_f)
+    sel_g = moba.gate(q4, k4, 256, 5)
+    torch.cuda.synchronize()
+    assert torch.equal(sel_f, sel_g)
+
+
+# ---------------------------------------------------------------- workloads
+def test_workload_tiny_all_rows(moba):
+    stats = _check_forward(moba, S.TINY)
+    print("tiny", stats)
+
+
+@pytest.mark.slow
+@pytest.mark.timeout(3600)
+@pytest.mark.parametrize("name", ["fine_32k", "long_128k", "long_128k_k32", "varlen_8seq",
+                                  "prefill_1m"])
+def test_workload_sampled_rows(moba, name):
+    w = S.LONG_128K.with_k(32) if name == "long_128k_k32" else S.WORKLOADS[name]
+    rows = S.sample_rows(w, PARITY_ROWS)
+    stats = _check_forward(moba, w, rows=rows, label=name)
+    print(name, stats)
+
+
+@pytest.mark.slow
+@pytest.mark.timeout(3600)
+@pytest.mark.parametrize("name", ["fine_32k", "long_128k"])
+def test_workload_dense_sampled_rows(moba, name):
+    w = S.WORKLOADS[name]
+    q, k, v = S.make_qkv(w, "cuda")
+    N = w.lengths[0]
+    o, lse = moba.full_causal(*(x.view(1, N, x.shape[1], x.shape[2]) for x in (q, k, v)))
+    torch.cuda.synchronize()
+    orc = Oracle(bf16_bits(q), bf16_bits(k), bf16_bits(v), w.cu, w.Hq, w.Hkv, w.d, w.B, w.k)
+    rows = S.sample_rows(w, 256, seed=99)
+    Og, Lg, _ = gather_rows_packed(o, lse, None, rows, w.Hq, False, N)
+    print(name, compare_dense(orc, rows, Og, Lg, label=name))
