@@ -33,11 +33,12 @@ def check_selection_invariants(sel, own, k):
     assert np.all(valid.sum(axis=2) == cnt[:, None]), "wrong number of chosen blocks"
     # valid entries first, ascending, unique; own block last
     idx = np.arange(k)[None, None, :]
-    assert np.all(valid == (idx < cnt[:, None, None])), "padding not at the end"
+    assert np.all(valid == np.broadcast_to(idx < cnt[:, None, None], sel.shape)), \
+        "padding not at the end"
     last = np.take_along_axis(sel, (cnt - 1)[:, None, None].repeat(H, 1), axis=2)[..., 0]
     assert np.all(last == own[:, None]), "own block not chosen"
     d = np.diff(sel, axis=2)
-    inner = (idx[..., 1:] < cnt[:, None, None])
+    inner = np.broadcast_to(idx[..., 1:] < cnt[:, None, None], d.shape)
     assert np.all(d[inner] > 0), "not strictly ascending"
     assert np.all(sel[valid] >= 0) and np.all(sel.max(axis=2) <= own[:, None]), "future block"
 
