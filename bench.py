@@ -251,7 +251,9 @@ def run_moba(args, w):
         q, k, v = (x.view(b, N, x.shape[1], x.shape[2]) for x in (q, k, v))
         p = moba.make_params(b, N, w.Hq, w.Hkv, w.d, w.B, w.k)
         size_fn = lambda n: moba.workspace_size(p, n)
-    hp = moba.pick_heads_per_pass(size_fn, w.Hkv)
+    budget = (moba.DEFAULT_WS_BUDGET if args.ws_budget_gb is None
+              else int(args.ws_budget_gb * (1 << 30)))
+    hp = moba.pick_heads_per_pass(size_fn, w.Hkv, budget)
     ws = moba.alloc_workspace(size_fn(hp), dev)
     o = torch.empty_like(q)
     lse = torch.empty((w.Hq, T) if varlen else (len(w.lengths), w.Hq, w.lengths[0]),
@@ -426,6 +428,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ws-budget-gb", type=float, default=None,
+                    help="workspace budget (default: the binding's, 32 GiB)")
     ap.add_argument("--ref-step-seconds", type=float, default=20.0)
     args = ap.parse_args()
     import synthetic as S
