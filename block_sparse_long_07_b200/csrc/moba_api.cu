@@ -685,3 +685,97 @@ int moba_profile_read(moba_kernel_time* out, int max_entries) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free gate.
+//
+// Some callers cannot hand this library a workspace: code embedded in a host
+// framework that owns every device allocation and exposes no allocator to
+// its plugins, or a latency-critical loop that must never call cudaMalloc
+// (which can synchronise the device).  moba_gate_noalloc serves them: the
+// gate's scratch (status word, block numbering, block means) lives in one
+// file-scope device array of fixed size, so the call allocates nothing.
+//
+// Limits and sharing rules:
+//   * the array holds kGateScratchBytes (16 MiB); a shape whose scratch is
+//     larger is refused with MOBA_ERR_WORKSPACE before anything is launched;
+//   * every GPU that loads the library holds its own copy until exit;
+//   * every call on a device uses the same array and leaves its contents
+//     behind, so calls that can overlap on the GPU (other streams, other
+//     threads) race; the caller must order them;
+//   * the first call on each device looks up the array's device address
+//     (cudaGetSymbolAddress) with that device current; make that first call
+//     before any stream capture.
+namespace {
+
+constexpr size_t kGateScratchBytes = size_t(16) << 20;
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_gate_scratch[kGateScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_gate_scratch_mu;
+void* g_gate_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_gate_scratch on the current device (looked up once).
+moba_status gate_scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOBA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOBA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_gate_scratch_mu);
+  if (!g_gate_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_gate_scratch) != cudaSuccess || !p) return MOBA_ERR_CUDA;
+    g_gate_scratch_addr[dev] = p;
+  }
+  *out = g_gate_scratch_addr[dev];
+  return MOBA_OK;
+}
+
+// Gate-only scratch layout (status word, plan arrays, block means).
+Ws carve_gate_scratch(const Problem& pr, char* base) {
+  Ws w;
+  memset(&w, 0, sizeof w);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + bytes);
+    return p;
+  };
+  const int64_t NB = pr.NBmax;
+  w.status = reinterpret_cast<uint32_t*>(take(kAlign));
+  w.P.totals = reinterpret_cast<int32_t*>(take(4 * sizeof(int32_t)));
+  w.P.blk_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (pr.nseq + 1)));
+  w.P.qt_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (pr.nseq + 1)));
+  w.P.blk_tok = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * NB));
+  w.P.blk_len = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * NB));
+  w.kbar = reinterpret_cast<float*>(take(sizeof(float) * (size_t)pr.Hkv * NB * pr.D));
+  w.bytes = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" moba_status moba_gate_noalloc(const void* q, const void* k, int32_t* sel,
+                                         const moba_params* p, moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  if (!q || !k || !sel || !aligned16(q) || !aligned16(k) ||
+      (reinterpret_cast<uintptr_t>(sel) & 3))
+    return MOBA_ERR_INVALID_ARG;
+  if (!topk_supported(pr)) return MOBA_ERR_UNSUPPORTED;
+  if (carve_gate_scratch(pr, nullptr).bytes > kGateScratchBytes) return MOBA_ERR_WORKSPACE;
+  if (pr.T == 0) return MOBA_OK;
+  void* base = nullptr;
+  MOBA_TRY(gate_scratch_address(&base));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Ws w = carve_gate_scratch(pr, static_cast<char*>(base));
+  // the status word is the only state a call reads before writing it
+  MOBA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st));
+  MOBA_TRY(run_plan_pool(pr, k, w, st));
+  return pr.D == 128 ? launch_gate<128>(pr, q, w, sel, nullptr, st)
+                     : launch_gate<64>(pr, q, w, sel, nullptr, st);
+}

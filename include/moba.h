@@ -99,6 +99,24 @@ moba_status moba_gate_varlen(const void *q, const void *k, const int32_t *cu_seq
                              const moba_params *p, void *ws, size_t ws_bytes,
                              moba_stream_t stream);
 
+/* Allocation-free variant of moba_gate (batch layout only).  The method
+ * described in the pages has no counterpart to this call: it exists for
+ * callers that cannot allocate device memory or pass a workspace, such as
+ * code inside a host framework that owns every device allocation, or a
+ * latency-critical loop that must not call cudaMalloc.  Its scratch is one
+ * fixed 16 MiB device array inside the library, so:
+ *   - a shape whose gate scratch (block means: 4 * num_kv_heads *
+ *     ceil(seqlen / block_size) * batch * head_dim bytes, plus a few KB)
+ *     exceeds 16 MiB returns MOBA_ERR_WORKSPACE and launches nothing;
+ *   - every GPU that loads the library keeps that array until exit;
+ *   - all calls on a device share it and leave their data in it: calls that
+ *     can overlap on the GPU race, and the caller must order them;
+ *   - the first call on a device looks up the array's address with that
+ *     device current; make that first call before any stream capture.
+ * Results equal moba_gate's for the same inputs. */
+moba_status moba_gate_noalloc(const void *q, const void *k, int32_t *sel, const moba_params *p,
+                              moba_stream_t stream);
+
 /* Full MoBA prefill forward: o and lse; sel_out (nullable) receives the
  * selection. */
 moba_status moba_forward(const void *q, const void *k, const void *v, void *o, float *lse,
