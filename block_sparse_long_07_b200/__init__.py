@@ -26,14 +26,15 @@ EXPORTS = ("moba_workspace_size", "moba_workspace_size_varlen", "moba_gate", "mo
            "moba_gate_noalloc",
            "moba_forward", "moba_forward_varlen", "moba_full_causal_workspace_size",
            "moba_full_causal", "moba_full_causal_varlen", "moba_last_device_status",
-           "moba_status_string", "moba_version", "moba_profile_enable", "moba_profile_reset",
+           "moba_status_string", "moba_version", "moba_last_error_string", "moba_profile_enable", "moba_profile_reset",
            "moba_profile_read")
 
 
 class MobaError(RuntimeError):
-    def __init__(self, code, what):
+    def __init__(self, code, what, detail=""):
         self.code = code
-        super().__init__("%s failed: %s" % (what, _STATUS.get(code, str(code))))
+        msg = "%s failed: %s" % (what, _STATUS.get(code, str(code)))
+        super().__init__(msg + (" (%s)" % detail if detail else ""))
 
 
 class MobaParams(ctypes.Structure):
@@ -88,6 +89,8 @@ def load_library(path=None):
     lib.moba_status_string.argtypes = [i32]
     lib.moba_version.restype = i32
     lib.moba_version.argtypes = []
+    lib.moba_last_error_string.restype = ctypes.c_char_p
+    lib.moba_last_error_string.argtypes = []
     lib.moba_profile_enable.restype = None
     lib.moba_profile_enable.argtypes = [i32]
     lib.moba_profile_reset.restype = None
@@ -106,7 +109,10 @@ def _torch():
 
 def _check(code, what):
     if code != MOBA_OK:
-        raise MobaError(code, what)
+        detail = ""
+        if code == 4:
+            detail = load_library().moba_last_error_string().decode()
+        raise MobaError(code, what, detail)
 
 
 def _ptr(t):

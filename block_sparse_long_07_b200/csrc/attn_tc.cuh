@@ -402,22 +402,33 @@ __global__ void __launch_bounds__(224, 1)
           for (int c = 0; c < kTileN; ++c)
             if (c > lim) s[c] = -INFINITY;
         }
-        float mx = s[0];
+        // row max: 8 independent chains of 3-input max, then a short tree
+        float mp[8];
 #pragma unroll
-        for (int c = 1; c < kTileN; ++c) mx = fmaxf(mx, s[c]);
+        for (int e = 0; e < 8; ++e) mp[e] = fmaxf(s[e], s[e + 8]);
+#pragma unroll
+        for (int c = 16; c < kTileN; c += 16) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mp[e] = fmax3f(mp[e], s[c + e], s[c + 8 + e]);
+        }
+        const float mx = fmaxf(fmax3f(mp[0], mp[1], mp[2]),
+                               fmax3f(fmax3f(mp[3], mp[4], mp[5]), mp[6], mp[7]));
         const float m_new = fmaxf(m_run, mx * a.scale_log2);
         const bool need = (j == 0) || (m_new > m_run + 8.0f);
         const float m_use = need ? m_new : m_run;
         const float alpha = (j == 0) ? 0.f : (need ? ex2_approx(m_run - m_use) : 1.f);
         uint32_t pk[kTileN / 2];
-        float sum = 0.f;
+        float sp[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sp[e] = 0.f;
 #pragma unroll
         for (int c = 0; c < kTileN; c += 2) {
           const float p0 = ex2_approx(fmaf(s[c], a.scale_log2, -m_use));
           const float p1 = ex2_approx(fmaf(s[c + 1], a.scale_log2, -m_use));
-          sum += p0 + p1;
+          sp[(c / 2) & 7] += p0 + p1;
           pk[c / 2] = pack_bf16x2(p0, p1);
         }
+        const float sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
         // previous PV done: P buffer free, O stable
         if (n > 0) {
           ok = mbar_wait(pv_done, (n - 1) & 1, abort_flag, st);

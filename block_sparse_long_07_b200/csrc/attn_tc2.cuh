@@ -1,0 +1,609 @@
+// attn_tc2.cuh -- exact softmax attention on the sm_100a tensor cores for the
+// MoBA prefill forward, two query sub-tiles per CTA.
+//
+// Modes (MoBA: Mixture of Block Attention, wispaper.ai blog, "Efficiency and
+// Implementation": current-block attention plus attention over the routed
+// historical blocks, combined by online softmax):
+//   kRouted : up to 256 gathered (token, q-head) rows that chose the same past
+//             block J, against the B keys of J, no mask.  Each row writes a
+//             normalised partial O (bf16) and its log2-domain lse to its slot.
+//   kOwn    : two consecutive 128-row query tiles of one head against their
+//             own block up to the diagonal, causal mask on the diagonal tile
+//             (wispaper.ai blog, "The Change": the current block is always
+//             attended, causally).  Rows whose selection is the own block
+//             alone write the final O / lse; the others an fp32 partial.
+//   kDense  : two consecutive 128-row tiles against every earlier key of the
+//             sequence: full causal attention, the k = n limit.
+//
+// Work item = two 128-row sub-tiles (X = 0, 1) sharing one stream of 128-key
+// K/V tiles; sub-tile X uses the first nkv[X] of them.  CTA = 11 warps:
+//   warps 0-3   softmax + epilogue of sub-tile 0 (thread r = row r = TMEM lane r)
+//   warps 4-7   softmax + epilogue of sub-tile 1
+//   warp  8     TMA producer: Q tiles (own/dense) and the K/V ring
+//   warp  9     TMEM allocation and the single-thread MMA issuer
+//   warp 10     Q row gather for routed items (cp.async into swizzled smem)
+// TMEM (512 columns): S_X at 128*X (fp32 scores; after the softmax the first
+// 64 columns hold P_X as packed bf16), O_X at 256 + D*X.
+// Per KV tile j and sub-tile X: S_X = Q_X K_j^T (both operands in shared
+// memory); the softmax reads S_X, keeps a running max / sum, writes P_X back
+// into TMEM; O_X += P_X V_j takes P_X straight from TMEM, so P never touches
+// shared memory.  The MMA thread alternates the sub-tiles, so one softmax
+// warpgroup works while the tensor core runs the other sub-tile's MMAs.
+// Tensor-core operations issued by one thread complete in issue order: when
+// S_X(j) is complete, PV_X(j-1) (issued before it) is too, which is what lets
+// the softmax rescale O_X right after seeing S_X(j).  The max is rescaled
+// lazily (only when it grows by more than 2^8).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "layout.cuh"
+
+namespace moba {
+
+enum AttnMode : int { kRouted = 0, kOwn = 1, kDense = 2 };
+
+struct AttnArgs {
+  const __nv_bfloat16* q;  // [T][Hq][D] (routed gather)
+  int Hq, Hkv, G, B, topk;
+  float scale_log2;        // softmax scale * log2(e)
+  SeqLayout L;
+  Plan P;
+  RowLayout R;             // lse row layout of the final outputs
+  int u0, nu;              // pass: kv heads u0 .. u0+nu-1
+  const int32_t* tile_off;   // routed: [nu*NB + 1] work items per bucket, prefix
+  const int32_t* entry_off;  // routed: [nu*NB + 1] bucket entries, prefix
+  const uint2* entries;
+  __nv_bfloat16* part_O;     // [nu][T][G][topk-1][D]
+  float* part_lse;           // [nu][T][G][topk-1]
+  float* own_O;              // [nu][T][G][D]
+  float* own_lse;            // [nu][T][G]
+  __nv_bfloat16* o;          // [T][Hq][D]
+  float* lse;
+  uint32_t* status;
+};
+
+template <int D>
+struct Attn2Cfg {
+  static constexpr int kStages = (D == 128) ? 3 : 4;
+  static constexpr int kHalfBytes = kTileM * 128;          // 128 rows x 64 columns bf16
+  static constexpr int kSubQBytes = kTileM * D * 2;        // one 128-row Q sub-tile
+  static constexpr int kQBytes = 2 * kSubQBytes;           // one work item's Q
+  static constexpr int kKVBytes = kTileN * D * 2;
+  static constexpr int kOffQ = 0;                          // two Q buffers
+  static constexpr int kOffKV = kOffQ + 2 * kQBytes;
+  static constexpr int kOffBar = kOffKV + kStages * kKVBytes;
+  static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 1;
+  static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false, false);
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, false, true);
+  static constexpr int kThreads = 352;
+  static __host__ __device__ constexpr uint32_t col_s(int x) { return 128u * x; }
+  static __host__ __device__ constexpr uint32_t col_o(int x) { return 256u + D * x; }
+};
+
+struct Item {
+  int g;              // kv head
+  int h;              // q head (own/dense)
+  int u;              // unit (kv head) within the pass
+  int64_t kstart;     // first key of KV tile 0
+  int nkv;            // KV tiles streamed (max over sub-tiles)
+  int nkv_x[2];       // KV tiles each sub-tile uses (0 = sub-tile idle)
+  int rows_x[2];      // valid rows of each sub-tile
+  int64_t qstart;     // own/dense: first query token of sub-tile 0
+  int seq;
+  int64_t seq_start;
+  int own_block;      // own/dense: block index of the tiles within the sequence
+  int64_t e0;         // routed: first entry of sub-tile 0
+};
+
+template <int MODE>
+__device__ __forceinline__ int64_t num_items2(const AttnArgs& a, int pair_own) {
+  if (MODE == kRouted) return a.tile_off[a.nu * a.P.totals[0]];
+  const int64_t HP = (MODE == kOwn) ? (int64_t)a.nu * a.G : a.Hq;
+  // items per head: query-tile pairs (or single tiles when own tiles cannot pair)
+  const int64_t tiles = a.P.totals[1];
+  const int64_t per_head = (MODE == kOwn && !pair_own) ? tiles : a.P.totals[2];
+  return per_head * HP;
+}
+
+// Work item w of the launch.  For own/dense modes the items of one head are
+// query-tile pairs numbered through P.totals[2] / P.pair_off (see plan).
+template <int MODE>
+__device__ __forceinline__ Item item_info(const AttnArgs& a, int64_t w, int pair_own) {
+  Item it;
+  if (MODE == kRouted) {
+    const int NB = a.P.totals[0];
+    const int M = a.nu * NB;
+    const int f = upper_index(a.tile_off, M + 1, w);
+    const int u = f / NB, J = f % NB;
+    const int64_t row0 = (w - a.tile_off[f]) * (int64_t)(2 * kTileM);
+    const int64_t cnt = (int64_t)a.entry_off[f + 1] - a.entry_off[f];
+    const int64_t left = cnt - row0;
+    it.u = u;
+    it.g = a.u0 + u;
+    it.h = -1;
+    it.kstart = a.P.blk_tok[J];
+    it.nkv = a.B / kTileN;
+    it.rows_x[0] = (int)min((int64_t)kTileM, left);
+    it.rows_x[1] = (int)max((int64_t)0, min((int64_t)kTileM, left - kTileM));
+    it.nkv_x[0] = it.nkv;
+    it.nkv_x[1] = it.rows_x[1] > 0 ? it.nkv : 0;
+    it.qstart = 0;
+    it.seq = 0;
+    it.seq_start = 0;
+    it.own_block = 0;
+    it.e0 = a.entry_off[f] + row0;
+  } else {
+    const int HP = (MODE == kOwn) ? a.nu * a.G : a.Hq;
+    const bool paired = (MODE == kDense) || pair_own;
+    const int64_t per_head = paired ? a.P.totals[2] : a.P.totals[1];
+    int64_t idx = w / HP;
+    const int hl = (int)(w % HP);
+    if (MODE == kDense) idx = per_head - 1 - idx;  // longest rows first
+    int s;
+    int64_t p0;
+    if (paired) {
+      s = upper_index(a.P.pair_off, a.L.nseq + 1, idx);
+      p0 = (idx - a.P.pair_off[s]) * (int64_t)(2 * kTileM);
+    } else {
+      s = upper_index(a.P.qt_off, a.L.nseq + 1, idx);
+      p0 = (idx - a.P.qt_off[s]) * (int64_t)kTileM;
+    }
+    const int64_t st = seq_start(a.L, s), len = seq_len(a.L, s);
+    it.h = (MODE == kOwn) ? a.u0 * a.G + hl : hl;
+    it.g = it.h / a.G;
+    it.u = (MODE == kOwn) ? hl / a.G : 0;
+    it.seq = s;
+    it.seq_start = st;
+    it.qstart = st + p0;
+    it.own_block = (int)(p0 / a.B);
+    const int64_t k0 = (MODE == kOwn) ? (int64_t)it.own_block * a.B : 0;
+    it.kstart = st + k0;
+    it.rows_x[0] = (int)min((int64_t)kTileM, len - p0);
+    it.rows_x[1] = paired ? (int)max((int64_t)0, min((int64_t)kTileM, len - p0 - kTileM)) : 0;
+    it.nkv_x[0] = (int)((p0 - k0) / kTileN) + 1;
+    it.nkv_x[1] = it.rows_x[1] > 0 ? it.nkv_x[0] + 1 : 0;
+    it.nkv = max(it.nkv_x[0], it.nkv_x[1]);
+    it.e0 = 0;
+  }
+  return it;
+}
+
+// Row max of one 128-key score tile held in TMEM (this thread's lane),
+// read 64 columns at a time.  MASK hides keys c > r (diagonal tile).
+template <bool MASK>
+__device__ __forceinline__ float tile_row_max(uint32_t tS, int r) {
+  float mp[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mp[e] = -INFINITY;
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    float sv[64];
+    tmem_ld32(tS + h2 * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+    tmem_ld32(tS + h2 * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+    tc_wait_ld();
+    if (MASK) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c)
+        if (h2 * 64 + c > r) sv[c] = -INFINITY;
+    }
+#pragma unroll
+    for (int c = 0; c < 64; c += 16) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mp[e] = fmax3f(mp[e], sv[c + e], sv[c + 8 + e]);
+    }
+  }
+  return fmaxf(fmax3f(mp[0], mp[1], mp[2]), fmax3f(fmax3f(mp[3], mp[4], mp[5]), mp[6], mp[7]));
+}
+
+// P = 2^(s * scale_log2 - m) for one score tile, written back as packed bf16
+// pairs into the tile's first 64 TMEM columns (chunk h2 of 64 scores becomes
+// 32 packed columns, which never overlap scores still to be read).  Returns
+// the row sum of the fp32 probabilities.
+template <bool MASK>
+__device__ __forceinline__ float tile_exp_to_p(uint32_t tS, int r, float scale_log2,
+                                               float m_use) {
+  float sp[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) sp[e] = 0.f;
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    float sv[64];
+    tmem_ld32(tS + h2 * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+    tmem_ld32(tS + h2 * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+    tc_wait_ld();
+    if (MASK) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c)
+        if (h2 * 64 + c > r) sv[c] = -INFINITY;
+    }
+#pragma unroll
+    for (int q2 = 0; q2 < 2; ++q2) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float p0 = ex2_approx(fmaf(sv[q2 * 32 + 2 * e], scale_log2, -m_use));
+        const float p1 = ex2_approx(fmaf(sv[q2 * 32 + 2 * e + 1], scale_log2, -m_use));
+        sp[e & 7] += p0 + p1;
+        pk[e] = pack_bf16x2(p0, p1);
+      }
+      tmem_st16(tS + h2 * 32 + q2 * 16, pk);
+    }
+  }
+  return ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+}
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(352, 1)
+    attn2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const AttnArgs a, int pair_own) {
+  using C = Attn2Cfg<D>;
+  constexpr int ST = C::kStages;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sQ = smem + C::kOffQ;
+  unsigned char* sKV = smem + C::kOffKV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* q_full = bars + 0;          // [2] Q buffer loaded
+  uint64_t* q_empty = bars + 2;         // [2] Q buffer free (last S MMAs done)
+  uint64_t* kv_full = bars + 4;         // [ST]
+  uint64_t* kv_empty = kv_full + ST;    // [ST]
+  uint64_t* s_full = kv_empty + ST;     // [2] S_X written
+  uint64_t* p_full = s_full + 2;        // [2] P_X in TMEM (and O_X rescaled)
+  uint64_t* o_full = p_full + 2;        // [2] last PV_X of an item done
+  uint64_t* o_free = o_full + 2;        // [2] epilogue has read O_X
+  uint64_t* td_bar = o_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(td_bar + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&q_empty[b], 1);
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], kTileM);
+      mbar_init(&o_full[b], 1);
+      mbar_init(&o_free[b], kTileM);
+    }
+    for (int sl = 0; sl < ST; ++sl) {
+      mbar_init(&kv_full[sl], 1);
+      mbar_init(&kv_empty[sl], 1);
+    }
+    mbar_init(td_bar, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    if (MODE != kRouted) tma_prefetch_desc(&tm_q);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int64_t items = num_items2<MODE>(a, pair_own);
+  const int64_t first = blockIdx.x, step = gridDim.x;
+  uint32_t* st = a.status;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t kv_it = 0, lt = 0;
+      bool ok = true;
+      for (int64_t w = first; w < items && ok; w += step, ++lt) {
+        const Item it = item_info<MODE>(a, w, pair_own);
+        if (MODE != kRouted) {
+          const int qb = lt & 1;
+          ok = mbar_wait(&q_empty[qb], ((lt >> 1) & 1) ^ 1, abort_flag, st);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
+#pragma unroll
+          for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int hx = 0; hx < D / 64; ++hx)
+              tma_load_3d(sQ + qb * C::kQBytes + x * C::kSubQBytes + hx * C::kHalfBytes, &tm_q,
+                          &q_full[qb], hx * 64, it.h, (int)(it.qstart + x * kTileM));
+        }
+        for (int j = 0; j < it.nkv && ok; ++j) {
+          const int krow = (int)(it.kstart + (int64_t)j * kTileN);
+#pragma unroll
+          for (int which = 0; which < 2; ++which) {
+            const int sl = kv_it % ST;
+            ok = mbar_wait(&kv_empty[sl], ((kv_it / ST) & 1) ^ 1, abort_flag, st);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&kv_full[sl], C::kKVBytes);
+#pragma unroll
+            for (int hx = 0; hx < D / 64; ++hx)
+              tma_load_3d(sKV + sl * C::kKVBytes + hx * C::kHalfBytes, which ? &tm_v : &tm_k,
+                          &kv_full[sl], hx * 64, it.g, krow);
+            ++kv_it;
+          }
+        }
+      }
+      if (!ok) {
+        const uint32_t n = kv_it < (uint32_t)ST ? kv_it : (uint32_t)ST;
+        for (uint32_t b = 0; b < n; ++b) {
+          const uint32_t i2 = kv_it - 1 - b;
+          mbar_wait_teardown(&kv_full[i2 % ST], (i2 / ST) & 1, 200000000ull);
+        }
+        if (MODE != kRouted && lt > 0) {
+          for (uint32_t b = 0; b < (lt < 2 ? lt : 2u); ++b) {
+            const uint32_t l = lt - 1 - b;
+            mbar_wait_teardown(&q_full[l & 1], (l >> 1) & 1, 200000000ull);
+          }
+        }
+      }
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ Q gather
+    if (MODE == kRouted) {
+      uint32_t lt = 0;
+      bool ok = true;
+      constexpr int CPR = D / 8;     // 16-B chunks per row
+      constexpr int RPI = 32 / CPR;  // rows per warp instruction
+      for (int64_t w = first; w < items && ok; w += step, ++lt) {
+        const Item it = item_info<MODE>(a, w, pair_own);
+        const int qb = lt & 1;
+        ok = mbar_wait(&q_empty[qb], ((lt >> 1) & 1) ^ 1, abort_flag, st);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        const int nrows = it.rows_x[0] + it.rows_x[1];
+        const int c = lane % CPR;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          uint2 ent[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            int r = x * kTileM + lane + 32 * m;
+            if (r >= nrows) r = 0;
+            ent[m] = a.entries[it.e0 + r];
+          }
+          unsigned char* qdst = sQ + qb * C::kQBytes + x * C::kSubQBytes + (c >> 3) * C::kHalfBytes;
+#pragma unroll
+          for (int i = 0; i < kTileM / RPI; ++i) {
+            const int r = i * RPI + lane / CPR;
+            const int m = (i * RPI) / 32;
+            const uint2 e = make_uint2(__shfl_sync(0xffffffffu, ent[m].x, r & 31),
+                                       __shfl_sync(0xffffffffu, ent[m].y, r & 31));
+            const bool good = e.x < (uint32_t)a.L.T && (e.y & 0xFFFFu) < (uint32_t)a.G;
+            const int hq = it.g * a.G + (good ? (int)(e.y & 0xFFFFu) : 0);
+            const __nv_bfloat16* src =
+                a.q + ((size_t)(good ? e.x : 0u) * a.Hq + hq) * D + c * 8;
+            cp_async_16(qdst + sw128_offset(r, c & 7), src);
+          }
+        }
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_full[qb]);
+      }
+      cp_async_wait_all();
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t kv_it = 0, lt = 0;
+      uint32_t ns[2] = {0, 0};  // S MMAs issued per sub-tile (p_full phases follow)
+      uint32_t no[2] = {0, 0};  // items per sub-tile (o_full / o_free phases)
+      bool ok = true;
+      const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
+      auto issue_s = [&](int x, uint32_t qbase, uint32_t ks) {
+        const uint32_t kbase = sKVa + ks * C::kKVBytes;
+        const uint32_t qx = qbase + x * C::kSubQBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
+          tc_mma_ss(tmem + C::col_s(x), sdesc_kmajor_sw128(qx + off),
+                    sdesc_kmajor_sw128(kbase + off), C::kIdescS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[x]);
+        ns[x]++;
+      };
+      auto issue_pv = [&](int x, uint32_t vs, bool acc) {
+        const uint32_t vbase = sKVa + vs * C::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTileN / 16; ++kk)
+          tc_mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8,
+                    sdesc_mnmajor_sw128(vbase + kk * 2048, C::kHalfBytes, 1024), C::kIdescPV,
+                    (acc || kk > 0) ? 1u : 0u);
+      };
+      for (int64_t w = first; w < items && ok; w += step, ++lt) {
+        const Item it = item_info<MODE>(a, w, pair_own);
+        const int qb = lt & 1;
+        const uint32_t qbase = sQa + qb * C::kQBytes;
+        ok = mbar_wait(&q_full[qb], (lt >> 1) & 1, abort_flag, st);
+        if (!ok) break;
+        // K_0
+        uint32_t ks = kv_it % ST;
+        ok = mbar_wait(&kv_full[ks], (kv_it / ST) & 1, abort_flag, st);
+        if (!ok) break;
+        ++kv_it;
+        tc_fence_after();
+        for (int x = 0; x < 2; ++x)
+          if (it.nkv_x[x] > 0) issue_s(x, qbase, ks);
+        tc_commit(&kv_empty[ks]);
+        for (int j = 0; j < it.nkv && ok; ++j) {
+          const uint32_t vs = kv_it % ST;
+          ok = mbar_wait(&kv_full[vs], (kv_it / ST) & 1, abort_flag, st);
+          if (!ok) break;
+          ++kv_it;
+          const bool more = (j + 1 < it.nkv);
+          uint32_t ks2 = 0;
+          if (more) {
+            ks2 = kv_it % ST;
+            ok = mbar_wait(&kv_full[ks2], (kv_it / ST) & 1, abort_flag, st);
+            if (!ok) break;
+            ++kv_it;
+          }
+          for (int x = 0; x < 2 && ok; ++x) {
+            if (j >= it.nkv_x[x]) continue;
+            // P_X(j) ready (S_X(j) has been read and turned into P)
+            ok = mbar_wait(&p_full[x], (ns[x] - 1) & 1, abort_flag, st);
+            if (!ok) break;
+            if (j == 0 && no[x] > 0) {  // the previous item's epilogue has read O_X
+              ok = mbar_wait(&o_free[x], (no[x] - 1) & 1, abort_flag, st);
+              if (!ok) break;
+            }
+            tc_fence_after();
+            issue_pv(x, vs, j > 0);
+            if (j == it.nkv_x[x] - 1) {
+              tc_commit(&o_full[x]);
+              no[x]++;
+            }
+            if (j + 1 < it.nkv_x[x]) issue_s(x, qbase, ks2);
+          }
+          if (!ok) break;
+          tc_commit(&kv_empty[vs]);
+          if (more) tc_commit(&kv_empty[ks2]);
+        }
+        if (ok) tc_commit(&q_empty[qb]);
+      }
+      tc_commit(td_bar);
+      mbar_wait_teardown(td_bar, 0, 500000000ull);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax (warps 0-7)
+    const int x = warp >> 2;               // sub-tile
+    const int r = threadIdx.x & 127;       // row = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::col_s(x);
+    const uint32_t tO = tmem + lane_off + C::col_o(x);
+    uint32_t ns = 0, no = 0;
+    bool ok = true;
+    for (int64_t w = first; w < items && ok; w += step) {
+      const int nkv = item_info<MODE>(a, w, pair_own).nkv_x[x];
+      if (nkv == 0) continue;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < nkv; ++j) {
+        ok = mbar_wait(&s_full[x], ns & 1, abort_flag, st);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        // diagonal tile (own/dense): key c of the tile is visible to row r
+        // only when c <= r, since the tile starts at the sub-tile's first row
+        const bool diag_tile = (MODE != kRouted) && (j == nkv - 1);
+        const float mx = diag_tile ? tile_row_max<true>(tS, r) : tile_row_max<false>(tS, r);
+        const float m_new = fmaxf(m_run, mx * a.scale_log2);
+        const bool need = (j == 0) || (m_new > m_run + 8.0f);
+        const float m_use = need ? m_new : m_run;
+        const float alpha = (j == 0) ? 0.f : (need ? ex2_approx(m_run - m_use) : 1.f);
+        // O_X rescale: PV_X(j-1) finished before S_X(j), which we have seen
+        if (__any_sync(0xffffffffu, j > 0 && need)) {
+          const float f = (j > 0 && need) ? alpha : 1.f;
+#pragma unroll
+          for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c4 * 32, ov);
+            tc_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+            tmem_st32(tO + c4 * 32, ov);
+          }
+        }
+        const float sum = diag_tile ? tile_exp_to_p<true>(tS, r, a.scale_log2, m_use)
+                                    : tile_exp_to_p<false>(tS, r, a.scale_log2, m_use);
+        l_run = l_run * alpha + sum;
+        m_run = m_use;
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[x]);
+        ++ns;
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      ok = mbar_wait(&o_full[x], no & 1, abort_flag, st);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const Item it = item_info<MODE>(a, w, pair_own);
+      const bool valid = r < it.rows_x[x];
+      const float inv = 1.f / l_run;
+      const float lse2 = m_run + lg2_approx(l_run);
+      // destination of this row
+      int kind = 0;  // 0 skip, 1 bf16 partial, 2 fp32 partial, 3 final
+      __nv_bfloat16* dst16 = nullptr;
+      float* dst32 = nullptr;
+      float* lse_dst = nullptr;
+      float lse_val = lse2;
+      if (valid) {
+        if (MODE == kRouted) {
+          const uint2 e = a.entries[it.e0 + x * kTileM + r];
+          const int hh = (int)(e.y & 0xFFFFu), sl = (int)(e.y >> 16);
+          if (e.x < (uint32_t)a.L.T && hh < a.G && sl < a.topk - 1) {
+            const int64_t prow =
+                (((int64_t)it.u * a.L.T + e.x) * a.G + hh) * (a.topk - 1) + sl;
+            kind = 1;
+            dst16 = a.part_O + prow * D;
+            lse_dst = a.part_lse + prow;
+          } else {
+            atomicOr(a.status, MOBA_DEV_BAD_INDEX);
+          }
+        } else {
+          const int64_t t = it.qstart + (int64_t)x * kTileM + r;
+          const bool final_row = (MODE == kDense) || a.topk == 1 || it.own_block == 0;
+          if (final_row) {
+            kind = 3;
+            dst16 = a.o + ((size_t)t * a.Hq + it.h) * D;
+            lse_dst = a.lse + row_index(a.R, it.seq, it.h, t - it.seq_start, t);
+            lse_val = lse2 * 0.6931471805599453f;
+          } else {
+            const int64_t prow = ((int64_t)it.u * a.L.T + t) * a.G + (it.h % a.G);
+            kind = 2;
+            dst32 = a.own_O + prow * D;
+            lse_dst = a.own_lse + prow;
+          }
+        }
+      }
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t ov[32];
+        tmem_ld32(tO + c4 * 32, ov);
+        tc_wait_ld();
+        if (kind == 1 || kind == 3) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst16 + c4 * 32);
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            const float* f = reinterpret_cast<const float*>(&ov[q8 * 8]);
+            d4[q8] = make_uint4(pack_bf16x2(f[0] * inv, f[1] * inv),
+                                pack_bf16x2(f[2] * inv, f[3] * inv),
+                                pack_bf16x2(f[4] * inv, f[5] * inv),
+                                pack_bf16x2(f[6] * inv, f[7] * inv));
+          }
+        } else if (kind == 2) {
+          float4* d4 = reinterpret_cast<float4*>(dst32 + c4 * 32);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            d4[q4] = make_float4(__uint_as_float(ov[4 * q4]) * inv,
+                                 __uint_as_float(ov[4 * q4 + 1]) * inv,
+                                 __uint_as_float(ov[4 * q4 + 2]) * inv,
+                                 __uint_as_float(ov[4 * q4 + 3]) * inv);
+        }
+      }
+      if (kind != 0) *lse_dst = lse_val;
+      tc_fence_before();
+      mbar_arrive(&o_free[x]);
+      ++no;
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace moba

@@ -25,20 +25,21 @@ namespace moba {
 // One CTA.  Validates cu_seqlens and writes block / query-tile numbering.
 __global__ void plan_kernel(SeqLayout L, int B, Plan P, int NBmax, int NQTmax,
                             uint32_t* status) {
-  __shared__ int32_t carry_b, carry_q;
+  __shared__ int32_t carry_b, carry_q, carry_p;
   __shared__ int bad;
-  __shared__ int32_t sb[1024], sq[1024];
+  __shared__ int32_t sb[1024], sq[1024], sp[1024];
   const int tid = threadIdx.x, nt = blockDim.x;
   if (tid == 0) {
     carry_b = 0;
     carry_q = 0;
+    carry_p = 0;
     bad = 0;
     if (L.cu && (L.cu[0] != 0 || (int64_t)L.cu[L.nseq] != L.T)) bad = 1;
   }
   __syncthreads();
   for (int base = 0; base < L.nseq; base += nt) {
     int s = base + tid;
-    int32_t nb = 0, nq = 0;
+    int32_t nb = 0, nq = 0, np = 0;
     if (s < L.nseq) {
       int64_t len = seq_len(L, s);
       if (len < 0) {
@@ -47,41 +48,50 @@ __global__ void plan_kernel(SeqLayout L, int B, Plan P, int NBmax, int NQTmax,
       }
       nb = (int32_t)((len + B - 1) / B);
       nq = (int32_t)((len + kTileM - 1) / kTileM);
+      np = (int32_t)((len + 2 * kTileM - 1) / (2 * kTileM));
     }
     sb[tid] = nb;
     sq[tid] = nq;
+    sp[tid] = np;
     __syncthreads();
     for (int off = 1; off < nt; off <<= 1) {  // inclusive Hillis-Steele scan
       int32_t vb = tid >= off ? sb[tid - off] : 0;
       int32_t vq = tid >= off ? sq[tid - off] : 0;
+      int32_t vp = tid >= off ? sp[tid - off] : 0;
       __syncthreads();
       sb[tid] += vb;
       sq[tid] += vq;
+      sp[tid] += vp;
       __syncthreads();
     }
     if (s < L.nseq) {
       P.blk_off[s] = carry_b + sb[tid] - nb;
       P.qt_off[s] = carry_q + sq[tid] - nq;
+      P.pair_off[s] = carry_p + sp[tid] - np;
     }
     __syncthreads();
     if (tid == nt - 1) {
       carry_b += sb[tid];
       carry_q += sq[tid];
+      carry_p += sp[tid];
     }
     __syncthreads();
   }
   if (tid == 0) {
-    int nbt = carry_b, nqt = carry_q;
+    int nbt = carry_b, nqt = carry_q, npt = carry_p;
     if (nbt > NBmax || nqt > NQTmax) bad = 1;
     if (bad) {
       atomicOr(status, MOBA_DEV_BAD_SEQLENS);
       nbt = 0;
       nqt = 0;
+      npt = 0;
     }
     P.blk_off[L.nseq] = nbt;
     P.qt_off[L.nseq] = nqt;
+    P.pair_off[L.nseq] = npt;
     P.totals[0] = nbt;
     P.totals[1] = nqt;
+    P.totals[2] = npt;
   }
   __syncthreads();
   if (bad) return;
@@ -320,9 +330,10 @@ __global__ void __launch_bounds__(128) gate_kernel(
 // ------------------------------------------------------------------- scan
 // One CTA.  For the units (kv heads) of one pass, flattened as f = u*NB + J:
 // entry_off = exclusive scan of the bucket sizes, tile_off = exclusive scan
-// of ceil(size/128); both get a final total.  Also clears the scatter cursors.
+// of ceil(size/item_rows) (attention work items); both get a final total.  Also clears the scatter cursors.
 __global__ void bucket_scan_kernel(const uint32_t* __restrict__ counts, int u0, int nu,
-                                   const Plan P, int NBmax, int32_t* __restrict__ entry_off,
+                                   int item_rows, const Plan P, int NBmax,
+                                   int32_t* __restrict__ entry_off,
                                    int32_t* __restrict__ tile_off,
                                    uint32_t* __restrict__ cursor) {
   __shared__ int64_t se[1024], stl[1024];
@@ -341,7 +352,7 @@ __global__ void bucket_scan_kernel(const uint32_t* __restrict__ counts, int u0, 
     if (f < M) {
       const int u = f / NB, J = f % NB;
       c = counts[(size_t)(u0 + u) * NBmax + J];
-      tl = (c + kTileM - 1) / kTileM;
+      tl = (c + item_rows - 1) / item_rows;
       cursor[f] = 0;
     }
     se[tid] = c;

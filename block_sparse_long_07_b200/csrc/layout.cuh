@@ -27,9 +27,10 @@ struct SeqLayout {
 
 // Device plan written by plan_kernel (workspace).
 struct Plan {
-  int32_t* totals;    // [0] = number of blocks NB, [1] = number of query tiles NQT
+  int32_t* totals;    // [0] blocks NB, [1] query tiles NQT, [2] query-tile pairs
   int32_t* blk_off;   // [nseq+1] first global block of each sequence
   int32_t* qt_off;    // [nseq+1] first query tile of each sequence
+  int32_t* pair_off;  // [nseq+1] first query-tile pair (256 rows) of each sequence
   int32_t* blk_tok;   // [NBmax] first token of each global block
   int32_t* blk_len;   // [NBmax] tokens in each global block
 };

@@ -23,7 +23,7 @@
 
 #include "moba.h"
 #include "aux_kernels.cuh"
-#include "attn_tc.cuh"
+#include "attn_tc2.cuh"
 #include "common.cuh"
 #include "layout.cuh"
 
@@ -70,6 +70,26 @@ struct Timed {
     timer().pending.push_back(TimedLaunch{cls, a, b});
   }
 };
+
+// Last CUDA runtime error seen by this thread inside the library.
+thread_local const char* g_last_cuda_error = "no error";
+
+moba_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MOBA_OK;
+  g_last_cuda_error = cudaGetErrorString(e);
+  return MOBA_ERR_CUDA;
+}
+
+#define MOBA_TRY(x)                      \
+  do {                                   \
+    moba_status _s = (x);                \
+    if (_s != MOBA_OK) return _s;        \
+  } while (0)
+#define MOBA_CUDA(x)                                   \
+  do {                                                 \
+    moba_status _c = cuda_status(x);                   \
+    if (_c != MOBA_OK) return _c;                      \
+  } while (0)
 
 constexpr size_t kAlign = 256;
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -121,6 +141,7 @@ Ws carve(const Problem& pr, int nu, char* base) {
   w.P.totals = reinterpret_cast<int32_t*>(take(4 * sizeof(int32_t)));
   w.P.blk_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (pr.nseq + 1)));
   w.P.qt_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (pr.nseq + 1)));
+  w.P.pair_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (pr.nseq + 1)));
   w.P.blk_tok = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * NB));
   w.P.blk_len = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * NB));
   w.kbar = reinterpret_cast<float*>(take(sizeof(float) * (size_t)pr.Hkv * NB * pr.D));
@@ -255,17 +276,16 @@ int num_sms() {
 
 template <int D, int MODE>
 moba_status launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const AttnArgs& a, cudaStream_t stream) {
-  using C = AttnCfg<D>;
-  auto kern = attn_tc_kernel<D, MODE>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-      cudaSuccess)
-    return MOBA_ERR_CUDA;
+                        const AttnArgs& a, int pair_own, cudaStream_t stream) {
+  using C = Attn2Cfg<D>;
+  auto kern = attn2_kernel<D, MODE>;
+  MOBA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes));
   const int grid = num_sms();
   if (grid <= 0) return MOBA_ERR_CUDA;
   Timed tm(MODE == kRouted ? kKRouted : (MODE == kOwn ? kKOwn : kKDense), stream);
-  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, a);
-  return cudaGetLastError() == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA;
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, a, pair_own);
+  return cuda_status(cudaGetLastError());
 }
 
 template <int D, int KM>
@@ -273,17 +293,15 @@ moba_status launch_gate_km(const Problem& pr, const void* q, const Ws& w, int32_
                            uint32_t* counts, cudaStream_t st) {
   const size_t smem = sizeof(float) * kGateChunk * D + sizeof(uint32_t) * kMaxBlocksPerSeq;
   auto kern = gate_kernel<D, KM>;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-          cudaSuccess)
-    return MOBA_ERR_CUDA;
+  if (smem > 48 * 1024)
+    MOBA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
   dim3 grid((unsigned)pr.NQTmax, (unsigned)pr.Hq);
   Timed tm(kKGate, st);
   kern<<<grid, 128, smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(q), pr.Hq, pr.G, pr.B,
                                 pr.topk, L, w.P, (int)pr.NBmax, w.kbar, sel, pr.R, counts,
                                 w.status);
-  return cudaGetLastError() == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA;
+  return cuda_status(cudaGetLastError());
 }
 
 template <int D>
@@ -312,7 +330,7 @@ moba_status launch_scatter_ks(const Problem& pr, const Ws& w, const int32_t* sel
   bucket_scatter_kernel<KS><<<grid, 128, sizeof(uint32_t) * kMaxBlocksPerSeq, st>>>(
       sel, pr.R, pr.topk, pr.B, pr.G, u0, nu, L, w.P, w.entry_off, w.cursor, w.entries,
       w.status);
-  return cudaGetLastError() == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA;
+  return cuda_status(cudaGetLastError());
 }
 
 moba_status launch_scatter(const Problem& pr, const Ws& w, const int32_t* sel, int u0, int nu,
@@ -344,16 +362,6 @@ moba_status check_ws(void* ws, size_t ws_bytes, size_t need) {
   if (ws_bytes < need) return MOBA_ERR_WORKSPACE;
   return MOBA_OK;
 }
-
-#define MOBA_TRY(x)                      \
-  do {                                   \
-    moba_status _s = (x);                \
-    if (_s != MOBA_OK) return _s;        \
-  } while (0)
-#define MOBA_CUDA(x)                                   \
-  do {                                                 \
-    if ((x) != cudaSuccess) return MOBA_ERR_CUDA;      \
-  } while (0)
 
 moba_status run_plan_pool(const Problem& pr, const void* k, const Ws& w, cudaStream_t st) {
   SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
@@ -428,14 +436,15 @@ moba_status forward_passes(const Problem& pr, const void* q, const void* k, cons
     if (pr.topk > 1) {
       {
         Timed tm(kKScan, st);
-        bucket_scan_kernel<<<1, 1024, 0, st>>>(w.counts, u0, nu, w.P, (int)pr.NBmax,
-                                               w.entry_off, w.tile_off, w.cursor);
+        bucket_scan_kernel<<<1, 1024, 0, st>>>(w.counts, u0, nu, 2 * kTileM, w.P,
+                                               (int)pr.NBmax, w.entry_off, w.tile_off,
+                                               w.cursor);
       }
       MOBA_CUDA(cudaGetLastError());
       MOBA_TRY(launch_scatter(pr, w, sel, u0, nu, st));
-      MOBA_TRY((launch_attn<D, kRouted>(tq, tk, tv, a, st)));
+      MOBA_TRY((launch_attn<D, kRouted>(tq, tk, tv, a, 1, st)));
     }
-    MOBA_TRY((launch_attn<D, kOwn>(tq, tk, tv, a, st)));
+    MOBA_TRY((launch_attn<D, kOwn>(tq, tk, tv, a, pr.B % (2 * kTileM) == 0 ? 1 : 0, st)));
     if (pr.topk > 1) {
       const int64_t warps = pr.T * nu * pr.G;
       const unsigned blocks = (unsigned)((warps + 7) / 8);
@@ -534,8 +543,8 @@ moba_status dense_impl(const Problem& pr, const void* q, const void* k, const vo
   a.status = w.status;
   a.u0 = 0;
   a.nu = pr.Hkv;
-  return pr.D == 128 ? launch_attn<128, kDense>(tq, tk, tv, a, st)
-                     : launch_attn<64, kDense>(tq, tk, tv, a, st);
+  return pr.D == 128 ? launch_attn<128, kDense>(tq, tk, tv, a, 1, st)
+                     : launch_attn<64, kDense>(tq, tk, tv, a, 1, st);
 }
 
 }  // namespace
@@ -645,6 +654,8 @@ const char* moba_status_string(moba_status s) {
 
 int moba_version(void) { return 100; }
 
+const char* moba_last_error_string(void) { return g_last_cuda_error; }
+
 void moba_profile_enable(int on) { timer().on = (on != 0); }
 
 void moba_profile_reset(void) {
@@ -750,6 +761,7 @@ Ws carve_gate_scratch(const Problem& pr, char* base) {
   w.P.totals = reinterpret_cast<int32_t*>(take(4 * sizeof(int32_t)));
   w.P.blk_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (pr.nseq + 1)));
   w.P.qt_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (pr.nseq + 1)));
+  w.P.pair_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (pr.nseq + 1)));
   w.P.blk_tok = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * NB));
   w.P.blk_len = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * NB));
   w.kbar = reinterpret_cast<float*>(take(sizeof(float) * (size_t)pr.Hkv * NB * pr.D));

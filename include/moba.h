@@ -163,6 +163,10 @@ int moba_profile_read(moba_kernel_time *out, int max_entries);
 /* Static, human-readable name of a status code. */
 const char *moba_status_string(moba_status s);
 
+/* Text of the last CUDA runtime error that made a call on this thread
+ * return MOBA_ERR_CUDA ("no error" if none). */
+const char *moba_last_error_string(void);
+
 /* Library version: major * 10000 + minor * 100 + patch. */
 int moba_version(void);
 
