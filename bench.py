@@ -122,16 +122,22 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def load_traffic(name):
-    """Per-launch DRAM bytes of a kernel from a committed ncu summary, or None."""
+def load_traffic(name, entries_per_launch):
+    """DRAM bytes per launch of a kernel from the committed ncu summary, scaled
+    to this workload by work entries, or None when the kernel source changed
+    since the counters were taken."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            d = json.load(f)
-        ent = d.get(name)
-        return ent
-    except (OSError, ValueError):
+            ent = json.load(f).get(name)
+        with open(os.path.join(ROOT, ent["source_file"]), "rb") as f:
+            sha = hashlib.sha1(f.read()).hexdigest()
+    except (OSError, ValueError, KeyError, TypeError):
         return None
+    if sha != ent.get("source_sha1"):
+        return None
+    return float(ent["bytes_per_entry"]) * entries_per_launch
 
 
 def dist_setup():
@@ -303,7 +309,8 @@ def run_moba(args, w):
     rl = None
     if r_launch:
         achieved = routed_flops * args.steps / (r_ms / 1e3) / 1e12
-        traffic = load_traffic("attn_routed")
+        entries_per_launch = routed_pairs * w.Hq / w.B * args.steps / r_launch
+        traffic = load_traffic("attn_routed", entries_per_launch)
         rl = {"bound": "tensor", "kernel": "attn_routed", "achieved": achieved,
               "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
               "peak_source": "%s bf16_tflops_sustained (kernel runs inside a long step)" % peak_src,
