@@ -67,15 +67,18 @@ struct AttnArgs {
 
 template <int D>
 struct Attn2Cfg {
-  static constexpr int kStages = (D == 128) ? 3 : 4;
+  // One Q buffer and a deep K/V ring: the ring must run a full KV step ahead
+  // so that each TMA load has an MMA iteration to land in.
+  static constexpr int kQBufs = 1;
+  static constexpr int kStages = (D == 128) ? 5 : 8;
   static constexpr int kHalfBytes = kTileM * 128;          // 128 rows x 64 columns bf16
   static constexpr int kSubQBytes = kTileM * D * 2;        // one 128-row Q sub-tile
   static constexpr int kQBytes = 2 * kSubQBytes;           // one work item's Q
   static constexpr int kKVBytes = kTileN * D * 2;
-  static constexpr int kOffQ = 0;                          // two Q buffers
-  static constexpr int kOffKV = kOffQ + 2 * kQBytes;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = kOffQ + kQBufs * kQBytes;
   static constexpr int kOffBar = kOffKV + kStages * kKVBytes;
-  static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 2 * kQBufs + 2 * kStages + 2 + 2 + 2 + 2 + 1;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false, false);
@@ -249,9 +252,10 @@ __global__ void __launch_bounds__(352, 1)
   unsigned char* sQ = smem + C::kOffQ;
   unsigned char* sKV = smem + C::kOffKV;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* q_full = bars + 0;          // [2] Q buffer loaded
-  uint64_t* q_empty = bars + 2;         // [2] Q buffer free (last S MMAs done)
-  uint64_t* kv_full = bars + 4;         // [ST]
+  constexpr int QB = C::kQBufs;
+  uint64_t* q_full = bars + 0;          // [QB] Q buffer loaded
+  uint64_t* q_empty = bars + QB;        // [QB] Q buffer free (last S MMAs done)
+  uint64_t* kv_full = bars + 2 * QB;    // [ST]
   uint64_t* kv_empty = kv_full + ST;    // [ST]
   uint64_t* s_full = kv_empty + ST;     // [2] S_X written
   uint64_t* p_full = s_full + 2;        // [2] P_X in TMEM (and O_X rescaled)
@@ -263,13 +267,15 @@ __global__ void __launch_bounds__(352, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < QB; ++b) {
       mbar_init(&q_full[b], 1);
       mbar_init(&q_empty[b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], kTileM);
+      mbar_init(&p_full[b], kTileM / 32);  // one elected arrival per softmax warp
       mbar_init(&o_full[b], 1);
-      mbar_init(&o_free[b], kTileM);
+      mbar_init(&o_free[b], kTileM / 32);
     }
     for (int sl = 0; sl < ST; ++sl) {
       mbar_init(&kv_full[sl], 1);
@@ -304,8 +310,8 @@ __global__ void __launch_bounds__(352, 1)
       for (int64_t w = first; w < items && ok; w += step, ++lt) {
         const Item it = item_info<MODE>(a, w, pair_own);
         if (MODE != kRouted) {
-          const int qb = lt & 1;
-          ok = mbar_wait(&q_empty[qb], ((lt >> 1) & 1) ^ 1, abort_flag, st);
+          const int qb = lt % QB;
+          ok = mbar_wait(&q_empty[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
           if (!ok) break;
           mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
 #pragma unroll
@@ -338,9 +344,9 @@ __global__ void __launch_bounds__(352, 1)
           mbar_wait_teardown(&kv_full[i2 % ST], (i2 / ST) & 1, 200000000ull);
         }
         if (MODE != kRouted && lt > 0) {
-          for (uint32_t b = 0; b < (lt < 2 ? lt : 2u); ++b) {
+          for (uint32_t b = 0; b < (lt < (uint32_t)QB ? lt : (uint32_t)QB); ++b) {
             const uint32_t l = lt - 1 - b;
-            mbar_wait_teardown(&q_full[l & 1], (l >> 1) & 1, 200000000ull);
+            mbar_wait_teardown(&q_full[l % QB], (l / QB) & 1, 200000000ull);
           }
         }
       }
@@ -354,8 +360,8 @@ __global__ void __launch_bounds__(352, 1)
       constexpr int RPI = 32 / CPR;  // rows per warp instruction
       for (int64_t w = first; w < items && ok; w += step, ++lt) {
         const Item it = item_info<MODE>(a, w, pair_own);
-        const int qb = lt & 1;
-        ok = mbar_wait(&q_empty[qb], ((lt >> 1) & 1) ^ 1, abort_flag, st);
+        const int qb = lt % QB;
+        ok = mbar_wait(&q_empty[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         const int nrows = it.rows_x[0] + it.rows_x[1];
@@ -392,86 +398,85 @@ __global__ void __launch_bounds__(352, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t kv_it = 0, lt = 0;
-      uint32_t ns[2] = {0, 0};  // S MMAs issued per sub-tile (p_full phases follow)
-      uint32_t no[2] = {0, 0};  // items per sub-tile (o_full / o_free phases)
-      bool ok = true;
-      const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
-      auto issue_s = [&](int x, uint32_t qbase, uint32_t ks) {
-        const uint32_t kbase = sKVa + ks * C::kKVBytes;
-        const uint32_t qx = qbase + x * C::kSubQBytes;
+    // The whole warp runs this loop in lock-step (all values warp-uniform);
+    // each tcgen05 instruction is issued by one elected lane.
+    uint32_t kv_it = 0, lt = 0;
+    uint32_t ns0 = 0, ns1 = 0;  // S MMAs issued per sub-tile (p_full phases follow)
+    uint32_t no0 = 0, no1 = 0;  // items per sub-tile (o_full / o_free phases)
+    bool ok = true;
+    const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      const bool r = mbar_wait(bar, parity, abort_flag, st);
+      return __all_sync(0xffffffffu, r);
+    };
+    auto issue_s = [&](int x, uint32_t qbase, uint32_t ks) {
+      const uint32_t kbase = sKVa + ks * C::kKVBytes;
+      const uint32_t qx = qbase + x * C::kSubQBytes;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
-          tc_mma_ss(tmem + C::col_s(x), sdesc_kmajor_sw128(qx + off),
-                    sdesc_kmajor_sw128(kbase + off), C::kIdescS, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&s_full[x]);
-        ns[x]++;
-      };
-      auto issue_pv = [&](int x, uint32_t vs, bool acc) {
-        const uint32_t vbase = sKVa + vs * C::kKVBytes;
-#pragma unroll
-        for (int kk = 0; kk < kTileN / 16; ++kk)
-          tc_mma_ts(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8,
-                    sdesc_mnmajor_sw128(vbase + kk * 2048, C::kHalfBytes, 1024), C::kIdescPV,
-                    (acc || kk > 0) ? 1u : 0u);
-      };
-      for (int64_t w = first; w < items && ok; w += step, ++lt) {
-        const Item it = item_info<MODE>(a, w, pair_own);
-        const int qb = lt & 1;
-        const uint32_t qbase = sQa + qb * C::kQBytes;
-        ok = mbar_wait(&q_full[qb], (lt >> 1) & 1, abort_flag, st);
-        if (!ok) break;
-        // K_0
-        uint32_t ks = kv_it % ST;
-        ok = mbar_wait(&kv_full[ks], (kv_it / ST) & 1, abort_flag, st);
-        if (!ok) break;
-        ++kv_it;
-        tc_fence_after();
-        for (int x = 0; x < 2; ++x)
-          if (it.nkv_x[x] > 0) issue_s(x, qbase, ks);
-        tc_commit(&kv_empty[ks]);
-        for (int j = 0; j < it.nkv && ok; ++j) {
-          const uint32_t vs = kv_it % ST;
-          ok = mbar_wait(&kv_full[vs], (kv_it / ST) & 1, abort_flag, st);
-          if (!ok) break;
-          ++kv_it;
-          const bool more = (j + 1 < it.nkv);
-          uint32_t ks2 = 0;
-          if (more) {
-            ks2 = kv_it % ST;
-            ok = mbar_wait(&kv_full[ks2], (kv_it / ST) & 1, abort_flag, st);
-            if (!ok) break;
-            ++kv_it;
-          }
-          for (int x = 0; x < 2 && ok; ++x) {
-            if (j >= it.nkv_x[x]) continue;
-            // P_X(j) ready (S_X(j) has been read and turned into P)
-            ok = mbar_wait(&p_full[x], (ns[x] - 1) & 1, abort_flag, st);
-            if (!ok) break;
-            if (j == 0 && no[x] > 0) {  // the previous item's epilogue has read O_X
-              ok = mbar_wait(&o_free[x], (no[x] - 1) & 1, abort_flag, st);
-              if (!ok) break;
-            }
-            tc_fence_after();
-            issue_pv(x, vs, j > 0);
-            if (j == it.nkv_x[x] - 1) {
-              tc_commit(&o_full[x]);
-              no[x]++;
-            }
-            if (j + 1 < it.nkv_x[x]) issue_s(x, qbase, ks2);
-          }
-          if (!ok) break;
-          tc_commit(&kv_empty[vs]);
-          if (more) tc_commit(&kv_empty[ks2]);
-        }
-        if (ok) tc_commit(&q_empty[qb]);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::kHalfBytes + (kk & 3) * 32;
+        tc_mma_ss_warp(tmem + C::col_s(x), sdesc_kmajor_sw128(qx + off),
+                       sdesc_kmajor_sw128(kbase + off), C::kIdescS, kk > 0 ? 1u : 0u);
       }
-      tc_commit(td_bar);
-      mbar_wait_teardown(td_bar, 0, 500000000ull);
+      tc_commit_warp(&s_full[x]);
+      if (x == 0) ++ns0; else ++ns1;
+    };
+    auto issue_pv = [&](int x, uint32_t vs, bool acc) {
+      const uint32_t vbase = sKVa + vs * C::kKVBytes;
+#pragma unroll
+      for (int kk = 0; kk < kTileN / 16; ++kk)
+        tc_mma_ts_warp(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8,
+                       sdesc_mnmajor_sw128(vbase + kk * 2048, C::kHalfBytes, 1024), C::kIdescPV,
+                       (acc || kk > 0) ? 1u : 0u);
+    };
+    // one sub-tile's share of KV step j: PV_X(j), then S_X(j+1)
+    auto kv_step = [&](int x, const Item& it, int j, uint32_t vs, uint32_t ks2, uint32_t qbase) {
+      if (j >= it.nkv_x[x]) return true;
+      const uint32_t nsx = x == 0 ? ns0 : ns1;
+      const uint32_t nox = x == 0 ? no0 : no1;
+      if (!wait(&p_full[x], (nsx - 1) & 1)) return false;  // P_X(j) is in TMEM
+      if (j == 0 && nox > 0 && !wait(&o_free[x], (nox - 1) & 1)) return false;
+      tc_fence_after();
+      issue_pv(x, vs, j > 0);
+      if (j == it.nkv_x[x] - 1) {
+        tc_commit_warp(&o_full[x]);
+        if (x == 0) ++no0; else ++no1;
+      }
+      if (j + 1 < it.nkv_x[x]) issue_s(x, qbase, ks2);
+      return true;
+    };
+    for (int64_t w = first; w < items && ok; w += step, ++lt) {
+      const Item it = item_info<MODE>(a, w, pair_own);
+      const int qb = lt % QB;
+      const uint32_t qbase = sQa + qb * C::kQBytes;
+      if (!(ok = wait(&q_full[qb], (lt / QB) & 1))) break;
+      const uint32_t ks = kv_it % ST;
+      if (!(ok = wait(&kv_full[ks], (kv_it / ST) & 1))) break;
+      ++kv_it;
+      tc_fence_after();
+      if (it.nkv_x[0] > 0) issue_s(0, qbase, ks);
+      if (it.nkv_x[1] > 0) issue_s(1, qbase, ks);
+      tc_commit_warp(&kv_empty[ks]);
+      for (int j = 0; j < it.nkv && ok; ++j) {
+        const uint32_t vs = kv_it % ST;
+        if (!(ok = wait(&kv_full[vs], (kv_it / ST) & 1))) break;
+        ++kv_it;
+        const bool more = (j + 1 < it.nkv);
+        uint32_t ks2 = 0;
+        if (more) {
+          ks2 = kv_it % ST;
+          if (!(ok = wait(&kv_full[ks2], (kv_it / ST) & 1))) break;
+          ++kv_it;
+        }
+        if (!(ok = kv_step(0, it, j, vs, ks2, qbase))) break;
+        if (!(ok = kv_step(1, it, j, vs, ks2, qbase))) break;
+        tc_commit_warp(&kv_empty[vs]);
+        if (more) tc_commit_warp(&kv_empty[ks2]);
+      }
+      if (ok) tc_commit_warp(&q_empty[qb]);
     }
+    tc_commit_warp(td_bar);
+    mbar_wait_teardown(td_bar, 0, 500000000ull);
   } else {
     // ------------------------------------------------------------ softmax (warps 0-7)
     const int x = warp >> 2;               // sub-tile
@@ -517,7 +522,8 @@ __global__ void __launch_bounds__(352, 1)
         m_run = m_use;
         tc_wait_st();
         tc_fence_before();
-        mbar_arrive(&p_full[x]);
+        __syncwarp();  // the warp's TMEM stores are ordered before lane 0's arrival
+        if (lane == 0) mbar_arrive(&p_full[x]);
         ++ns;
       }
       if (!ok) break;
@@ -592,7 +598,8 @@ __global__ void __launch_bounds__(352, 1)
       }
       if (kind != 0) *lse_dst = lse_val;
       tc_fence_before();
-      mbar_arrive(&o_free[x]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_free[x]);
       ++no;
     }
   }

@@ -22,9 +22,10 @@ enum : uint32_t {
   MOBA_DEV_CAPACITY = 8u,
 };
 
-// Longest any single wait may take before it is declared stuck (ns).
-#ifndef MOBA_WAIT_LIMIT_NS
-#define MOBA_WAIT_LIMIT_NS 2000000000ull
+// Longest any single wait may take before it is declared stuck, in SM clock
+// cycles (about 2 s at the B200's 1.9 GHz boost clock).
+#ifndef MOBA_WAIT_LIMIT_CYCLES
+#define MOBA_WAIT_LIMIT_CYCLES 4000000000ll
 #endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -66,17 +67,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Bounded wait for the phase of `bar` with the given parity to complete.
 // Returns false (and raises the abort flag) when the CTA is aborting or the
-// wait exceeds MOBA_WAIT_LIMIT_NS.
+// wait exceeds MOBA_WAIT_LIMIT_CYCLES.  The time limit and the abort flag are
+// only checked every 256 polls, so a wait that ends soon costs nothing extra.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           volatile uint32_t* abort_flag,
                                           uint32_t* dev_status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
+  long long t0 = 0;
+  for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
+    if ((it & 255u) == 255u) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > MOBA_WAIT_LIMIT_NS) {
+      const long long now = clock64();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > MOBA_WAIT_LIMIT_CYCLES) {
         *abort_flag = 1u;
         atomicOr(dev_status, MOBA_DEV_TIMEOUT);
         return false;
@@ -167,6 +171,38 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Warp-collective forms: every lane of the warp executes the call with the
+// same operands (so the compiler keeps them in uniform registers) and one
+// lane, chosen by elect.sync, issues the instruction.
+__device__ __forceinline__ void tc_mma_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
       : "memory");
 }
 
