@@ -27,7 +27,7 @@ EXPORTS = ("moba_workspace_size", "moba_workspace_size_varlen", "moba_gate", "mo
            "moba_forward", "moba_forward_varlen", "moba_full_causal_workspace_size",
            "moba_full_causal", "moba_full_causal_varlen", "moba_last_device_status",
            "moba_status_string", "moba_version", "moba_last_error_string", "moba_profile_enable", "moba_profile_reset",
-           "moba_profile_read")
+           "moba_profile_read", "moba_selftest_wait_timeout")
 
 
 class MobaError(RuntimeError):
@@ -95,6 +95,8 @@ def load_library(path=None):
     lib.moba_profile_enable.argtypes = [i32]
     lib.moba_profile_reset.restype = None
     lib.moba_profile_reset.argtypes = []
+    lib.moba_selftest_wait_timeout.restype = i32
+    lib.moba_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_longlong, vp]
     lib.moba_profile_read.restype = i32
     lib.moba_profile_read.argtypes = [ctypes.POINTER(KernelTime), i32]
     if path is None:

@@ -20,7 +20,7 @@
 //   warps 0-3   softmax + epilogue of sub-tile 0 (thread r = row r = TMEM lane r)
 //   warps 4-7   softmax + epilogue of sub-tile 1
 //   warp  8     TMA producer: Q tiles (own/dense) and the K/V ring
-//   warp  9     TMEM allocation and the single-thread MMA issuer
+//   warp  9     TMEM allocation and MMA issue (one elected lane per MMA)
 //   warp 10     Q row gather for routed items (cp.async into swizzled smem)
 // TMEM (512 columns): S_X at 128*X (fp32 scores; after the softmax the first
 // 64 columns hold P_X as packed bf16), O_X at 256 + D*X.

@@ -451,26 +451,33 @@ __global__ void __launch_bounds__(128) bucket_scatter_kernel(
 }
 
 // ------------------------------------------------------------------ merge
-// One warp per (token, head of the pass).  The row's partials -- one per
-// routed past block (bf16 O, log2-domain lse) and the own-block partial
-// (fp32 O, log2 lse) -- are combined by the online-softmax rule
+// The row's partials -- one per routed past block (bf16 O, log2-domain lse)
+// and the own-block partial (fp32 O, log2 lse) -- are combined by the
+// online-softmax rule
 //   m = max lse_s, w_s = 2^(lse_s - m), O = sum w_s O_s / sum w_s,
 //   lse = m + log2(sum w_s)   (output converted to natural log).
-// Rows whose selection is the own block alone were finished by the
-// own-block kernel and are skipped.  Slots are combined in ascending order.
+// A group of D/8 lanes owns one (token, head) row; each lane owns 8 of its
+// columns, so every partial row is read with one 16-byte load per lane and
+// four slots are loaded before any is used.  Rows whose selection is the own
+// block alone were finished by the own-block kernel and are skipped.  The
+// own-block partial is combined first, then the routed slots in ascending
+// order.
 template <int D>
 __global__ void __launch_bounds__(256) merge_kernel(
     const __nv_bfloat16* __restrict__ part_O, const float* __restrict__ part_lse,
     const float* __restrict__ own_O, const float* __restrict__ own_lse, int topk, int B, int G,
     int Hq, int u0, int nu, SeqLayout L, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
     RowLayout R) {
-  constexpr int EPL = D / 32;  // elements per lane
+  constexpr int LPR = D / 8;       // lanes per row
+  constexpr int RPW = 32 / LPR;    // rows per warp
   const int lane = threadIdx.x & 31;
-  const int64_t wid = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int sub = lane % LPR;
+  const int64_t row =
+      ((int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)) * RPW + lane / LPR;
   const int HP = nu * G;
-  if (wid >= L.T * HP) return;
-  const int64_t t = wid / HP;
-  const int hl = (int)(wid % HP);
+  if (row >= L.T * HP) return;
+  const int64_t t = row / HP;
+  const int hl = (int)(row % HP);
   const int u = hl / G, hh = hl % G, h = u0 * G + hl;
   const int s = seq_of_token(L, t);
   const int64_t pos = t - seq_start(L, s);
@@ -480,54 +487,68 @@ __global__ void __launch_bounds__(256) merge_kernel(
   const int npast = cnt - 1;
   const int64_t prow = ((int64_t)u * L.T + t) * G + hh;  // partial row
   const int64_t pbase = prow * (topk - 1);
-  // lse of every slot: past slots first, own block last
-  float m = -INFINITY;
-  for (int sl = lane; sl <= npast; sl += 32) {
-    float v = (sl < npast) ? part_lse[pbase + sl] : own_lse[prow];
-    m = fmaxf(m, v);
+  const float* lrow = part_lse + pbase;
+  const float lown = own_lse[prow];
+  float m = lown;
+  for (int sl = 0; sl < npast; ++sl) m = fmaxf(m, lrow[sl]);
+  float acc[8];
+  float den;
+  {
+    const float w = ex2_approx(lown - m);
+    den = w;
+    const float4* src = reinterpret_cast<const float4*>(own_O + prow * D + sub * 8);
+    const float4 a = src[0], b = src[1];
+    acc[0] = w * a.x;
+    acc[1] = w * a.y;
+    acc[2] = w * a.z;
+    acc[3] = w * a.w;
+    acc[4] = w * b.x;
+    acc[5] = w * b.y;
+    acc[6] = w * b.z;
+    acc[7] = w * b.w;
   }
+  const uint4* orow = reinterpret_cast<const uint4*>(part_O + pbase * D) + sub;
+  constexpr int kStride = D / 8;  // uint4 per partial row
+  int sl = 0;
+  for (; sl + 4 <= npast; sl += 4) {
+    uint4 v[4];
+    float w[4];
 #pragma unroll
-  for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  float acc[EPL];
+    for (int q = 0; q < 4; ++q) v[q] = orow[(sl + q) * kStride];
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
-  float den = 0.f;
-  for (int sl = 0; sl < npast; ++sl) {
-    const float w = ex2_approx(part_lse[pbase + sl] - m);
-    den += w;
-    const __nv_bfloat16* src = part_O + (pbase + sl) * D + lane * EPL;
-    if constexpr (EPL == 4) {
-      uint2 raw = *reinterpret_cast<const uint2*>(src);
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-      float2 a = __bfloat1622float2(h2[0]), b = __bfloat1622float2(h2[1]);
-      acc[0] = fmaf(w, a.x, acc[0]);
-      acc[1] = fmaf(w, a.y, acc[1]);
-      acc[2] = fmaf(w, b.x, acc[2]);
-      acc[3] = fmaf(w, b.y, acc[3]);
-    } else {
-      uint32_t raw = *reinterpret_cast<const uint32_t*>(src);
-      float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw));
-      acc[0] = fmaf(w, a.x, acc[0]);
-      acc[1] = fmaf(w, a.y, acc[1]);
+    for (int q = 0; q < 4; ++q) w[q] = ex2_approx(lrow[sl + q] - m);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      den += w[q];
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[q]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        acc[2 * e] = fmaf(w[q], f.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(w[q], f.y, acc[2 * e + 1]);
+      }
     }
   }
-  {
-    const float w = ex2_approx(own_lse[prow] - m);
+  for (; sl < npast; ++sl) {
+    const uint4 v = orow[sl * kStride];
+    const float w = ex2_approx(lrow[sl] - m);
     den += w;
-    const float* src = own_O + prow * D + lane * EPL;
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, src[e], acc[e]);
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h2[e]);
+      acc[2 * e] = fmaf(w, f.x, acc[2 * e]);
+      acc[2 * e + 1] = fmaf(w, f.y, acc[2 * e + 1]);
+    }
   }
   const float inv = 1.f / den;
-  __nv_bfloat16* dst = o + ((size_t)t * Hq + h) * D + lane * EPL;
-  if constexpr (EPL == 4) {
-    uint2 outv = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv),
-                            pack_bf16x2(acc[2] * inv, acc[3] * inv));
-    *reinterpret_cast<uint2*>(dst) = outv;
-  } else {
-    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-  }
-  if (lane == 0) lse[row_index(R, s, h, pos, t)] = (m + lg2_approx(den)) * 0.6931471805599453f;
+  uint4 out;
+  out.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  out.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  out.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  out.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  *(reinterpret_cast<uint4*>(o + ((size_t)t * Hq + h) * D) + sub) = out;
+  if (sub == 0) lse[row_index(R, s, h, pos, t)] = (m + lg2_approx(den)) * 0.6931471805599453f;
 }
 
 }  // namespace moba

@@ -70,8 +70,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // wait exceeds MOBA_WAIT_LIMIT_CYCLES.  The time limit and the abort flag are
 // only checked every 256 polls, so a wait that ends soon costs nothing extra.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile uint32_t* abort_flag,
-                                          uint32_t* dev_status) {
+                                          volatile uint32_t* abort_flag, uint32_t* dev_status,
+                                          long long limit_cycles = MOBA_WAIT_LIMIT_CYCLES) {
   long long t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -80,7 +80,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
       const long long now = clock64();
       if (t0 == 0) {
         t0 = now;
-      } else if (now - t0 > MOBA_WAIT_LIMIT_CYCLES) {
+      } else if (now - t0 > limit_cycles) {
         *abort_flag = 1u;
         atomicOr(dev_status, MOBA_DEV_TIMEOUT);
         return false;

@@ -446,8 +446,9 @@ moba_status forward_passes(const Problem& pr, const void* q, const void* k, cons
     }
     MOBA_TRY((launch_attn<D, kOwn>(tq, tk, tv, a, pr.B % (2 * kTileM) == 0 ? 1 : 0, st)));
     if (pr.topk > 1) {
-      const int64_t warps = pr.T * nu * pr.G;
-      const unsigned blocks = (unsigned)((warps + 7) / 8);
+      const int64_t rows = pr.T * nu * pr.G;
+      const int64_t rows_per_block = 8 * (32 / (D / 8));
+      const unsigned blocks = (unsigned)((rows + rows_per_block - 1) / rows_per_block);
       Timed tm(kKMerge, st);
       merge_kernel<D><<<blocks, 256, 0, st>>>(w.part_O, w.part_lse, w.own_O, w.own_lse, pr.topk,
                                               pr.B, pr.G, pr.Hq, u0, nu, L,
@@ -547,9 +548,32 @@ moba_status dense_impl(const Problem& pr, const void* q, const void* k, const vo
                      : launch_attn<64, kDense>(tq, tk, tv, a, 1, st);
 }
 
+// One thread waits, with the pipelines' bounded wait and a short limit, on a
+// barrier nothing ever arrives on.  The wait must give up, raise the timeout
+// bit in the status word and let the kernel return.
+__global__ void wait_selftest_kernel(uint32_t* status, long long limit_cycles) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  abort_flag = 0u;
+  fence_barrier_init();
+  mbar_wait(&bar, 0, &abort_flag, status, limit_cycles);
+}
+
 }  // namespace
 
 extern "C" {
+
+moba_status moba_selftest_wait_timeout(void* ws, size_t ws_bytes, long long limit_cycles,
+                                       moba_stream_t stream) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) || ws_bytes < kAlign)
+    return MOBA_ERR_WORKSPACE;
+  if (limit_cycles <= 0 || limit_cycles > MOBA_WAIT_LIMIT_CYCLES) return MOBA_ERR_INVALID_ARG;
+  wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint32_t*>(ws), limit_cycles);
+  return cuda_status(cudaGetLastError());
+}
 
 size_t moba_workspace_size(const moba_params* p, int heads_per_pass) {
   Problem pr;

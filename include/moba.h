@@ -160,6 +160,15 @@ void moba_profile_enable(int on);
 void moba_profile_reset(void);
 int moba_profile_read(moba_kernel_time *out, int max_entries);
 
+/* Diagnostic: launches one thread that waits, with the same bounded wait the
+ * pipelines use but a limit of `limit_cycles` SM clocks (1 .. 4e9), on a
+ * barrier nothing arrives on.  The wait gives up and latches the timeout bit
+ * in ws's status word; moba_last_device_status(ws) then returns
+ * MOBA_ERR_TIMEOUT and the context stays usable.  Shows that a stuck pipeline
+ * ends in an error status instead of a hang.  ws needs 256 bytes. */
+moba_status moba_selftest_wait_timeout(void *ws, size_t ws_bytes, long long limit_cycles,
+                                       moba_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 const char *moba_status_string(moba_status s);
 

@@ -143,3 +143,11 @@ def test_topk_limit(lib):
 def test_binding_refuses_missing_library(tmp_path):
     with pytest.raises(OSError):
         moba.load_library(str(tmp_path / "nope.so"))
+
+
+def test_selftest_argument_checks(lib):
+    assert lib.moba_selftest_wait_timeout(None, 4096, 1000, None) == WORKSPACE
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.moba_selftest_wait_timeout(fake, 4096, 0, None) == INVALID
+    assert lib.moba_selftest_wait_timeout(fake, 4096, 10**12, None) == INVALID
+    assert lib.moba_selftest_wait_timeout(fake, 16, 1000, None) == WORKSPACE
