@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...     # the fp64 CPU oracle, bounded sample
+    python bench.py --mode decode ...        # one decode step against the workload as a cache
 
 A step is one full MoBA prefill forward (pool, gate, bucketing, routed and
 own-block attention, merge) over the workload's synthetic input, through the
@@ -35,6 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoBA prefill ms & effective TFLOP/s at 1M tokens; % bf16 tensor peak; x vs dense"
+DECODE_METRIC = "MoBA decode steps/s (one new token per sequence) against a 1M-token KV cache"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -422,6 +424,228 @@ def run_moba(args, w):
     return 0 if status == 0 else 1
 
 
+# ----------------------------------------------------------------- decode
+def decode_bytes(sel, N, B, Hkv, G, d):
+    """Algorithmic HBM bytes of one decode step of a batch of sequences of N
+    tokens: K and V of the union of the blocks the q heads of each kv head
+    chose (a block shared by several heads is read once), the block means the
+    gate scores, and the new token's q / o / lse."""
+    b, Hq, k = sel.shape
+    i = (N - 1) // B
+    keys = 0
+    for s in range(b):
+        for g in range(Hkv):
+            for j in set(sel[s, g * G:(g + 1) * G].ravel().tolist()) - {-1}:
+                keys += min(N, (j + 1) * B) - j * B
+    kv = keys * d * 2 * 2
+    kbar = b * Hkv * i * d * 4
+    io = b * Hq * (d * 2 * 2 + 4)
+    return kv, kv + kbar + io
+
+
+def run_decode(args, w):
+    """One decode step per sequence: the workload's K / V are the cache, the
+    new token is each sequence's last, the block-mean cache is built before
+    timing (a prefill leaves it) and updated for the completed block inside
+    every step."""
+    import torch
+    import block_sparse_long_07_b200 as moba
+    import synthetic as S
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=dev)
+        pg = dist
+    if not w.batch_mode:
+        raise SystemExit("decode mode takes a batch workload")
+    b, N = len(w.lengths), w.lengths[0]
+    G = w.Hq // w.Hkv
+    q, k, v = S.make_qkv(w, dev, seed=w.seed + 1000 * rank)
+    kc = k.view(b, N, w.Hkv, w.d)
+    vc = v.view(b, N, w.Hkv, w.d)
+    qd = q.view(b, N, w.Hq, w.d)[:, N - 1].contiguous()
+    del q
+    lens = torch.full((b,), N, dtype=torch.int32, device=dev)
+    p = moba.make_decode_params(b, N, w.Hq, w.Hkv, w.d, w.B, w.k)
+    ws = moba.alloc_workspace(moba.decode_workspace_size(p), dev)
+    kbar = moba.alloc_kbar_cache(kc, w.B)
+    moba.kbar_cache_update(kc, lens, kbar, w.B, ws=ws)
+    o = torch.empty_like(qd)
+    lse = torch.empty(b, w.Hq, dtype=torch.float32, device=dev)
+    sel = torch.empty(b, w.Hq, w.k, dtype=torch.int32, device=dev)
+
+    def step(qin=qd):
+        moba.kbar_cache_update(kc, lens, kbar, w.B, only_last=True, ws=ws)
+        moba.decode(qin, kc, vc, lens, kbar, w.B, w.k, ws=ws, out=o, lse=lse, sel_out=sel)
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    def max_over_ranks(x):
+        if pg is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = moba.last_device_status(ws)
+    if status != 0:
+        raise RuntimeError("device status %d after warm-up" % status)
+    kv_bytes, algo_bytes = decode_bytes(sel.cpu().numpy(), N, w.B, w.Hkv, G, w.d)
+
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    moba.profile_enable(True)
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    kern = moba.profile_read()
+    moba.profile_enable(False)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    value = world * b / (ms / 1e3)
+
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    a_launch, a_ms = kern.get("decode_attn", (0, 0.0))
+    rl = None
+    if a_launch:
+        achieved = kv_bytes * args.steps / a_launch / (a_ms / a_launch / 1e3) / 1e9
+        rl = {"bound": "hbm", "kernel": "decode_attn", "achieved": achieved, "peak": hbm,
+              "unit": "GB/s", "frac": achieved / hbm,
+              "peak_source": "%s hbm_gbs (copy bandwidth)" % peak_src, "traffic": None,
+              "bytes_per_launch": kv_bytes, "ms_per_launch": a_ms / a_launch}
+    launches = int(sum(n for n, _ in kern.values()))
+    kernels_ms = {name: round(t / args.steps, 5) for name, (n, t) in kern.items() if n}
+
+    # ---- end to end: the new token's q from pinned host memory, o and lse back
+    e2e = None
+    if not args.no_e2e:
+        qh = qd.cpu().pin_memory()
+        oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        qdev = torch.empty_like(qd)
+
+        def estep():
+            qdev.copy_(qh, non_blocking=True)
+            step(qdev)
+            oh.copy_(o, non_blocking=True)
+            lh.copy_(lse, non_blocking=True)
+
+        for _ in range(args.warmup):
+            estep()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            estep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        e2e = {"value": world * b / (ems / 1e3), "unit": "steps/s", "ms_per_step": ems,
+               "h2d_bytes_per_step": qh.numel() * qh.element_size(),
+               "d2h_bytes_per_step": oh.numel() * oh.element_size() +
+               lh.numel() * lh.element_size()}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu:
+        from oracle import bf16_bits
+        cpu = cpu_decode_baseline(w, bf16_bits(qd.view(b, 1, w.Hq, w.d)), bf16_bits(k),
+                                  bf16_bits(v), budget_s=args.cpu_seconds)
+    if rank == 0:
+        line = {"metric": DECODE_METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "us_per_step": 1e3 * ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "decode_" + w.name, "context_tokens": N, "sequences": b,
+                           "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
+                           "block_size": w.B, "top_k": w.k,
+                           "l2": "chosen blocks' K / V ({:.0f} MB) exceed L2; no flush".format(
+                               kv_bytes / 1e6),
+                           "parallelism": "replicas x%d (independent problems)" % world},
+                "algorithmic_bytes_per_step": algo_bytes,
+                "roofline": rl, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+                "kernels_ms_per_step": kernels_ms, "clocks": clk, "device_status": status}
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+    return 0
+
+
+def cpu_decode_baseline(w, qdec_bits, k_bits, v_bits, budget_s=15.0):
+    """The oracle on the decode rows (every sequence's last token, all heads),
+    repeated for about budget_s seconds; the block means are computed once
+    beforehand, as the GPU path keeps them in its cache."""
+    from oracle import Oracle
+    b, N = len(w.lengths), w.lengths[0]
+    q_bits = np.zeros((w.T, w.Hq, w.d), dtype=np.uint16)  # lazily backed; decode rows set
+    rows = np.array([s * N + N - 1 for s in range(b)], dtype=np.int64)
+    q_bits[rows] = qdec_bits.reshape(b, w.Hq, w.d)
+    orc = Oracle(q_bits, k_bits, v_bits, w.cu, w.Hq, w.Hkv, w.d, w.B, w.k)
+    orc.block_means()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        orc.forward(rows)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    secs = (time.perf_counter() - t0) / n
+    return {"value": b / secs, "unit": "steps/s", "cores": Oracle.num_threads(),
+            "kind": "oracle", "seconds": secs,
+            "sample": "%d decode steps of %d sequence(s) x %d heads at %d context tokens "
+                      "(block means precomputed)" % (n, b, w.Hq, N)}
+
+
+def run_decode_reference(args, w):
+    import synthetic as S
+    from oracle import bf16_bits
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    b, N = len(w.lengths), w.lengths[0]
+    q, k, v = S.make_qkv(w, "cpu")
+    qd = q.view(b, N, w.Hq, w.d)[:, N - 1].contiguous()
+    qb, kb, vb = bf16_bits(qd), bf16_bits(k), bf16_bits(v)
+    del q, k, v
+    for _ in range(args.warmup):
+        cpu_decode_baseline(w, qb, kb, vb, budget_s=0.5)
+    res = [cpu_decode_baseline(w, qb, kb, vb, budget_s=args.ref_step_seconds / 4)
+           for _ in range(args.steps)]
+    secs = float(np.mean([r["seconds"] for r in res]))
+    value = b / secs
+    line = {"impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "steps/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "decode_" + w.name, "context_tokens": N, "sequences": b,
+                       "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
+                       "block_size": w.B, "top_k": w.k},
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": res[0]["cores"],
+                             "kind": "oracle", "sample": res[0]["sample"]},
+            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -438,12 +662,17 @@ def main():
     ap.add_argument("--ws-budget-gb", type=float, default=None,
                     help="workspace budget (default: the binding's, 32 GiB)")
     ap.add_argument("--ref-step-seconds", type=float, default=20.0)
+    ap.add_argument("--mode", default="prefill", choices=["prefill", "decode"])
     args = ap.parse_args()
     import synthetic as S
     if args.workload.endswith("_k32"):
         w = S.WORKLOADS[args.workload[:-4]].with_k(32)
     else:
         w = S.WORKLOADS[args.workload]
+    if args.mode == "decode":
+        if args.impl == "reference":
+            return run_decode_reference(args, w)
+        return run_decode(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_moba(args, w)

@@ -27,7 +27,8 @@ EXPORTS = ("moba_workspace_size", "moba_workspace_size_varlen", "moba_gate", "mo
            "moba_forward", "moba_forward_varlen", "moba_full_causal_workspace_size",
            "moba_full_causal", "moba_full_causal_varlen", "moba_last_device_status",
            "moba_status_string", "moba_version", "moba_last_error_string", "moba_profile_enable", "moba_profile_reset",
-           "moba_profile_read", "moba_selftest_wait_timeout")
+           "moba_profile_read", "moba_selftest_wait_timeout", "moba_decode_workspace_size",
+           "moba_kbar_cache_size", "moba_kbar_cache_update", "moba_decode")
 
 
 class MobaError(RuntimeError):
@@ -39,6 +40,13 @@ class MobaError(RuntimeError):
 
 class MobaParams(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("seqlen", ctypes.c_int),
+                ("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("block_size", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("softmax_scale", ctypes.c_float)]
+
+
+class MobaDecodeParams(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("cache_len", ctypes.c_int),
                 ("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int),
                 ("head_dim", ctypes.c_int), ("block_size", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("softmax_scale", ctypes.c_float)]
@@ -99,6 +107,15 @@ def load_library(path=None):
     lib.moba_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_longlong, vp]
     lib.moba_profile_read.restype = i32
     lib.moba_profile_read.argtypes = [ctypes.POINTER(KernelTime), i32]
+    dp = ctypes.POINTER(MobaDecodeParams)
+    lib.moba_decode_workspace_size.restype = sz
+    lib.moba_decode_workspace_size.argtypes = [dp]
+    lib.moba_kbar_cache_size.restype = sz
+    lib.moba_kbar_cache_size.argtypes = [dp]
+    lib.moba_kbar_cache_update.restype = i32
+    lib.moba_kbar_cache_update.argtypes = [vp, vp, vp, i32, dp, vp, sz, vp]
+    lib.moba_decode.restype = i32
+    lib.moba_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, dp, vp, sz, vp]
     if path is None:
         _lib = lib
     return lib
@@ -177,8 +194,8 @@ def profile_enable(on=True):
 
 def profile_read():
     """{kernel class: (launches, total device ms)} since profile_enable."""
-    arr = (KernelTime * 16)()
-    n = load_library().moba_profile_read(arr, 16)
+    arr = (KernelTime * 32)()
+    n = load_library().moba_profile_read(arr, 32)
     return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n)}
 
 
@@ -303,4 +320,64 @@ def full_causal_varlen(q, k, v, cu_seqlens, softmax_scale=0.0, ws=None, out=None
                                                   nseq, T, _ptr(out), _ptr(lse), ctypes.byref(p),
                                                   _ptr(ws), ws.numel(), _stream(stream)),
            "moba_full_causal_varlen")
+    return out, lse
+
+
+# ---------------------------------------------------------------- decode
+def make_decode_params(batch, cache_len, Hq, Hkv, d, block_size, top_k, softmax_scale=0.0):
+    return MobaDecodeParams(int(batch), int(cache_len), int(Hq), int(Hkv), int(d),
+                            int(block_size), int(top_k), float(softmax_scale))
+
+
+def decode_workspace_size(params):
+    return int(load_library().moba_decode_workspace_size(ctypes.byref(params)))
+
+
+def kbar_cache_size(params):
+    return int(load_library().moba_kbar_cache_size(ctypes.byref(params)))
+
+
+def _decode_params(k_cache, q_heads, block_size, top_k, softmax_scale):
+    b, cap, Hkv, d = k_cache.shape
+    return make_decode_params(b, cap, q_heads, Hkv, d, block_size, top_k, softmax_scale)
+
+
+def alloc_kbar_cache(k_cache, block_size):
+    """Zeroed fp32 block-mean cache [b, Hkv, ceil(cap / B), d] for k_cache [b, cap, Hkv, d]."""
+    torch = _torch()
+    b, cap, Hkv, d = k_cache.shape
+    return torch.zeros(b, Hkv, (cap + block_size - 1) // block_size, d, dtype=torch.float32,
+                       device=k_cache.device)
+
+
+def kbar_cache_update(k_cache, seqlens, kbar, block_size, only_last=False, ws=None, stream=None):
+    """Block means of the complete cache blocks (all, or the one the newest token completed)."""
+    _require_cuda_bf16(k_cache)
+    p = _decode_params(k_cache, k_cache.shape[2], block_size, 1, 0.0)
+    if ws is None:
+        ws = alloc_workspace(decode_workspace_size(p), k_cache.device)
+    _check(load_library().moba_kbar_cache_update(_ptr(k_cache), _ptr(seqlens), _ptr(kbar),
+                                                 1 if only_last else 0, ctypes.byref(p),
+                                                 _ptr(ws), ws.numel(), _stream(stream)),
+           "moba_kbar_cache_update")
+    return kbar
+
+
+def decode(q, k_cache, v_cache, seqlens, kbar, block_size, top_k, softmax_scale=0.0, ws=None,
+           out=None, lse=None, sel_out=None, stream=None):
+    """One decode step for q [b, Hq, d] against k/v caches [b, cap, Hkv, d]: (o, lse [b, Hq])."""
+    torch = _torch()
+    _require_cuda_bf16(q, k_cache, v_cache)
+    b, Hq, d = q.shape
+    p = _decode_params(k_cache, Hq, block_size, top_k, softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(b, Hq, dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(decode_workspace_size(p), q.device)
+    _check(load_library().moba_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
+                                      _ptr(kbar), _ptr(out), _ptr(lse), _ptr(sel_out),
+                                      ctypes.byref(p), _ptr(ws), ws.numel(), _stream(stream)),
+           "moba_decode")
     return out, lse

@@ -206,7 +206,10 @@ __device__ __forceinline__ float tile_row_max(uint32_t tS, int r) {
 // P = 2^(s * scale_log2 - m) for one score tile, written back as packed bf16
 // pairs into the tile's first 64 TMEM columns (chunk h2 of 64 scores becomes
 // 32 packed columns, which never overlap scores still to be read).  Returns
-// the row sum of the fp32 probabilities.
+// the row sum of the fp32 probabilities.  Scale-and-shift and the sums run
+// as packed pairs; one pair in eight takes 2^x from a polynomial on the FMA
+// pipe, the rest from the special-function unit, whose throughput otherwise
+// bounds this loop.
 template <bool MASK>
 __device__ __forceinline__ float tile_exp_to_p(uint32_t tS, int r, float scale_log2,
                                                float m_use) {
@@ -229,9 +232,17 @@ __device__ __forceinline__ float tile_exp_to_p(uint32_t tS, int r, float scale_l
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const float p0 = ex2_approx(fmaf(sv[q2 * 32 + 2 * e], scale_log2, -m_use));
-        const float p1 = ex2_approx(fmaf(sv[q2 * 32 + 2 * e + 1], scale_log2, -m_use));
-        sp[e & 7] += p0 + p1;
+        float x0, x1;
+        ffma2(x0, x1, sv[q2 * 32 + 2 * e], sv[q2 * 32 + 2 * e + 1], scale_log2, scale_log2,
+              -m_use, -m_use);
+        float p0, p1;
+        if ((e & 7) == 7) {  // one pair in eight on the FMA pipe
+          exp2_poly2(p0, p1, x0, x1);
+        } else {
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
+        }
+        fadd2(sp[2 * (e & 3)], sp[2 * (e & 3) + 1], p0, p1);
         pk[e] = pack_bf16x2(p0, p1);
       }
       tmem_st16(tS + h2 * 32 + q2 * 16, pk);

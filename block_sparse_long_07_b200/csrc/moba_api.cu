@@ -24,6 +24,8 @@
 #include "moba.h"
 #include "aux_kernels.cuh"
 #include "attn_tc2.cuh"
+#include "gate_tc.cuh"
+#include "decode.cuh"
 #include "common.cuh"
 #include "layout.cuh"
 
@@ -33,10 +35,13 @@ namespace {
 
 // ------------------------------------------------------------ kernel timer
 enum KernelClass {
-  kKPlan, kKPool, kKGate, kKScan, kKScatter, kKRouted, kKOwn, kKMerge, kKDense, kKNum
+  kKPlan, kKPool, kKGate, kKGateCount, kKScan, kKScatter, kKRouted, kKOwn, kKMerge, kKDense,
+  kKKbarCache, kKDecGate, kKDecAttn, kKDecMerge, kKNum
 };
-const char* const kKernelNames[kKNum] = {"plan", "pool", "gate", "bucket_scan", "bucket_scatter",
-                                         "attn_routed", "attn_own", "merge", "attn_dense"};
+const char* const kKernelNames[kKNum] = {
+    "plan",        "pool",     "gate",       "gate_count",  "bucket_scan",
+    "bucket_scatter", "attn_routed", "attn_own", "merge",    "attn_dense",
+    "kbar_cache",  "decode_gate", "decode_attn", "decode_merge"};
 struct TimedLaunch {
   int cls;
   cudaEvent_t a, b;
@@ -304,10 +309,70 @@ moba_status launch_gate_km(const Problem& pr, const void* q, const Ws& w, int32_
   return cuda_status(cudaGetLastError());
 }
 
+// Tensor-core gate: scores as tcgen05 MMAs, branch-free selection; then
+// the bucket sizes from the written selections.
+template <int D, int KM>
+moba_status launch_gate_tc_km(const Problem& pr, const void* q, const Ws& w, int32_t* sel,
+                              uint32_t* counts, cudaStream_t st) {
+  using C = GateTcCfg<D>;
+  CUtensorMap tq;
+  if (!make_tmap(&tq, q, pr.Hq, pr.T, D)) return MOBA_ERR_CUDA;
+  auto kern = gate_tc_kernel<D, KM>;
+  MOBA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes));
+  const int grid = num_sms();
+  if (grid <= 0) return MOBA_ERR_CUDA;
+  SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
+  GateTcArgs a;
+  a.kbar = w.kbar;
+  a.Hq = pr.Hq;
+  a.G = pr.G;
+  a.B = pr.B;
+  a.topk = pr.topk;
+  a.NBmax = (int)pr.NBmax;
+  a.L = L;
+  a.P = w.P;
+  a.R = pr.R;
+  a.sel = sel;
+  a.status = w.status;
+  {
+    Timed tm(kKGate, st);
+    kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, a);
+    MOBA_CUDA(cudaGetLastError());
+  }
+  if (counts) {
+    const size_t smem = sizeof(uint32_t) * kMaxBlocksPerSeq;
+    dim3 cgrid((unsigned)pr.NQTmax, (unsigned)pr.Hkv);
+    Timed tm(kKGateCount, st);
+    gate_count_kernel<<<cgrid, 128, smem, st>>>(sel, pr.R, pr.topk, pr.B, pr.G, L, w.P,
+                                                (int)pr.NBmax, counts, w.status);
+    MOBA_CUDA(cudaGetLastError());
+  }
+  return MOBA_OK;
+}
+
+// The tensor-core gate ranks up to 16 past blocks out of at most 256 per sequence.
+bool gate_tc_fits(const Problem& pr) {
+  const int64_t npast = pr.topk - 1;
+  return npast >= 1 && npast <= kGateTcMaxKeep && npast < pr.max_blocks_per_seq - 1 &&
+         pr.max_blocks_per_seq - 1 <= kGateTcMaxPast;
+}
+
 template <int D>
 moba_status launch_gate(const Problem& pr, const void* q, const Ws& w, int32_t* sel,
                         uint32_t* counts, cudaStream_t st) {
   const int64_t npast = pr.topk - 1;
+  if (gate_tc_fits(pr)) {
+    switch (pow2_at_least(npast)) {
+      case 1: return launch_gate_tc_km<D, 1>(pr, q, w, sel, counts, st);
+      case 2: return launch_gate_tc_km<D, 2>(pr, q, w, sel, counts, st);
+      case 4: return launch_gate_tc_km<D, 4>(pr, q, w, sel, counts, st);
+      case 8: return launch_gate_tc_km<D, 8>(pr, q, w, sel, counts, st);
+      default:
+        if (npast <= 12) return launch_gate_tc_km<D, 12>(pr, q, w, sel, counts, st);
+        return launch_gate_tc_km<D, 16>(pr, q, w, sel, counts, st);
+    }
+  }
   const int64_t need = (npast >= pr.max_blocks_per_seq - 1) ? 1 : npast;
   switch (pow2_at_least(need)) {
     case 1: return launch_gate_km<D, 1>(pr, q, w, sel, counts, st);
@@ -561,6 +626,120 @@ __global__ void wait_selftest_kernel(uint32_t* status, long long limit_cycles) {
   mbar_wait(&bar, 0, &abort_flag, status, limit_cycles);
 }
 
+// ---------------------------------------------------------------- decode
+struct DecodeShape {
+  int b, cap, Hq, Hkv, G, D, B, topk, nbcap, nchunk;
+  float scale;
+};
+
+moba_status make_decode_shape(const moba_decode_params* p, DecodeShape* out) {
+  if (!p) return MOBA_ERR_INVALID_ARG;
+  DecodeShape d;
+  if (p->batch <= 0 || p->cache_len <= 0 || p->num_q_heads <= 0 || p->num_kv_heads <= 0 ||
+      p->num_q_heads % p->num_kv_heads || p->block_size <= 0 || p->top_k <= 0)
+    return MOBA_ERR_INVALID_ARG;
+  if (p->head_dim != 64 && p->head_dim != 128) return MOBA_ERR_UNSUPPORTED;
+  if (p->block_size % kTileM) return MOBA_ERR_UNSUPPORTED;
+  if (p->top_k > 65) return MOBA_ERR_UNSUPPORTED;  // at most 64 ranked past blocks
+  d.b = p->batch;
+  d.cap = p->cache_len;
+  d.Hq = p->num_q_heads;
+  d.Hkv = p->num_kv_heads;
+  d.G = d.Hq / d.Hkv;
+  d.D = p->head_dim;
+  d.B = p->block_size;
+  d.topk = p->top_k;
+  const int64_t nb = ((int64_t)d.cap + d.B - 1) / d.B;
+  if (nb > kDecodeMaxBlocks) return MOBA_ERR_UNSUPPORTED;
+  if ((int64_t)d.b * d.cap * d.Hkv * d.D >= (int64_t(1) << 40)) return MOBA_ERR_UNSUPPORTED;
+  if ((int64_t)d.b * d.Hq > 65535 * 1024) return MOBA_ERR_UNSUPPORTED;
+  d.nbcap = (int)nb;
+  d.nchunk = (d.B + kDecodeChunk - 1) / kDecodeChunk;
+  d.scale = (p->softmax_scale > 0.f) ? p->softmax_scale : 1.0f / sqrtf((float)d.D);
+  if (!(d.scale < INFINITY)) return MOBA_ERR_INVALID_ARG;
+  *out = d;
+  return MOBA_OK;
+}
+
+struct DecodeWs {
+  uint32_t* status;
+  int32_t* sel;
+  float* part;
+  size_t bytes;
+};
+
+DecodeWs carve_decode(const DecodeShape& d, char* base) {
+  DecodeWs w;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + bytes);
+    return p;
+  };
+  w.status = reinterpret_cast<uint32_t*>(take(kAlign));
+  w.sel = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)d.b * d.Hq * d.topk));
+  w.part = reinterpret_cast<float*>(
+      take(sizeof(float) * (size_t)d.b * d.Hq * d.topk * d.nchunk * (d.D + 2)));
+  w.bytes = off;
+  return w;
+}
+
+DecodeArgs decode_args(const DecodeShape& d, const DecodeWs& w, const void* q, const void* kc,
+                       const void* vc, const int32_t* lens, float* kbar) {
+  DecodeArgs a;
+  memset(&a, 0, sizeof a);
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.kc = reinterpret_cast<const __nv_bfloat16*>(kc);
+  a.vc = reinterpret_cast<const __nv_bfloat16*>(vc);
+  a.lens = lens;
+  a.kbar = kbar;
+  a.sel = w.sel;
+  a.part = w.part;
+  a.batch = d.b;
+  a.cap = d.cap;
+  a.Hq = d.Hq;
+  a.Hkv = d.Hkv;
+  a.G = d.G;
+  a.B = d.B;
+  a.topk = d.topk;
+  a.nbcap = d.nbcap;
+  a.nchunk = d.nchunk;
+  a.scale_log2 = d.scale * 1.4426950408889634f;
+  a.status = w.status;
+  return a;
+}
+
+template <int D>
+moba_status kbar_update_impl(const DecodeShape& d, const DecodeArgs& a, int only_last,
+                             cudaStream_t st) {
+  dim3 grid(only_last ? 1u : (unsigned)d.nbcap, (unsigned)d.Hkv, (unsigned)d.b);
+  Timed tm(kKKbarCache, st);
+  kbar_cache_kernel<D><<<grid, 128, 0, st>>>(a, only_last);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int D>
+moba_status decode_impl(const DecodeShape& d, DecodeArgs a, cudaStream_t st) {
+  const size_t gsmem = sizeof(float) * (size_t)d.nbcap;
+  {
+    Timed tm(kKDecGate, st);
+    decode_gate_kernel<D><<<dim3((unsigned)d.Hq, (unsigned)d.b), 256, gsmem, st>>>(a);
+    MOBA_CUDA(cudaGetLastError());
+  }
+  {
+    Timed tm(kKDecAttn, st);
+    decode_attn_kernel<D>
+        <<<dim3((unsigned)(d.b * d.Hq), (unsigned)d.topk, (unsigned)d.nchunk), 128, 0, st>>>(a);
+    MOBA_CUDA(cudaGetLastError());
+  }
+  {
+    Timed tm(kKDecMerge, st);
+    decode_merge_kernel<D><<<(unsigned)(d.b * d.Hq), D, 0, st>>>(a);
+    MOBA_CUDA(cudaGetLastError());
+  }
+  return MOBA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -717,6 +896,58 @@ int moba_profile_read(moba_kernel_time* out, int max_entries) {
     ++n;
   }
   return n;
+}
+
+// ---------------------------------------------------------------- decode
+size_t moba_decode_workspace_size(const moba_decode_params* p) {
+  DecodeShape d;
+  if (make_decode_shape(p, &d) != MOBA_OK) return 0;
+  return carve_decode(d, nullptr).bytes;
+}
+
+size_t moba_kbar_cache_size(const moba_decode_params* p) {
+  DecodeShape d;
+  if (make_decode_shape(p, &d) != MOBA_OK) return 0;
+  return sizeof(float) * (size_t)d.b * d.Hkv * d.nbcap * d.D;
+}
+
+moba_status moba_kbar_cache_update(const void* k_cache, const int32_t* seqlens,
+                                   float* kbar_cache, int only_last,
+                                   const moba_decode_params* p, void* ws, size_t ws_bytes,
+                                   moba_stream_t stream) {
+  DecodeShape d;
+  MOBA_TRY(make_decode_shape(p, &d));
+  if (!k_cache || !seqlens || !kbar_cache || !aligned16(k_cache) || !aligned16(kbar_cache) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3))
+    return MOBA_ERR_INVALID_ARG;
+  MOBA_TRY(check_ws(ws, ws_bytes, carve_decode(d, nullptr).bytes));
+  const DecodeWs w = carve_decode(d, static_cast<char*>(ws));
+  const DecodeArgs a = decode_args(d, w, nullptr, k_cache, nullptr, seqlens, kbar_cache);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return d.D == 128 ? kbar_update_impl<128>(d, a, only_last ? 1 : 0, st)
+                    : kbar_update_impl<64>(d, a, only_last ? 1 : 0, st);
+}
+
+moba_status moba_decode(const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* seqlens, const float* kbar_cache, void* o, float* lse,
+                        int32_t* sel_out, const moba_decode_params* p, void* ws,
+                        size_t ws_bytes, moba_stream_t stream) {
+  DecodeShape d;
+  MOBA_TRY(make_decode_shape(p, &d));
+  if (!q || !k_cache || !v_cache || !seqlens || !kbar_cache || !o || !lse)
+    return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(kbar_cache) ||
+      !aligned16(o) || (reinterpret_cast<uintptr_t>(seqlens) & 3) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3) || (reinterpret_cast<uintptr_t>(sel_out) & 3))
+    return MOBA_ERR_INVALID_ARG;
+  MOBA_TRY(check_ws(ws, ws_bytes, carve_decode(d, nullptr).bytes));
+  DecodeWs w = carve_decode(d, static_cast<char*>(ws));
+  if (sel_out) w.sel = sel_out;
+  DecodeArgs a = decode_args(d, w, q, k_cache, v_cache, seqlens, const_cast<float*>(kbar_cache));
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return d.D == 128 ? decode_impl<128>(d, a, st) : decode_impl<64>(d, a, st);
 }
 
 }  // extern "C"

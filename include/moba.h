@@ -140,6 +140,68 @@ moba_status moba_full_causal_varlen(const void *q, const void *k, const void *v,
                                     const moba_params *p, void *ws, size_t ws_bytes,
                                     moba_stream_t stream);
 
+/* ------------------------------------------------------------------ decode
+ * One decode step: a single new query per sequence against its KV cache.
+ * The new token of sequence b is at position t = seqlens[b] - 1 of the cache
+ * (its key and value already written there), in block i = t / block_size.
+ * Its selection and attention follow the same rules as the prefill (cited
+ * at the top of this file): scores against the means of blocks 0..i-1, the
+ * k-1 best kept (ties to the lower block), the own block i always kept,
+ * attention over the kept blocks with the own block ending at t.  The pages
+ * evaluate MoBA for prefill with full attention during generation
+ * (wispaper.ai blog, "Real-World LLM and Benchmark Evidence") and name its
+ * extension to generation as a next step ("Deep Insight and Conclusion");
+ * the operation here is exactly the prefill's last row, computed against a
+ * cache.
+ *
+ * Layouts (device memory, contiguous):
+ *   q        [batch][num_q_heads][head_dim] bf16: the new token's queries
+ *   k_cache, v_cache [batch][cache_len][num_kv_heads][head_dim] bf16
+ *   seqlens  [batch] int32: tokens in each cache, the new one included
+ *            (1 <= seqlens[b] <= cache_len; others latch MOBA_ERR_DEVICE_CHECK)
+ *   kbar     [batch][num_kv_heads][ceil(cache_len / block_size)][head_dim]
+ *            fp32: means of the complete blocks, kept by
+ *            moba_kbar_cache_update (moba_kbar_cache_size bytes)
+ *   o        [batch][num_q_heads][head_dim] bf16
+ *   lse      [batch][num_q_heads] fp32 (natural log)
+ *   sel_out  [batch][num_q_heads][top_k] int32, nullable: the kept blocks,
+ *            ascending, own block last, -1 padded
+ * Same ownership and error rules as above; top_k is at most 65. */
+typedef struct moba_decode_params {
+  int batch;           /* sequences */
+  int cache_len;       /* capacity of each sequence's cache, in tokens */
+  int num_q_heads;     /* Hq */
+  int num_kv_heads;    /* Hkv, divides Hq */
+  int head_dim;        /* 64 or 128 */
+  int block_size;      /* multiple of 128 */
+  int top_k;           /* 1 .. 65, the own block included */
+  float softmax_scale; /* <= 0 selects 1/sqrt(head_dim) */
+} moba_decode_params;
+
+/* Workspace bytes for moba_decode and moba_kbar_cache_update (0 if the
+ * parameters are invalid). */
+size_t moba_decode_workspace_size(const moba_decode_params *p);
+
+/* Bytes of the block-mean cache kbar. */
+size_t moba_kbar_cache_size(const moba_decode_params *p);
+
+/* Writes the mean of cache blocks into kbar.  only_last = 0: every complete
+ * block of each sequence (blocks j with (j + 1) * block_size <= seqlens[b]),
+ * e.g. after a prefill; only_last != 0: only the block the newest token
+ * completed (when seqlens[b] is a multiple of block_size), e.g. after each
+ * appended token.  Block means as defined above (wispaper.ai blog,
+ * "The Change"; sherconan.github.io step 1). */
+moba_status moba_kbar_cache_update(const void *k_cache, const int32_t *seqlens, float *kbar,
+                                   int only_last, const moba_decode_params *p, void *ws,
+                                   size_t ws_bytes, moba_stream_t stream);
+
+/* The decode step: o, lse and (optionally) sel for every sequence's new
+ * token. */
+moba_status moba_decode(const void *q, const void *k_cache, const void *v_cache,
+                        const int32_t *seqlens, const float *kbar, void *o, float *lse,
+                        int32_t *sel_out, const moba_decode_params *p, void *ws,
+                        size_t ws_bytes, moba_stream_t stream);
+
 /* Synchronises `stream`, returns and clears the device status latched in
  * `ws` by earlier calls (MOBA_OK, MOBA_ERR_TIMEOUT or MOBA_ERR_DEVICE_CHECK). */
 moba_status moba_last_device_status(void *ws, moba_stream_t stream);
@@ -147,9 +209,10 @@ moba_status moba_last_device_status(void *ws, moba_stream_t stream);
 /* Per-kernel timing, for benchmarks: while enabled, every kernel launch the
  * library makes is bracketed by CUDA events recorded on the launch stream.
  * moba_profile_read synchronises those events and returns, per kernel class
- * (plan, pool, gate, bucket_scan, bucket_scatter, attn_routed, attn_own,
- * merge, attn_dense), the launch count and summed device milliseconds since
- * the last reset.  Returns the number of classes written (<= max_entries).
+ * (plan, pool, gate, gate_count, bucket_scan, bucket_scatter, attn_routed,
+ * attn_own, merge, attn_dense, kbar_cache, decode_gate, decode_attn,
+ * decode_merge), the launch count and summed device milliseconds since the
+ * last reset.  Returns the number of classes written (<= max_entries).
  * Not thread safe; meant for one benchmarking thread. */
 typedef struct moba_kernel_time {
   char name[24];

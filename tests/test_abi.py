@@ -151,3 +151,51 @@ def test_selftest_argument_checks(lib):
     assert lib.moba_selftest_wait_timeout(fake, 4096, 0, None) == INVALID
     assert lib.moba_selftest_wait_timeout(fake, 4096, 10**12, None) == INVALID
     assert lib.moba_selftest_wait_timeout(fake, 16, 1000, None) == WORKSPACE
+
+
+def _dp(**kw):
+    d = dict(batch=2, cap=8192, Hq=8, Hkv=2, d=128, B=256, k=4)
+    d.update(kw)
+    return moba.make_decode_params(d["batch"], d["cap"], d["Hq"], d["Hkv"], d["d"], d["B"],
+                                   d["k"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), UNSUPPORTED),
+    (dict(B=100), UNSUPPORTED),
+    (dict(k=66), UNSUPPORTED),
+    (dict(k=0), INVALID),
+    (dict(Hq=6, Hkv=4), INVALID),
+    (dict(batch=0), INVALID),
+    (dict(cap=0), INVALID),
+    (dict(cap=256 * 8192 + 1), UNSUPPORTED),  # 8193 blocks of 256
+])
+def test_decode_bad_params_rejected(lib, kw, code):
+    p = _dp(**kw)
+    fake = ctypes.c_void_p(1 << 20)
+    rc = lib.moba_decode(fake, fake, fake, fake, fake, fake, fake, None, ctypes.byref(p), fake,
+                         1 << 40, None)
+    assert rc == code
+    assert moba.decode_workspace_size(p) == 0 and moba.kbar_cache_size(p) == 0
+
+
+def test_decode_pointer_and_workspace_checks(lib):
+    p = _dp()
+    fake = ctypes.c_void_p(1 << 20)
+    need = moba.decode_workspace_size(p)
+    assert need > 0
+    assert moba.kbar_cache_size(p) == 4 * 2 * 2 * (8192 // 256) * 128
+    args = [fake] * 8
+    for bad in range(7):  # q, k, v, seqlens, kbar, o, lse may not be null
+        a = list(args)
+        a[bad] = None
+        assert lib.moba_decode(*a, ctypes.byref(p), fake, need, None) == INVALID
+    a = list(args)
+    a[0] = ctypes.c_void_p((1 << 20) + 8)  # q not 16-byte aligned
+    assert lib.moba_decode(*a, ctypes.byref(p), fake, need, None) == INVALID
+    assert lib.moba_decode(*args, ctypes.byref(p), fake, need - 1, None) == WORKSPACE
+    assert lib.moba_decode(*args, ctypes.byref(p), None, need, None) == WORKSPACE
+    assert lib.moba_kbar_cache_update(fake, fake, fake, 0, ctypes.byref(p), fake, need - 1,
+                                      None) == WORKSPACE
+    assert lib.moba_kbar_cache_update(None, fake, fake, 0, ctypes.byref(p), fake, need,
+                                      None) == INVALID

@@ -189,6 +189,29 @@ def test_gate_only_matches_forward_selection(moba):
     assert torch.equal(sel_f, sel_g)
 
 
+@pytest.mark.parametrize("mode,k", [("all_equal", 5), ("pairs_equal", 4)])
+def test_gate_exact_ties(moba, mode, k):
+    """Blocks with equal key means give exactly equal scores, so the tie rule
+    (the lower block index wins) alone decides the kept set.  With every block
+    equal, rows past 24 blocks take the many-ties path of the gate; with equal
+    pairs, the cut falls inside a pair.  Checked exactly on every row against
+    the oracle's selection, with no near-tie exemption."""
+    N, Hq, Hkv, d, B = 4096, 4, 1, 128, 128
+    w = S.Workload("ties", [N], Hq, Hkv, d, B, k, seed=909)
+    q, kk, v = S.make_qkv(w, "cuda")
+    kb = kk.view(N // B, B, Hkv, d)
+    if mode == "all_equal":
+        kb[1:] = kb[0:1].clone()
+    else:
+        kb[1::2] = kb[0::2].clone()
+    sel = moba.gate(q.view(1, N, Hq, d), kk.view(1, N, Hkv, d), B, k)
+    torch.cuda.synchronize()
+    orc = Oracle(bf16_bits(q), bf16_bits(kk), bf16_bits(v), w.cu, Hq, Hkv, d, B, k)
+    osel, _, _ = orc.select(np.arange(N, dtype=np.int64))
+    gsel = sel[0].permute(1, 0, 2).cpu().numpy()
+    assert np.array_equal(gsel, osel)
+
+
 # ---------------------------------------------------------------- workloads
 def test_workload_tiny_all_rows(moba):
     stats = _check_forward(moba, S.TINY)
