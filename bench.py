@@ -301,6 +301,9 @@ def run_moba(args, w):
     clk = clocks.stop()
     kern = moba.profile_read()
     moba.profile_enable(False)
+    status = moba.last_device_status(ws)  # the timed steps' device checks
+    if status != 0:
+        print("device status %d after the timed steps" % status, file=sys.stderr)
     ms_local = e0.elapsed_time(e1) / args.steps
     ms = max_over_ranks(ms_local)
     value = world * flops / (ms / 1e3) / 1e12
@@ -520,6 +523,9 @@ def run_decode(args, w):
     clk = clocks.stop()
     kern = moba.profile_read()
     moba.profile_enable(False)
+    status = moba.last_device_status(ws)  # the timed steps' device checks
+    if status != 0:
+        print("device status %d after the timed steps" % status, file=sys.stderr)
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
     value = world * b / (ms / 1e3)
 
@@ -587,7 +593,7 @@ def run_decode(args, w):
         print(json.dumps(line), flush=True)
     if pg is not None:
         pg.destroy_process_group()
-    return 0
+    return 0 if status == 0 else 1
 
 
 def cpu_decode_baseline(w, qdec_bits, k_bits, v_bits, budget_s=15.0):

@@ -181,8 +181,12 @@ def pick_heads_per_pass(size_fn, num_kv_heads, budget=DEFAULT_WS_BUDGET):
 
 
 def alloc_workspace(nbytes, device=None):
+    """A workspace of nbytes whose status word (first 256 bytes) starts at zero,
+    as the library requires of a workspace's first use."""
     torch = _torch()
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+    ws[:256].zero_()
+    return ws
 
 
 def profile_enable(on=True):

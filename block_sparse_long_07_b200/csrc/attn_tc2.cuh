@@ -28,7 +28,10 @@
 // memory); the softmax reads S_X, keeps a running max / sum, writes P_X back
 // into TMEM; O_X += P_X V_j takes P_X straight from TMEM, so P never touches
 // shared memory.  The MMA thread alternates the sub-tiles, so one softmax
-// warpgroup works while the tensor core runs the other sub-tile's MMAs.
+// warpgroup works while the tensor core runs the other sub-tile's MMAs.  The
+// softmax signals once the first 64 keys of P_X are in TMEM (p_half) and
+// again when all are (p_full): the first half of the PV MMAs runs while the
+// second half of the exponentials is computed.
 // Tensor-core operations issued by one thread complete in issue order: when
 // S_X(j) is complete, PV_X(j-1) (issued before it) is too, which is what lets
 // the softmax rescale O_X right after seeing S_X(j).  The max is rescaled
@@ -78,7 +81,7 @@ struct Attn2Cfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = kOffQ + kQBufs * kQBytes;
   static constexpr int kOffBar = kOffKV + kStages * kKVBytes;
-  static constexpr int kNumBars = 2 * kQBufs + 2 * kStages + 2 + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 2 * kQBufs + 2 * kStages + 2 + 2 + 2 + 2 + 1 + 2;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false, false);
@@ -212,7 +215,7 @@ __device__ __forceinline__ float tile_row_max(uint32_t tS, int r) {
 // bounds this loop.
 template <bool MASK>
 __device__ __forceinline__ float tile_exp_to_p(uint32_t tS, int r, float scale_log2,
-                                               float m_use) {
+                                               float m_use, uint64_t* half_bar, int lane) {
   float sp[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) sp[e] = 0.f;
@@ -247,6 +250,12 @@ __device__ __forceinline__ float tile_exp_to_p(uint32_t tS, int r, float scale_l
       }
       tmem_st16(tS + h2 * 32 + q2 * 16, pk);
     }
+    if (h2 == 0) {  // P of keys 0..63 is in TMEM: the first half of PV may start
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(half_bar);
+    }
   }
   return ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
 }
@@ -273,7 +282,8 @@ __global__ void __launch_bounds__(352, 1)
   uint64_t* o_full = p_full + 2;        // [2] last PV_X of an item done
   uint64_t* o_free = o_full + 2;        // [2] epilogue has read O_X
   uint64_t* td_bar = o_free + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(td_bar + 1);
+  uint64_t* p_half = td_bar + 1;        // [2] first 64 keys of P_X in TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(p_half + 2);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -285,6 +295,7 @@ __global__ void __launch_bounds__(352, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
       mbar_init(&p_full[b], kTileM / 32);  // one elected arrival per softmax warp
+      mbar_init(&p_half[b], kTileM / 32);
       mbar_init(&o_full[b], 1);
       mbar_init(&o_free[b], kTileM / 32);
     }
@@ -432,10 +443,10 @@ __global__ void __launch_bounds__(352, 1)
       tc_commit_warp(&s_full[x]);
       if (x == 0) ++ns0; else ++ns1;
     };
-    auto issue_pv = [&](int x, uint32_t vs, bool acc) {
+    auto issue_pv = [&](int x, uint32_t vs, bool acc, int kk0, int kk1) {
       const uint32_t vbase = sKVa + vs * C::kKVBytes;
 #pragma unroll
-      for (int kk = 0; kk < kTileN / 16; ++kk)
+      for (int kk = kk0; kk < kk1; ++kk)
         tc_mma_ts_warp(tmem + C::col_o(x), tmem + C::col_s(x) + kk * 8,
                        sdesc_mnmajor_sw128(vbase + kk * 2048, C::kHalfBytes, 1024), C::kIdescPV,
                        (acc || kk > 0) ? 1u : 0u);
@@ -445,10 +456,13 @@ __global__ void __launch_bounds__(352, 1)
       if (j >= it.nkv_x[x]) return true;
       const uint32_t nsx = x == 0 ? ns0 : ns1;
       const uint32_t nox = x == 0 ? no0 : no1;
-      if (!wait(&p_full[x], (nsx - 1) & 1)) return false;  // P_X(j) is in TMEM
+      if (!wait(&p_half[x], (nsx - 1) & 1)) return false;  // keys 0..63 of P_X(j)
       if (j == 0 && nox > 0 && !wait(&o_free[x], (nox - 1) & 1)) return false;
       tc_fence_after();
-      issue_pv(x, vs, j > 0);
+      issue_pv(x, vs, j > 0, 0, kTileN / 32);
+      if (!wait(&p_full[x], (nsx - 1) & 1)) return false;  // all of P_X(j)
+      tc_fence_after();
+      issue_pv(x, vs, true, kTileN / 32, kTileN / 16);
       if (j == it.nkv_x[x] - 1) {
         tc_commit_warp(&o_full[x]);
         if (x == 0) ++no0; else ++no1;
@@ -527,8 +541,9 @@ __global__ void __launch_bounds__(352, 1)
             tmem_st32(tO + c4 * 32, ov);
           }
         }
-        const float sum = diag_tile ? tile_exp_to_p<true>(tS, r, a.scale_log2, m_use)
-                                    : tile_exp_to_p<false>(tS, r, a.scale_log2, m_use);
+        const float sum = diag_tile
+                              ? tile_exp_to_p<true>(tS, r, a.scale_log2, m_use, &p_half[x], lane)
+                              : tile_exp_to_p<false>(tS, r, a.scale_log2, m_use, &p_half[x], lane);
         l_run = l_run * alpha + sum;
         m_run = m_use;
         tc_wait_st();

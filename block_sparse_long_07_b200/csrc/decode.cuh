@@ -11,8 +11,8 @@
 // ("Efficiency and Implementation").
 //
 // Kernels:
-//   kbar_cache_kernel   block means of complete cache blocks (all of them, or
-//                       the one the newest token completed)
+//   kbar_part_kernel,   block means of complete cache blocks (all of them, or
+//   kbar_reduce_kernel  the one the newest token completed), split over CTAs
 //   decode_gate_kernel  per (sequence, q head): scores against every past
 //                       block mean, top-(k-1) by repeated block-wide argmax
 //                       (ties to the lower index), own block appended
@@ -39,7 +39,7 @@ struct DecodeArgs {
   const __nv_bfloat16* kc;      // [b][cap][Hkv][D]
   const __nv_bfloat16* vc;      // [b][cap][Hkv][D]
   const int32_t* lens;          // [b] tokens in the cache, the new one included
-  float* kbar;                  // [b][Hkv][nbcap][D] (written only by kbar_cache_kernel)
+  float* kbar;                  // [b][Hkv][nbcap][D] (written only by kbar_reduce_kernel)
   int32_t* sel;                 // [b][Hq][k]
   float* part;                  // [b][Hq][k][nchunk][D + 2]: O (unnormalised), m, l (log2)
   __nv_bfloat16* o;             // [b][Hq][D]
@@ -49,42 +49,68 @@ struct DecodeArgs {
   uint32_t* status;
 };
 
-// Mean of cache block j of (sequence b, kv head g) over its B tokens, in a
-// fixed order (rows split over 4 row groups, then added in group order).
-// Grid (blocks, Hkv, batch) for a full rebuild, or (1, Hkv, batch) for the
-// block completed by the newest token (nothing when len % B != 0).
-template <int D>
-__global__ void __launch_bounds__(128) kbar_cache_kernel(const DecodeArgs a, int only_last) {
-  constexpr int C4 = D / 4;           // float4 columns per row
-  constexpr int RG = 128 / C4;        // row groups
-  __shared__ float red[RG][D];
-  const int g = blockIdx.y, b = blockIdx.z;
+// Block means of the cache, in two deterministic steps.  kbar_part_kernel:
+// CTA (x = j_local * S + split, kv head, sequence) sums rows
+// [split * kKbarRows, (split + 1) * kKbarRows) of block j (4 row groups, 8
+// loads in flight per thread, groups added in order) into part[...][split].
+// kbar_reduce_kernel adds the S partials in split order and divides by B.
+// only_last = 0: every complete block (j < len / B); otherwise only the block
+// the newest token completed (j = len / B - 1 when len % B == 0).
+constexpr int kKbarRows = 128;  // rows per partial (block sizes are multiples of 128)
+
+__device__ __forceinline__ int kbar_block(const DecodeArgs& a, int b, int jl, int only_last,
+                                          bool report) {
   const int len = a.lens[b];
   if (len < 1 || len > a.cap) {
-    if (threadIdx.x == 0) atomicOr(a.status, MOBA_DEV_BAD_SEQLENS);
-    return;
+    if (report) atomicOr(a.status, MOBA_DEV_BAD_SEQLENS);
+    return -1;
   }
   int j;
   if (only_last) {
-    if (len % a.B != 0) return;
+    if (len % a.B != 0) return -1;
     j = len / a.B - 1;
   } else {
-    j = blockIdx.x;
-    if (j >= len / a.B) return;  // only complete blocks
+    j = jl;
+    if (j >= len / a.B) return -1;  // only complete blocks
   }
-  if (j >= a.nbcap) return;
+  return j < a.nbcap ? j : -1;
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) kbar_part_kernel(const DecodeArgs a, int only_last,
+                                                        float* __restrict__ part) {
+  constexpr int C4 = D / 4;     // 8-byte (4 x bf16) columns per row
+  constexpr int RG = 128 / C4;  // row groups
+  constexpr int U = 8;          // loads in flight
+  __shared__ float red[RG][D];
+  const int S = a.B / kKbarRows;
+  const int jl = blockIdx.x / S, sp = blockIdx.x % S;
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int j = kbar_block(a, b, jl, only_last, blockIdx.x == 0 && g == 0 && threadIdx.x == 0);
+  if (j < 0) return;
   const int c4 = threadIdx.x % C4, rg = threadIdx.x / C4;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   const size_t rstride = (size_t)a.Hkv * D;
-  const __nv_bfloat16* base = a.kc + (((size_t)b * a.cap + (size_t)j * a.B) * a.Hkv + g) * D + 4 * c4;
-  for (int r = rg; r < a.B; r += RG) {
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(base + (size_t)r * rstride));
-    const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
-    const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
-    acc[0] += f0.x;
-    acc[1] += f0.y;
-    acc[2] += f1.x;
-    acc[3] += f1.y;
+  const __nv_bfloat16* base =
+      a.kc + (((size_t)b * a.cap + (size_t)j * a.B + (size_t)sp * kKbarRows) * a.Hkv + g) * D +
+      4 * c4;
+  for (int r0 = rg; r0 < kKbarRows; r0 += RG * U) {
+    uint2 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int r = r0 + u * RG;
+      v[u] = r < kKbarRows ? __ldg(reinterpret_cast<const uint2*>(base + (size_t)r * rstride))
+                           : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v[u].x));
+      const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v[u].y));
+      acc[0] += f0.x;
+      acc[1] += f0.y;
+      acc[2] += f1.x;
+      acc[3] += f1.y;
+    }
   }
 #pragma unroll
   for (int e = 0; e < 4; ++e) red[rg][4 * c4 + e] = acc[e];
@@ -93,19 +119,32 @@ __global__ void __launch_bounds__(128) kbar_cache_kernel(const DecodeArgs a, int
     float s = 0.f;
 #pragma unroll
     for (int q = 0; q < RG; ++q) s += red[q][threadIdx.x];
-    a.kbar[(((size_t)b * a.Hkv + g) * a.nbcap + j) * D + threadIdx.x] = s / (float)a.B;
+    const int nsel = only_last ? 1 : a.nbcap;
+    part[((((size_t)b * a.Hkv + g) * nsel + (only_last ? 0 : j)) * S + sp) * D + threadIdx.x] = s;
   }
 }
 
-// Gate for the new token of (sequence b, q head h).  256 threads: scores of
-// the past blocks into shared memory, then k-1 rounds of block-wide argmax
-// by (score desc, index asc).
+template <int D>
+__global__ void __launch_bounds__(D) kbar_reduce_kernel(const DecodeArgs a, int only_last,
+                                                        const float* __restrict__ part) {
+  const int jl = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int j = kbar_block(a, b, jl, only_last, false);
+  if (j < 0) return;
+  const int S = a.B / kKbarRows;
+  const int nsel = only_last ? 1 : a.nbcap;
+  const float* src = part + (((size_t)b * a.Hkv + g) * nsel + (only_last ? 0 : j)) * S * D;
+  float s = 0.f;
+  for (int sp = 0; sp < S; ++sp) s += src[(size_t)sp * D + threadIdx.x];
+  a.kbar[(((size_t)b * a.Hkv + g) * a.nbcap + j) * D + threadIdx.x] = s / (float)a.B;
+}
+
+// Gate for the new token of (sequence b, q head h).  256 threads score the
+// past blocks into shared memory; warp 0 then takes k-1 rounds of argmax by
+// (score desc, index asc).
 template <int D>
 __global__ void __launch_bounds__(256) decode_gate_kernel(const DecodeArgs a) {
   extern __shared__ float dg_smem[];  // scores [nbcap]
   __shared__ float qs[D];
-  __shared__ float red_v[8];
-  __shared__ int red_j[8];
   __shared__ int chosen[64];
   const int h = blockIdx.x, b = blockIdx.y;
   const int g = h / a.G;
@@ -147,13 +186,16 @@ __global__ void __launch_bounds__(256) decode_gate_kernel(const DecodeArgs a) {
     dg_smem[j] = (s0 + s1) + (s2 + s3);
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x >= 32) return;
+  // warp 0: k-1 rounds of argmax by (score desc, index asc); a taken score
+  // becomes NaN, which no comparison selects again
+  const int lane = threadIdx.x;
   for (int round = 0; round < npast; ++round) {
     float bv = __int_as_float(0xff800000);
     int bj = 0x7fffffff;
-    for (int j = threadIdx.x; j < i; j += blockDim.x) {
+    for (int j = lane; j < i; j += 32) {
       const float v = dg_smem[j];
-      if (v > bv || (v == bv && j < bj)) {  // removed entries hold NaN: never taken
+      if (v > bv || (v == bv && j < bj)) {
         bv = v;
         bj = j;
       }
@@ -167,26 +209,13 @@ __global__ void __launch_bounds__(256) decode_gate_kernel(const DecodeArgs a) {
         bj = oj;
       }
     }
-    if (lane == 0) {
-      red_v[warp] = bv;
-      red_j[warp] = bj;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float v = red_v[0];
-      int jj = red_j[0];
-      for (int w = 1; w < 8; ++w)
-        if (red_v[w] > v || (red_v[w] == v && red_j[w] < jj)) {
-          v = red_v[w];
-          jj = red_j[w];
-        }
-      // a row of non-finite scores can leave nothing selectable
-      chosen[round] = (jj >= 0 && jj < i) ? jj : -1;
-      if (jj >= 0 && jj < i) dg_smem[jj] = __int_as_float(0x7fc00000);
-    }
-    __syncthreads();
+    // a row of non-finite scores can leave nothing selectable
+    const bool hit = bj >= 0 && bj < i;
+    if (lane == 0) chosen[round] = hit ? bj : -1;
+    if (hit && lane == (bj & 31)) dg_smem[bj] = __int_as_float(0x7fc00000);
+    __syncwarp();
   }
-  if (threadIdx.x == 0) {
+  if (lane == 0) {
     // ascending block order; an unfilled round (-1) sorts last
     for (int u = 1; u < npast; ++u) {
       const unsigned x = (unsigned)chosen[u];
@@ -341,23 +370,57 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
 }
 
 // O = sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p over the (slot, chunk)
-// partials in ascending order; lse = (M + log2 L) ln 2.
+// partials in ascending order; lse = (M + log2 L) ln 2.  The partials' m and
+// l are staged in shared memory; each thread then walks its output column
+// with 8 independent loads in flight.
+constexpr int kDecodeMaxParts = 65 * 64;  // top_k <= 65, chunks per block <= 64 staged
+
 template <int D>
 __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeArgs a) {
+  __shared__ float sw[kDecodeMaxParts];  // weight 2^(m_p - M), 0 for empty partials
+  __shared__ float red[D / 32];
+  __shared__ float sM;
   const int bh = blockIdx.x;
   const float* src = a.part + (size_t)bh * a.topk * a.nchunk * (D + 2);
   const int np = a.topk * a.nchunk;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float M = __int_as_float(0xff800000);
-  for (int p = 0; p < np; ++p) M = fmaxf(M, src[(size_t)p * (D + 2) + D]);
+  for (int p = threadIdx.x; p < np; p += D) {
+    const float mp = src[(size_t)p * (D + 2) + D];
+    sw[p] = mp;
+    M = fmaxf(M, mp);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = red[0];
+    for (int w = 1; w < D / 32; ++w) m = fmaxf(m, red[w]);
+    sM = m;
+  }
+  __syncthreads();
+  M = sM;
+  const bool any = M != __int_as_float(0xff800000);
+  for (int p = threadIdx.x; p < np; p += D) {
+    const float mp = sw[p];
+    sw[p] = (any && mp != __int_as_float(0xff800000)) ? ex2_approx(mp - M) : 0.f;
+  }
+  __syncthreads();
   float L = 0.f, O = 0.f;
-  if (M != __int_as_float(0xff800000)) {
-    for (int p = 0; p < np; ++p) {
-      const float* pp = src + (size_t)p * (D + 2);
-      const float mp = pp[D];
-      if (mp == __int_as_float(0xff800000)) continue;
-      const float f = ex2_approx(mp - M);
-      L += f * pp[D + 1];
-      O += f * pp[threadIdx.x];
+  for (int p0 = 0; p0 < np; p0 += 8) {
+    float ov[8], lv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int p = min(p0 + u, np - 1);
+      ov[u] = src[(size_t)p * (D + 2) + threadIdx.x];
+      lv[u] = src[(size_t)p * (D + 2) + D + 1];
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float wgt = (p0 + u < np) ? sw[p0 + u] : 0.f;
+      L = fmaf(wgt, lv[u], L);
+      O = fmaf(wgt, ov[u], O);
     }
   }
   const bool ok = L > 0.f;

@@ -655,6 +655,8 @@ moba_status make_decode_shape(const moba_decode_params* p, DecodeShape* out) {
   if ((int64_t)d.b * d.Hq > 65535 * 1024) return MOBA_ERR_UNSUPPORTED;
   d.nbcap = (int)nb;
   d.nchunk = (d.B + kDecodeChunk - 1) / kDecodeChunk;
+  if (d.b > 65535 || d.Hkv > 65535) return MOBA_ERR_UNSUPPORTED;          // grid y / z
+  if ((int64_t)d.topk * d.nchunk > kDecodeMaxParts) return MOBA_ERR_UNSUPPORTED;  // merge staging
   d.scale = (p->softmax_scale > 0.f) ? p->softmax_scale : 1.0f / sqrtf((float)d.D);
   if (!(d.scale < INFINITY)) return MOBA_ERR_INVALID_ARG;
   *out = d;
@@ -665,6 +667,7 @@ struct DecodeWs {
   uint32_t* status;
   int32_t* sel;
   float* part;
+  float* kpart;  // block-mean partial sums [b][Hkv][nbcap][B / 128][D]
   size_t bytes;
 };
 
@@ -680,6 +683,8 @@ DecodeWs carve_decode(const DecodeShape& d, char* base) {
   w.sel = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)d.b * d.Hq * d.topk));
   w.part = reinterpret_cast<float*>(
       take(sizeof(float) * (size_t)d.b * d.Hq * d.topk * d.nchunk * (d.D + 2)));
+  w.kpart = reinterpret_cast<float*>(take(sizeof(float) * (size_t)d.b * d.Hkv * d.nbcap *
+                                          (d.B / kKbarRows) * d.D));
   w.bytes = off;
   return w;
 }
@@ -710,11 +715,16 @@ DecodeArgs decode_args(const DecodeShape& d, const DecodeWs& w, const void* q, c
 }
 
 template <int D>
-moba_status kbar_update_impl(const DecodeShape& d, const DecodeArgs& a, int only_last,
-                             cudaStream_t st) {
-  dim3 grid(only_last ? 1u : (unsigned)d.nbcap, (unsigned)d.Hkv, (unsigned)d.b);
+moba_status kbar_update_impl(const DecodeShape& d, const DecodeArgs& a, float* kpart,
+                             int only_last, cudaStream_t st) {
+  const unsigned nsel = only_last ? 1u : (unsigned)d.nbcap;
+  const unsigned S = (unsigned)(d.B / kKbarRows);
   Timed tm(kKKbarCache, st);
-  kbar_cache_kernel<D><<<grid, 128, 0, st>>>(a, only_last);
+  kbar_part_kernel<D><<<dim3(nsel * S, (unsigned)d.Hkv, (unsigned)d.b), 128, 0, st>>>(
+      a, only_last, kpart);
+  MOBA_CUDA(cudaGetLastError());
+  kbar_reduce_kernel<D><<<dim3(nsel, (unsigned)d.Hkv, (unsigned)d.b), D, 0, st>>>(a, only_last,
+                                                                                kpart);
   return cuda_status(cudaGetLastError());
 }
 
@@ -924,8 +934,8 @@ moba_status moba_kbar_cache_update(const void* k_cache, const int32_t* seqlens,
   const DecodeWs w = carve_decode(d, static_cast<char*>(ws));
   const DecodeArgs a = decode_args(d, w, nullptr, k_cache, nullptr, seqlens, kbar_cache);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return d.D == 128 ? kbar_update_impl<128>(d, a, only_last ? 1 : 0, st)
-                    : kbar_update_impl<64>(d, a, only_last ? 1 : 0, st);
+  return d.D == 128 ? kbar_update_impl<128>(d, a, w.kpart, only_last ? 1 : 0, st)
+                    : kbar_update_impl<64>(d, a, w.kpart, only_last ? 1 : 0, st);
 }
 
 moba_status moba_decode(const void* q, const void* k_cache, const void* v_cache,

@@ -40,9 +40,12 @@
  *
  * Errors: invalid arguments are reported before anything is launched.
  * Errors found on the device (a stuck pipeline wait, malformed cu_seqlens,
- * an out-of-range selection) are latched in the workspace's status word and
- * reported by moba_last_device_status().  Nothing crosses the ABI as an
- * exception.
+ * an out-of-range selection) are latched in the workspace's status word (its
+ * first 4 bytes) and reported, and cleared, by moba_last_device_status().
+ * The word accumulates over calls, so it must be zero when a workspace is
+ * first used: zero the first 256 bytes of a new workspace (or call
+ * moba_last_device_status once and discard the result).  Nothing crosses the
+ * ABI as an exception.
  */
 #ifndef MOBA_H
 #define MOBA_H

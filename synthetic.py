@@ -71,7 +71,15 @@ VARLEN = Workload("varlen_8seq", varlen_lengths(4, 8, 4096, 65536, 256), 32, 8, 
                   seed=4, batch_mode=False,
                   note="8 packed sequences, lengths U[4096,65536] rounded to 256, B=512, k=8")
 
-WORKLOADS = {w.name: w for w in (TINY, FINE_32K, LONG_128K, MILLION, VARLEN)}
+# The 10M-token setting (wispaper.ai blog, "Efficiency and Implementation":
+# n = 256 blocks and k fixed, B grown to 10M / 256 = 40960) does not fit one
+# GPU at 32 q heads; sharded by kv-head group across 8 GPUs, each GPU holds
+# one kv head and its 4 q heads.  This is that per-GPU shard.
+PREFILL_10M_SHARD = Workload("prefill_10m_shard", [10485760], 4, 1, 128, 40960, 12, seed=5,
+                             note="one kv-head group (4 q / 1 kv head) of the 32 q / 8 kv "
+                                  "model at N=10485760, B=40960 (256 blocks), k=12")
+
+WORKLOADS = {w.name: w for w in (TINY, FINE_32K, LONG_128K, MILLION, VARLEN, PREFILL_10M_SHARD)}
 
 
 def block_ids(lengths: List[int], B: int) -> np.ndarray:

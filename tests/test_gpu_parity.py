@@ -231,6 +231,17 @@ def test_workload_sampled_rows(moba, name):
 
 @pytest.mark.slow
 @pytest.mark.timeout(3600)
+def test_workload_10m_shard_sampled_rows(moba):
+    """One kv-head shard of the 10M-token setting (4 q heads, B = 40960), in
+    the benchmark's launch configuration, on a seeded sample of rows."""
+    w = S.PREFILL_10M_SHARD
+    rows = S.sample_rows(w, max(64, PARITY_ROWS // 8))
+    stats = _check_forward(moba, w, rows=rows, label=w.name)
+    print(w.name, stats)
+
+
+@pytest.mark.slow
+@pytest.mark.timeout(3600)
 @pytest.mark.parametrize("name", ["fine_32k", "long_128k"])
 def test_workload_dense_sampled_rows(moba, name):
     w = S.WORKLOADS[name]
