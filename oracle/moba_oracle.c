@@ -26,7 +26,10 @@
  *     selected blocks, causal inside the own block
  *     (wispaper.ai blog, "Starting Point" and "The Change";
  *     globaladvisors.biz, "Underlying computational mechanism");
- *   - the log-sum-exp of the scaled logits over I (natural log).
+ *   - the log-sum-exp of the scaled logits over I (natural log);
+ *   - the backward of that attention over a fixed selection (dQ, dK, dV for
+ *     an output gradient dO): no gradient passes through the hard gate
+ *     (wispaper.ai blog, "The Change").
  *
  * The attention is evaluated directly over I, never block by block, so the
  * GPU's block-wise online-softmax merge is checked against a result that
@@ -386,6 +389,145 @@ int oracle_attend(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const
         free(z);
         free(idx);
         free(qd);
+    }
+    return err;
+}
+
+/*
+ * Backward of oracle_attend over a fixed selection.  The top-k gate is a hard
+ * choice through which no gradient flows (wispaper.ai blog, "The Change":
+ * the gradient does not pass through the discrete selection), so the
+ * gradient is that of exact softmax attention over each row's key set I.
+ * For each listed row r and head h (kv head g), with I as in oracle_attend
+ * and z_u = scale * q.k_u, lse = log sum_u exp(z_u), P_u = exp(z_u - lse),
+ * O = sum_u P_u v_u, and the output gradient dO (bf16 bits):
+ *   D      = dO . O
+ *   dS_u   = P_u (dO . v_u - D)          (softmax Jacobian applied to dO V^T)
+ *   dQ[r,h] = scale * sum_u dS_u k_u
+ *   dK[u,g] += scale * dS_u q
+ *   dV[u,g] += P_u dO
+ * dQ [nrows][Hq][d]; dK, dV [T][Hkv][d] (zeroed here, then summed over the
+ * listed rows and the q heads of each kv head).  All fp64.  Work is split by
+ * kv head; rows are visited in the listed order, so sums are deterministic.
+ */
+int oracle_attend_backward(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                           const int64_t *cu, int nseq, int Hq, int Hkv, int d, int B, int k,
+                           double scale, const int64_t *rows, int64_t nrows, const int32_t *sel,
+                           const uint16_t *dO, double *dQ, double *dK, double *dV)
+{
+    if (check_common(cu, nseq, Hq, Hkv, d, B) || !Q || !K || !V || !rows || !sel || !dO ||
+        !dQ || !dK || !dV || k <= 0)
+        return ORC_EINVAL;
+    int64_t T = cu[nseq];
+    int G = Hq / Hkv;
+    int err = ORC_OK;
+    memset(dK, 0, sizeof(double) * (size_t)T * Hkv * d);
+    memset(dV, 0, sizeof(double) * (size_t)T * Hkv * d);
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= T)
+            return ORC_EINVAL;
+
+#pragma omp parallel for schedule(dynamic)
+    for (int g = 0; g < Hkv; ++g) {
+        size_t cap = (size_t)k * (size_t)B + 1;
+        double *p = (double *)malloc(sizeof(double) * cap);
+        int64_t *idx = (int64_t *)malloc(sizeof(int64_t) * cap);
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+        double *od = (double *)malloc(sizeof(double) * (size_t)d);
+        double *gd = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!p || !idx || !qd || !od || !gd) {
+#pragma omp atomic write
+            err = ORC_ENOMEM;
+        } else {
+            for (int64_t r = 0; r < nrows; ++r) {
+                int64_t t = rows[r];
+                int s = seq_of(cu, nseq, t);
+                int64_t i = (t - cu[s]) / B;
+                for (int hh = 0; hh < G; ++hh) {
+                    int h = g * G + hh;
+                    const int32_t *sr = sel + ((size_t)r * Hq + h) * k;
+                    size_t m = 0;
+                    int bad = 0;
+                    for (int u = 0; u < k; ++u) {
+                        int64_t j = sr[u];
+                        if (j < 0)
+                            continue;
+                        if (j > i) {
+                            bad = 1;
+                            break;
+                        }
+                        int64_t a = cu[s] + j * B;
+                        int64_t e = (j == i) ? (t + 1) : (a + B);
+                        if (e > cu[s + 1])
+                            e = cu[s + 1];
+                        for (int64_t u2 = a; u2 < e; ++u2)
+                            idx[m++] = u2;
+                    }
+                    if (bad) {
+#pragma omp atomic write
+                        err = ORC_EFUTURE;
+                        continue;
+                    }
+                    const uint16_t *qr = Q + ((size_t)t * Hq + h) * d;
+                    const uint16_t *gr = dO + ((size_t)r * Hq + h) * d;
+                    for (int c = 0; c < d; ++c) {
+                        qd[c] = bf16_bits_to_double(qr[c]);
+                        gd[c] = bf16_bits_to_double(gr[c]);
+                        od[c] = 0.0;
+                    }
+                    /* probabilities over I */
+                    double zmax = -INFINITY;
+                    for (size_t u = 0; u < m; ++u) {
+                        const uint16_t *kr = K + ((size_t)idx[u] * Hkv + g) * d;
+                        double acc = 0.0;
+                        for (int c = 0; c < d; ++c)
+                            acc += qd[c] * bf16_bits_to_double(kr[c]);
+                        p[u] = acc * scale;
+                        if (p[u] > zmax)
+                            zmax = p[u];
+                    }
+                    double den = 0.0;
+                    for (size_t u = 0; u < m; ++u) {
+                        p[u] = exp(p[u] - zmax);
+                        den += p[u];
+                    }
+                    for (size_t u = 0; u < m; ++u)
+                        p[u] /= den;
+                    /* O and D = dO . O */
+                    for (size_t u = 0; u < m; ++u) {
+                        const uint16_t *vr = V + ((size_t)idx[u] * Hkv + g) * d;
+                        for (int c = 0; c < d; ++c)
+                            od[c] += p[u] * bf16_bits_to_double(vr[c]);
+                    }
+                    double D = 0.0;
+                    for (int c = 0; c < d; ++c)
+                        D += gd[c] * od[c];
+                    double *dq = dQ + ((size_t)r * Hq + h) * d;
+                    for (int c = 0; c < d; ++c)
+                        dq[c] = 0.0;
+                    for (size_t u = 0; u < m; ++u) {
+                        const uint16_t *kr = K + ((size_t)idx[u] * Hkv + g) * d;
+                        const uint16_t *vr = V + ((size_t)idx[u] * Hkv + g) * d;
+                        double dp = 0.0;
+                        for (int c = 0; c < d; ++c)
+                            dp += gd[c] * bf16_bits_to_double(vr[c]);
+                        double ds = p[u] * (dp - D);
+                        double *dkr = dK + ((size_t)idx[u] * Hkv + g) * d;
+                        double *dvr = dV + ((size_t)idx[u] * Hkv + g) * d;
+                        for (int c = 0; c < d; ++c) {
+                            dq[c] += scale * ds * bf16_bits_to_double(kr[c]);
+                            dkr[c] += scale * ds * qd[c];
+                            dvr[c] += p[u] * gd[c];
+                        }
+                    }
+                }
+            }
+        }
+        free(p);
+        free(idx);
+        free(qd);
+        free(od);
+        free(gd);
     }
     return err;
 }

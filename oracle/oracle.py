@@ -44,6 +44,9 @@ def _load():
         lib.oracle_attend.restype = i32
         lib.oracle_attend.argtypes = [p, p, p, p, i32, i32, i32, i32, i32, i32, dbl,
                                       p, i64, p, p, p, p]
+        lib.oracle_attend_backward.restype = i32
+        lib.oracle_attend_backward.argtypes = [p, p, p, p, i32, i32, i32, i32, i32, i32, dbl,
+                                               p, i64, p, p, p, p, p]
         lib.oracle_dense_causal.restype = i32
         lib.oracle_dense_causal.argtypes = [p, p, p, p, i32, i32, i32, i32, dbl, p, i64,
                                             p, p]
@@ -172,6 +175,28 @@ class Oracle:
         if rc:
             raise RuntimeError("oracle_attend failed: %d" % rc)
         return O, lse, nk
+
+    def attend_backward(self, rows, sel, dO_bits):
+        """Gradients of the attention over a fixed selection (the gate passes
+        none): dQ [R][Hq][d] for the listed rows, and dK, dV [T][Hkv][d]
+        summed over the listed rows.  dO_bits: bf16 bits [R][Hq][d]."""
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        sel = np.ascontiguousarray(sel, dtype=np.int32)
+        dO_bits = np.ascontiguousarray(dO_bits, dtype=np.uint16)
+        R = len(rows)
+        assert sel.shape[:2] == (R, self.Hq) and dO_bits.shape == (R, self.Hq, self.d)
+        T = int(self.cu[-1])
+        dQ = np.zeros((R, self.Hq, self.d), dtype=np.float64)
+        dK = np.zeros((T, self.Hkv, self.d), dtype=np.float64)
+        dV = np.zeros((T, self.Hkv, self.d), dtype=np.float64)
+        rc = self.lib.oracle_attend_backward(_ptr(self.q), _ptr(self.k), _ptr(self.v),
+                                             _ptr(self.cu), self.nseq, self.Hq, self.Hkv,
+                                             self.d, self.B, sel.shape[2], self.scale,
+                                             _ptr(rows), R, _ptr(sel), _ptr(dO_bits), _ptr(dQ),
+                                             _ptr(dK), _ptr(dV))
+        if rc:
+            raise RuntimeError("oracle_attend_backward failed: %d" % rc)
+        return dQ, dK, dV
 
     def forward(self, rows):
         """Gate then attention: O [R][Hq][d], lse [R][Hq], sel, margin, maxabs."""
