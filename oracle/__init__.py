@@ -5,4 +5,5 @@ by the benchmark's CPU-baseline leg, never by the product path.
 """
 from .oracle import (  # noqa: F401
     Oracle, bf16_bits, online_softmax_merge, cu_from_lengths, local_block_info,
+    static_selection,
 )

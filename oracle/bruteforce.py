@@ -42,36 +42,60 @@ def blocks_of_sequence(start, end, B):
     return out
 
 
-def brute_select(qf, kf, cu, Hq, Hkv, B, k):
-    """sel[t][h] = sorted tuple of local block ids, for every token t."""
+def _best_subset(score, i, k):
+    """Admissible subset (own block i plus min(k, i+1) - 1 past blocks) of
+    largest total past score, ties to the lexicographically smallest."""
+    size = min(k, i + 1)
+    best = None
+    for sub in itertools.combinations(range(i), size - 1):
+        tot = sum((score[j] for j in sub), Fraction(0))
+        cand = tuple(sorted(sub + (i,)))
+        if best is None or tot > best[0] or (tot == best[0] and cand < best[1]):
+            best = (tot, cand)
+    return best[1]
+
+
+def _brute_select_by(block_score, qf, kf, cu, Hq, Hkv, B, k):
     T = int(cu[-1])
     G = Hq // Hkv
     sel = [[None] * Hq for _ in range(T)]
     for s in range(len(cu) - 1):
         blocks = blocks_of_sequence(int(cu[s]), int(cu[s + 1]), B)
-        # exact block means per kv head
-        means = []
-        for g in range(Hkv):
-            mg = []
-            for (a, e) in blocks:
-                tot = [sum(kf[t, g, c] for t in range(a, e)) for c in range(kf.shape[2])]
-                mg.append([x / (e - a) for x in tot])
-            means.append(mg)
         for t in range(int(cu[s]), int(cu[s + 1])):
             i = (t - int(cu[s])) // B
             for h in range(Hq):
                 g = h // G
-                score = {j: sum(qf[t, h, c] * means[g][j][c] for c in range(qf.shape[2]))
-                         for j in range(i)}
-                size = min(k, i + 1)
-                best = None
-                for sub in itertools.combinations(range(i), size - 1):
-                    tot = sum((score[j] for j in sub), Fraction(0))
-                    cand = tuple(sorted(sub + (i,)))
-                    if best is None or tot > best[0] or (tot == best[0] and cand < best[1]):
-                        best = (tot, cand)
-                sel[t][h] = best[1]
+                score = {j: block_score(qf[t, h], kf, g, blocks[j]) for j in range(i)}
+                sel[t][h] = _best_subset(score, i, k)
     return sel
+
+
+def _mean_score(qv, kf, g, blk):
+    a, e = blk
+    d = kf.shape[2]
+    return sum(qv[c] * sum(kf[t, g, c] for t in range(a, e)) / (e - a) for c in range(d))
+
+
+def _minmax_score(qv, kf, g, blk):
+    a, e = blk
+    d = kf.shape[2]
+    tot = Fraction(0)
+    for c in range(d):
+        col = [kf[t, g, c] for t in range(a, e)]
+        tot += max(qv[c] * max(col), qv[c] * min(col))
+    return tot
+
+
+def brute_select(qf, kf, cu, Hq, Hkv, B, k):
+    """sel[t][h] = sorted tuple of local block ids, for every token t (mean
+    pooling: s_j = q . mean of block j's keys, exact rationals)."""
+    return _brute_select_by(_mean_score, qf, kf, cu, Hq, Hkv, B, k)
+
+
+def brute_select_minmax(qf, kf, cu, Hq, Hkv, B, k):
+    """The same with min/max pooling: s_j = sum_c max(q_c max_t k_tc,
+    q_c min_t k_tc) over block j's keys, exact rationals."""
+    return _brute_select_by(_minmax_score, qf, kf, cu, Hq, Hkv, B, k)
 
 
 def mask_from_selection(sel_t_h, cu, B, T):

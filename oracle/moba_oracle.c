@@ -163,6 +163,49 @@ int oracle_block_means(const uint16_t *K, const int64_t *cu, int nseq, int Hkv, 
     return ORC_OK;
 }
 
+/*
+ * Min / max pooled block keys, the Quest-style block representation the pages
+ * name as a MoBA variant (elamur summary card, "Key points": Quest as MoBA
+ * with smaller blocks and min/max pooling).  Kmax, Kmin [Hkv][NB][d]: the
+ * elementwise maximum and minimum of the keys present in each block.
+ */
+int oracle_block_minmax(const uint16_t *K, const int64_t *cu, int nseq, int Hkv, int d, int B,
+                        double *Kmax, double *Kmin)
+{
+    if (check_common(cu, nseq, Hkv, Hkv, d, B) || !K || !Kmax || !Kmin)
+        return ORC_EINVAL;
+    int64_t NB = oracle_total_blocks(cu, nseq, B);
+    int64_t blk = 0;
+    for (int s = 0; s < nseq; ++s) {
+        int64_t nb = seq_blocks(cu, s, B);
+        for (int64_t j = 0; j < nb; ++j, ++blk) {
+            int64_t t0 = cu[s] + j * B;
+            int64_t t1 = t0 + B;
+            if (t1 > cu[s + 1])
+                t1 = cu[s + 1];
+            for (int g = 0; g < Hkv; ++g) {
+                double *mx = Kmax + ((size_t)g * NB + blk) * d;
+                double *mn = Kmin + ((size_t)g * NB + blk) * d;
+                for (int c = 0; c < d; ++c) {
+                    mx[c] = -INFINITY;
+                    mn[c] = INFINITY;
+                }
+                for (int64_t t = t0; t < t1; ++t) {
+                    const uint16_t *kr = K + ((size_t)t * Hkv + g) * d;
+                    for (int c = 0; c < d; ++c) {
+                        double x = bf16_bits_to_double(kr[c]);
+                        if (x > mx[c])
+                            mx[c] = x;
+                        if (x < mn[c])
+                            mn[c] = x;
+                    }
+                }
+            }
+        }
+    }
+    return ORC_OK;
+}
+
 typedef struct {
     double s;
     int64_t j;
@@ -195,9 +238,10 @@ static int cmp_i32(const void *a, const void *b)
  *   maxabs [nrows][Hq]     max |s_j| over the past blocks (0 if none).
  * margin and maxabs may be NULL.
  */
-int oracle_select(const uint16_t *Q, const double *Kbar, const int64_t *cu, int nseq, int Hq,
-                  int Hkv, int d, int B, int k, const int64_t *rows, int64_t nrows,
-                  int32_t *sel, double *margin, double *maxabs)
+static int select_impl(const uint16_t *Q, const double *Kbar, const double *Kmin,
+                       const int64_t *cu, int nseq, int Hq, int Hkv, int d, int B, int k,
+                       const int64_t *rows, int64_t nrows, int32_t *sel, double *margin,
+                       double *maxabs)
 {
     if (check_common(cu, nseq, Hq, Hkv, d, B) || !Q || !Kbar || !rows || !sel || k <= 0)
         return ORC_EINVAL;
@@ -240,8 +284,16 @@ int oracle_select(const uint16_t *Q, const double *Kbar, const int64_t *cu, int 
             for (int64_t j = 0; j < i; ++j) {
                 const double *kb = Kbar + ((size_t)g * NB + first + j) * d;
                 double acc = 0.0;
-                for (int c = 0; c < d; ++c)
-                    acc += qd[c] * kb[c];
+                if (!Kmin) { /* mean pooling: s_j = q . Kbar_j */
+                    for (int c = 0; c < d; ++c)
+                        acc += qd[c] * kb[c];
+                } else { /* min/max pooling: s_j = sum_c max(q_c Kmax_jc, q_c Kmin_jc) */
+                    const double *kn = Kmin + ((size_t)g * NB + first + j) * d;
+                    for (int c = 0; c < d; ++c) {
+                        double a = qd[c] * kb[c], b2 = qd[c] * kn[c];
+                        acc += (a > b2) ? a : b2;
+                    }
+                }
                 buf[j].s = acc;
                 buf[j].j = j;
                 if (fabs(acc) > mx)
@@ -275,6 +327,33 @@ int oracle_select(const uint16_t *Q, const double *Kbar, const int64_t *cu, int 
         free(qd);
     }
     return err;
+}
+
+int oracle_select(const uint16_t *Q, const double *Kbar, const int64_t *cu, int nseq, int Hq,
+                  int Hkv, int d, int B, int k, const int64_t *rows, int64_t nrows,
+                  int32_t *sel, double *margin, double *maxabs)
+{
+    return select_impl(Q, Kbar, NULL, cu, nseq, Hq, Hkv, d, B, k, rows, nrows, sel, margin,
+                       maxabs);
+}
+
+/*
+ * The same gate with the min/max-pooled block representation: the score of
+ * past block j is sum_c max(q_c Kmax_jc, q_c Kmin_jc), the largest q . x over
+ * the box spanned by the block's keys (so at least max over the block's keys
+ * of q . k; Quest's criticality bound, the scoring of the method the pages
+ * frame as MoBA with min/max pooling).  Same top-k, causality and tie rules,
+ * same margin / maxabs outputs.
+ */
+int oracle_select_minmax(const uint16_t *Q, const double *Kmax, const double *Kmin,
+                         const int64_t *cu, int nseq, int Hq, int Hkv, int d, int B, int k,
+                         const int64_t *rows, int64_t nrows, int32_t *sel, double *margin,
+                         double *maxabs)
+{
+    if (!Kmin)
+        return ORC_EINVAL;
+    return select_impl(Q, Kmax, Kmin, cu, nseq, Hq, Hkv, d, B, k, rows, nrows, sel, margin,
+                       maxabs);
 }
 
 /*

@@ -41,6 +41,11 @@ def _load():
         lib.oracle_select.restype = i32
         lib.oracle_select.argtypes = [p, p, p, i32, i32, i32, i32, i32, i32, p, i64,
                                       p, p, p]
+        lib.oracle_block_minmax.restype = i32
+        lib.oracle_block_minmax.argtypes = [p, p, i32, i32, i32, i32, p, p]
+        lib.oracle_select_minmax.restype = i32
+        lib.oracle_select_minmax.argtypes = [p, p, p, p, i32, i32, i32, i32, i32, i32, p, i64,
+                                             p, p, p]
         lib.oracle_attend.restype = i32
         lib.oracle_attend.argtypes = [p, p, p, p, i32, i32, i32, i32, i32, i32, dbl,
                                       p, i64, p, p, p, p]
@@ -107,6 +112,31 @@ def online_softmax_merge(parts_O, parts_lse):
     return out, m + np.log(den)
 
 
+def static_selection(cu, rows, B, k, mode):
+    """Static routings the pages describe as fixed corners of the MoBA gate
+    (wispaper.ai blog, "Why the Change Is Plausible"): "window" keeps the
+    own block and the k-1 most recent past blocks; "sink" keeps block 0, the
+    k-2 most recent past blocks and the own block.  With fewer than k blocks
+    every block is kept, as the gate does.  Returns sel [R][k] (local block
+    ids ascending, -1 padded); the same for every head."""
+    cu = np.asarray(cu, dtype=np.int64)
+    rows = np.asarray(rows, dtype=np.int64)
+    out = np.full((len(rows), k), -1, dtype=np.int32)
+    for r, t in enumerate(rows):
+        s = int(np.searchsorted(cu, t, side="right") - 1)
+        i = int((t - cu[s]) // B)
+        npast = min(k - 1, i)
+        if mode == "window" or npast == i or npast == 0:
+            past = list(range(i - npast, i))
+        elif mode == "sink":
+            past = [0] + list(range(i - npast + 1, i))
+        else:
+            raise ValueError(mode)
+        blocks = past + [i]
+        out[r, :len(blocks)] = blocks
+    return out
+
+
 class Oracle:
     """fp64 reference for one problem (one set of q, k, v and parameters)."""
 
@@ -156,6 +186,35 @@ class Oracle:
                                     _ptr(rows), R, _ptr(sel), _ptr(margin), _ptr(maxabs))
         if rc:
             raise RuntimeError("oracle_select failed: %d" % rc)
+        return sel, margin, maxabs
+
+    def block_minmax(self):
+        """(Kmax, Kmin) [Hkv][NB][d]: elementwise max / min of each block's keys."""
+        if getattr(self, "_kminmax", None) is None:
+            kx = np.zeros((self.Hkv, self.total_blocks, self.d), dtype=np.float64)
+            kn = np.zeros_like(kx)
+            rc = self.lib.oracle_block_minmax(_ptr(self.k), _ptr(self.cu), self.nseq, self.Hkv,
+                                              self.d, self.B, _ptr(kx), _ptr(kn))
+            if rc:
+                raise RuntimeError("oracle_block_minmax failed: %d" % rc)
+            self._kminmax = (kx, kn)
+        return self._kminmax
+
+    def select_minmax(self, rows):
+        """The gate with min/max-pooled blocks (score sum_c max(q_c Kmax_c, q_c Kmin_c)):
+        sel, margin, maxabs as select()."""
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        R = len(rows)
+        kx, kn = self.block_minmax()
+        sel = np.zeros((R, self.Hq, self.topk), dtype=np.int32)
+        margin = np.zeros((R, self.Hq), dtype=np.float64)
+        maxabs = np.zeros((R, self.Hq), dtype=np.float64)
+        rc = self.lib.oracle_select_minmax(_ptr(self.q), _ptr(kx), _ptr(kn), _ptr(self.cu),
+                                           self.nseq, self.Hq, self.Hkv, self.d, self.B,
+                                           self.topk, _ptr(rows), R, _ptr(sel), _ptr(margin),
+                                           _ptr(maxabs))
+        if rc:
+            raise RuntimeError("oracle_select_minmax failed: %d" % rc)
         return sel, margin, maxabs
 
     def attend(self, rows, sel):
