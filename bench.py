@@ -267,11 +267,26 @@ def run_moba(args, w):
     lse = torch.empty((w.Hq, T) if varlen else (len(w.lengths), w.Hq, w.lengths[0]),
                       dtype=torch.float32, device=dev)
 
+    route = getattr(args, "route", "gate")
+    if route != "gate" and varlen:
+        raise SystemExit("--route other than gate takes a batch workload")
+    rsel = None
+    if route != "gate":
+        rsel = torch.empty(len(w.lengths), w.Hq, w.lengths[0], w.k, dtype=torch.int32,
+                           device=dev)
+
     def step():
         if varlen:
             moba.forward_varlen(q, k, v, cu, w.B, w.k, ws=ws, out=o, lse=lse)
-        else:
+        elif route == "gate":
             moba.forward(q, k, v, w.B, w.k, ws=ws, out=o, lse=lse)
+        elif route == "minmax":
+            moba.forward_minmax(q, k, v, w.B, w.k, ws=ws, out=o, lse=lse, sel_out=rsel)
+        else:  # window / sink: the static selection is part of the step
+            moba.static_selection(len(w.lengths), w.lengths[0], w.Hq, w.B, w.k,
+                                  moba.ROUTE_WINDOW if route == "window" else moba.ROUTE_SINK,
+                                  sel=rsel)
+            moba.forward_selected(q, k, v, rsel, w.B, w.k, ws=ws, out=o, lse=lse)
 
     pairs, routed_pairs = selected_pairs(w)
     flops = flops_of_pairs(pairs, w)
@@ -412,6 +427,7 @@ def run_moba(args, w):
             "config": {"workload": w.name, "tokens": T, "sequences": len(w.lengths),
                        "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
                        "block_size": w.B, "top_k": w.k, "heads_per_pass": hp,
+                       **({} if route == "gate" else {"route": route}),
                        "l2": "inputs larger than L2 (no flush)",
                        "parallelism": "replicas x%d (independent problems)" % world},
             "moba_ms": ms, "dense_ms": dense_ms,
@@ -596,6 +612,87 @@ def run_decode(args, w):
     return 0 if status == 0 else 1
 
 
+BACKWARD_METRIC = "MoBA backward (dq, dk, dv over the forward's selection) ms & TFLOP/s at 1M tokens"
+
+
+def run_backward(args, w):
+    """The backward of the prefill's attention: one forward (untimed) gives
+    o, lse and the selection; each timed step is one moba_backward.  FLOPs:
+    2.5x the forward's 4*d per selected pair (S, dP, dQ, dK, dV against S, PV),
+    recomputation not counted."""
+    import torch
+    import block_sparse_long_07_b200 as moba
+    import synthetic as S
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        raise SystemExit("backward mode runs on one GPU")
+    if not w.batch_mode:
+        raise SystemExit("backward mode takes a batch workload")
+    b, N = len(w.lengths), w.lengths[0]
+    q, k, v = S.make_qkv(w, dev)
+    q, k, v = (x.view(b, N, x.shape[1], x.shape[2]) for x in (q, k, v))
+    sel = torch.empty(b, w.Hq, N, w.k, dtype=torch.int32, device=dev)
+    o, lse = moba.forward(q, k, v, w.B, w.k, sel_out=sel)
+    g = torch.Generator(device=dev).manual_seed(99)
+    dO = torch.randn(o.shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    p = moba.make_params(b, N, w.Hq, w.Hkv, w.d, w.B, w.k)
+    hp = moba.pick_heads_per_pass(lambda n: moba.backward_workspace_size(p, n), w.Hkv)
+    ws = moba.alloc_workspace(moba.backward_workspace_size(p, hp), dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def step():
+        moba.backward(q, k, v, o, lse, dO, sel, w.B, w.k, ws=ws, dq=dq, dk=dk, dv=dv)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = moba.last_device_status(ws)
+    if status != 0:
+        raise RuntimeError("device status %d after warm-up" % status)
+    pairs, _ = selected_pairs(w)
+    flops = 2.5 * flops_of_pairs(pairs, w)
+    clocks = ClockSampler(local)
+    torch.cuda.synchronize()
+    clocks.start()
+    moba.profile_enable(True)
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    kern = moba.profile_read()
+    moba.profile_enable(False)
+    status = moba.last_device_status(ws)
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks, peak_src = load_peaks()
+    peak_tf = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    value = flops / (ms / 1e3) / 1e12
+    line = {"metric": BACKWARD_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "backward_" + w.name, "tokens": w.T, "q_heads": w.Hq,
+                       "kv_heads": w.Hkv, "head_dim": w.d, "block_size": w.B, "top_k": w.k,
+                       "heads_per_pass": hp, "l2": "inputs larger than L2 (no flush)"},
+            "flops_per_step": flops,
+            "roofline": {"bound": "tensor", "kernel": "whole backward", "achieved": value,
+                         "peak": peak_tf, "unit": "TFLOP/s", "frac": value / peak_tf,
+                         "peak_source": "%s bf16_tflops_sustained" % peak_src, "traffic": None},
+            "gpu_launches": int(sum(n for n, _ in kern.values())),
+            "kernels_ms_per_step": {nm: round(t / args.steps, 4) for nm, (n, t) in kern.items()
+                                    if n},
+            "clocks": clk, "device_status": status}
+    print(json.dumps(line), flush=True)
+    return 0 if status == 0 else 1
+
+
 def cpu_decode_baseline(w, qdec_bits, k_bits, v_bits, budget_s=15.0):
     """The oracle on the decode rows (every sequence's last token, all heads),
     repeated for about budget_s seconds; the block means are computed once
@@ -668,13 +765,17 @@ def main():
     ap.add_argument("--ws-budget-gb", type=float, default=None,
                     help="workspace budget (default: the binding's, 32 GiB)")
     ap.add_argument("--ref-step-seconds", type=float, default=20.0)
-    ap.add_argument("--mode", default="prefill", choices=["prefill", "decode"])
+    ap.add_argument("--mode", default="prefill", choices=["prefill", "decode", "backward"])
+    ap.add_argument("--route", default="gate", choices=["gate", "minmax", "window", "sink"],
+                    help="prefill selection: the mean-pooled gate (the method), or a variant")
     args = ap.parse_args()
     import synthetic as S
     if args.workload.endswith("_k32"):
         w = S.WORKLOADS[args.workload[:-4]].with_k(32)
     else:
         w = S.WORKLOADS[args.workload]
+    if args.mode == "backward":
+        return run_backward(args, w)
     if args.mode == "decode":
         if args.impl == "reference":
             return run_decode_reference(args, w)

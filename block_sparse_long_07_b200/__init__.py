@@ -28,7 +28,11 @@ EXPORTS = ("moba_workspace_size", "moba_workspace_size_varlen", "moba_gate", "mo
            "moba_full_causal", "moba_full_causal_varlen", "moba_last_device_status",
            "moba_status_string", "moba_version", "moba_last_error_string", "moba_profile_enable", "moba_profile_reset",
            "moba_profile_read", "moba_selftest_wait_timeout", "moba_decode_workspace_size",
-           "moba_kbar_cache_size", "moba_kbar_cache_update", "moba_decode")
+           "moba_kbar_cache_size", "moba_kbar_cache_update", "moba_decode",
+           "moba_static_selection", "moba_gate_minmax", "moba_forward_selected",
+           "moba_forward_minmax", "moba_backward_workspace_size", "moba_backward")
+
+ROUTE_WINDOW, ROUTE_SINK = 0, 1
 
 
 class MobaError(RuntimeError):
@@ -107,6 +111,18 @@ def load_library(path=None):
     lib.moba_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_longlong, vp]
     lib.moba_profile_read.restype = i32
     lib.moba_profile_read.argtypes = [ctypes.POINTER(KernelTime), i32]
+    lib.moba_static_selection.restype = i32
+    lib.moba_static_selection.argtypes = [vp, i32, pp, vp]
+    lib.moba_gate_minmax.restype = i32
+    lib.moba_gate_minmax.argtypes = [vp, vp, vp, pp, vp, sz, vp]
+    lib.moba_forward_selected.restype = i32
+    lib.moba_forward_selected.argtypes = [vp, vp, vp, vp, vp, vp, pp, vp, sz, vp]
+    lib.moba_forward_minmax.restype = i32
+    lib.moba_forward_minmax.argtypes = [vp, vp, vp, vp, vp, vp, pp, vp, sz, vp]
+    lib.moba_backward_workspace_size.restype = sz
+    lib.moba_backward_workspace_size.argtypes = [pp, i32]
+    lib.moba_backward.restype = i32
+    lib.moba_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, pp, vp, sz, vp]
     dp = ctypes.POINTER(MobaDecodeParams)
     lib.moba_decode_workspace_size.restype = sz
     lib.moba_decode_workspace_size.argtypes = [dp]
@@ -385,3 +401,99 @@ def decode(q, k_cache, v_cache, seqlens, kbar, block_size, top_k, softmax_scale=
                                       ctypes.byref(p), _ptr(ws), ws.numel(), _stream(stream)),
            "moba_decode")
     return out, lse
+
+
+# ---------------------------------------------------------------- routing variants
+def static_selection(batch, seqlen, Hq, block_size, top_k, mode, device=None, sel=None,
+                     stream=None):
+    """Window (mode ROUTE_WINDOW) or sink (ROUTE_SINK) selection
+    sel [batch, Hq, seqlen, top_k]."""
+    torch = _torch()
+    p = make_params(batch, seqlen, Hq, Hq, 128, block_size, top_k)
+    if sel is None:
+        sel = torch.empty(batch, Hq, seqlen, top_k, dtype=torch.int32, device=device or "cuda")
+    _check(load_library().moba_static_selection(_ptr(sel), int(mode), ctypes.byref(p),
+                                                _stream(stream)), "moba_static_selection")
+    return sel
+
+
+def gate_minmax(q, k, block_size, top_k, softmax_scale=0.0, ws=None, sel=None, stream=None):
+    """Min/max-pooled gate: sel [b, Hq, N, top_k] for q [b,N,Hq,d], k [b,N,Hkv,d]."""
+    torch = _torch()
+    _require_cuda_bf16(q, k)
+    b, N, Hq, d = q.shape
+    p = make_params(b, N, Hq, k.shape[2], d, block_size, top_k, softmax_scale)
+    if sel is None:
+        sel = torch.empty(b, Hq, N, top_k, dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(workspace_size(p, 1), q.device)
+    _check(load_library().moba_gate_minmax(_ptr(q), _ptr(k), _ptr(sel), ctypes.byref(p),
+                                           _ptr(ws), ws.numel(), _stream(stream)),
+           "moba_gate_minmax")
+    return sel
+
+
+def _forward_common(q, k, v, block_size, top_k, softmax_scale, ws, out, lse):
+    torch = _torch()
+    _require_cuda_bf16(q, k, v)
+    b, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    p = make_params(b, N, Hq, Hkv, d, block_size, top_k, softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(b, Hq, N, dtype=torch.float32, device=q.device)
+    if ws is None:
+        hp = pick_heads_per_pass(lambda n: workspace_size(p, n), Hkv)
+        ws = alloc_workspace(workspace_size(p, hp), q.device)
+    return p, out, lse, ws
+
+
+def forward_selected(q, k, v, sel, block_size, top_k, softmax_scale=0.0, ws=None, out=None,
+                     lse=None, stream=None):
+    """MoBA forward over a given selection sel [b, Hq, N, top_k] (gate format)."""
+    p, out, lse, ws = _forward_common(q, k, v, block_size, top_k, softmax_scale, ws, out, lse)
+    _check(load_library().moba_forward_selected(_ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                                _ptr(lse), _ptr(sel), ctypes.byref(p),
+                                                _ptr(ws), ws.numel(), _stream(stream)),
+           "moba_forward_selected")
+    return out, lse
+
+
+def forward_minmax(q, k, v, block_size, top_k, softmax_scale=0.0, ws=None, out=None, lse=None,
+                   sel_out=None, stream=None):
+    """MoBA forward with the min/max-pooled gate: (o, lse)."""
+    p, out, lse, ws = _forward_common(q, k, v, block_size, top_k, softmax_scale, ws, out, lse)
+    _check(load_library().moba_forward_minmax(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                              _ptr(sel_out), ctypes.byref(p), _ptr(ws),
+                                              ws.numel(), _stream(stream)),
+           "moba_forward_minmax")
+    return out, lse
+
+
+# ---------------------------------------------------------------- backward
+def backward_workspace_size(params, heads_per_pass=0):
+    return int(load_library().moba_backward_workspace_size(ctypes.byref(params),
+                                                           int(heads_per_pass)))
+
+
+def backward(q, k, v, o, lse, dO, sel, block_size, top_k, softmax_scale=0.0, ws=None,
+             dq=None, dk=None, dv=None, stream=None):
+    """Gradients (dq, dk, dv) of the forward's attention over its selection
+    sel [b, Hq, N, top_k], for the output gradient dO [b, N, Hq, d]."""
+    torch = _torch()
+    _require_cuda_bf16(q, k, v, o, dO)
+    b, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    p = make_params(b, N, Hq, Hkv, d, block_size, top_k, softmax_scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if ws is None:
+        hp = pick_heads_per_pass(lambda n: backward_workspace_size(p, n), Hkv)
+        ws = alloc_workspace(backward_workspace_size(p, hp), q.device)
+    _check(load_library().moba_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO),
+                                        _ptr(sel), _ptr(dq), _ptr(dk), _ptr(dv),
+                                        ctypes.byref(p), _ptr(ws), ws.numel(), _stream(stream)),
+           "moba_backward")
+    return dq, dk, dv

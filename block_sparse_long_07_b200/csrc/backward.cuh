@@ -1,0 +1,565 @@
+// backward.cuh -- gradients of the MoBA attention over a fixed selection.
+//
+// No gradient passes through the hard top-k gate (wispaper.ai blog, "The
+// Change": the gradient does not flow through the discrete selection), so
+// the backward is that of exact softmax attention over each row's key set
+// I: with P_u = exp(scale q.k_u - lse) (the forward's lse), D = dO . O,
+//   dS_u = P_u (dO . v_u - D)
+//   dQ    = scale sum_u dS_u k_u,  dK_u += scale dS_u q,  dV_u += P_u dO.
+//
+// Work is organised like the forward.  For the routed part, the rows that
+// chose past block J (the forward's bucket of (kv head, J), gathered rows)
+// meet J's keys; for the own part, each block's rows meet the same block's
+// keys, causally.  Two kernels per part, each recomputing S and P:
+//   bw_kv_kernel  one CTA per (bucket or own block, 128-key tile): loops over
+//                 the rows in tiles of 128; S = Q K^T and dP = dO V^T into
+//                 TMEM, P and dS into shared memory as [rows][keys] tiles,
+//                 which are the transposed (MN-major) A operands of
+//                 dV += P^T dO and dK += dS^T Q, accumulated in TMEM
+//   bw_q_kernel   one CTA per tile of 128 rows (gathered or own): loops over
+//                 the block's key tiles; dS packed as bf16 into TMEM is the A
+//                 operand of dQ += dS K
+// The Q / dO tiles ([rows][d], 128-byte swizzled) serve both as K-major A
+// operands (S, dP) and as MN-major B operands (dK, dV); K / V tiles likewise.
+// Gradients are summed in fp32 buffers with atomic adds (each key gets one
+// routed and one own contribution per kv head; each row one per chosen
+// block) and converted to bf16 at the end.  This first version runs each
+// tile's MMAs and elementwise work in turn (no cross-tile pipelining).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "layout.cuh"
+
+namespace moba {
+
+enum { kBwRouted = 0, kBwOwn = 1 };
+
+struct BwArgs {
+  const __nv_bfloat16* q;   // [T][Hq][D]
+  const __nv_bfloat16* dO;  // [T][Hq][D]
+  const float2* dl;         // [T][Hq]: (D = dO . O, lse in log2 units)
+  float* dq32;              // [T][Hq][D]
+  float* dk32;              // [T][Hkv][D]
+  float* dv32;              // [T][Hkv][D]
+  const int32_t* entry_off; // routed: per (unit, block) bucket, as the forward
+  const int32_t* tile_off;  //         128-row items
+  const uint2* entries;
+  int Hq, Hkv, G, B, u0, nu, NBmax;
+  float scale_log2, scale;
+  SeqLayout L;
+  Plan P;
+  uint32_t* status;
+};
+
+template <int D>
+struct BwCfg {
+  static constexpr int kHalf = kTileM * 128;   // 128 rows x 64 columns bf16
+  static constexpr int kTile = kTileM * D * 2; // one [128][D] bf16 tile
+  static constexpr int kPT = kTileM * kTileN * 2;  // one [128 rows][128 keys] bf16 tile
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kTile;
+  static constexpr int kOffQ = kOffV + kTile;
+  static constexpr int kOffDO = kOffQ + kTile;
+  static constexpr int kOffP = kOffDO + kTile;
+  static constexpr int kOffDS = kOffP + kPT;
+  static constexpr int kOffBar = kOffDS + kPT;
+  static constexpr int kSmemBytes = kOffBar + 64 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  // TMEM columns
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColA = 256, kColB = 256 + D;
+};
+
+// (D = dO . O, lse * log2 e) per (token, q head), one warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) bw_prep_kernel(const __nv_bfloat16* __restrict__ o,
+                                                      const __nv_bfloat16* __restrict__ dO,
+                                                      const float* __restrict__ lse, int Hq,
+                                                      SeqLayout L, RowLayout R,
+                                                      float2* __restrict__ dl) {
+  constexpr int EPL = D / 32;
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);  // t * Hq + h
+  const int lane = threadIdx.x & 31;
+  if (row >= L.T * Hq) return;
+  const int64_t t = row / Hq;
+  const int h = (int)(row % Hq);
+  float acc = 0.f;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    const size_t idx = (size_t)row * D + lane * EPL + e;
+    acc = fmaf(__bfloat162float(o[idx]), __bfloat162float(dO[idx]), acc);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) {
+    const int s = seq_of_token(L, t);
+    const float l = lse[row_index(R, s, h, t - seq_start(L, s), t)];
+    dl[row] = make_float2(acc, l * 1.4426950408889634f);
+  }
+}
+
+// One thread per row of a 128-row tile: the row's (token, q head) or -1.
+struct BwRow {
+  int64_t t;
+  int h;
+};
+
+// Rows of tile `tile` of a CTA's work: routed -> entries[e0 + ...]; own ->
+// contiguous tokens of a block for one head.
+__device__ __forceinline__ BwRow bw_row_routed(const BwArgs& a, int g, int64_t e0, int64_t e1,
+                                               int r) {
+  BwRow x{-1, 0};
+  if (e0 + r < e1) {
+    const uint2 e = a.entries[e0 + r];
+    const int hh = (int)(e.y & 0xFFFFu);
+    if (e.x < (uint32_t)a.L.T && hh < a.G) {
+      x.t = e.x;
+      x.h = g * a.G + hh;
+    } else {
+      atomicOr(a.status, MOBA_DEV_BAD_INDEX);
+    }
+  }
+  return x;
+}
+
+// Copy row r's q and dO (128-byte swizzled halves of 64 columns) into the
+// tiles; a row with t < 0 copies token 0's data (finite; its P and dS are
+// forced to zero).
+template <int D>
+__device__ __forceinline__ void bw_load_row(const BwArgs& a, BwRow x, int r, unsigned char* sQ,
+                                            unsigned char* sDO) {
+  using C = BwCfg<D>;
+  const int64_t t = x.t < 0 ? 0 : x.t;
+  const __nv_bfloat16* qs = a.q + ((size_t)t * a.Hq + x.h) * D;
+  const __nv_bfloat16* gs = a.dO + ((size_t)t * a.Hq + x.h) * D;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    const uint32_t off = (uint32_t)(c >> 3) * C::kHalf + sw128_offset(r, c & 7);
+    cp_async_16(sQ + off, qs + c * 8);
+    cp_async_16(sDO + off, gs + c * 8);
+  }
+}
+
+// P and dS of row r for key tile [kbase, kbase + 128): reads S and dP from
+// TMEM (this thread's lane), masks keys >= nkeys and, when causal, keys
+// after the row's token.  Writes P and dS as bf16 [rows][keys] tiles
+// (128-byte swizzled halves of 64 keys) when to_smem, or dS packed into
+// TMEM columns [kColS, kColS + 64) otherwise.
+template <int D, bool TO_SMEM>
+__device__ __forceinline__ void bw_p_ds(const BwArgs& a, uint32_t tS, uint32_t tDP, int r,
+                                        float lse2, float Dr, int nkeys, bool causal,
+                                        int64_t trow, int64_t kbase, unsigned char* sP,
+                                        unsigned char* sDS) {
+  using C = BwCfg<D>;
+#pragma unroll 1
+  for (int c0 = 0; c0 < kTileN; c0 += 32) {
+    uint32_t sv[32], dv[32];
+    tmem_ld32(tS + c0, sv);
+    tmem_ld32(tDP + c0, dv);
+    tc_wait_ld();
+    uint32_t pp[16], dd[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      float p2[2], d2[2];
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const int j = c0 + 2 * e + x;
+        bool keep = j < nkeys;
+        if (causal) keep = keep && (kbase + j <= trow);
+        const float p =
+            keep ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + x]), a.scale_log2, -lse2)) : 0.f;
+        p2[x] = p;
+        d2[x] = p * (__uint_as_float(dv[2 * e + x]) - Dr);
+      }
+      pp[e] = pack_bf16x2(p2[0], p2[1]);
+      dd[e] = pack_bf16x2(d2[0], d2[1]);
+    }
+    if (TO_SMEM) {
+      // keys c0..c0+31 = 64 bytes = 4 16-byte units of half c0 / 64
+      const uint32_t hoff = (uint32_t)(c0 >> 6) * C::kHalf;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t off = hoff + sw128_offset(r, ((c0 & 63) >> 3) + u);
+        *reinterpret_cast<uint4*>(sP + off) =
+            make_uint4(pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
+        *reinterpret_cast<uint4*>(sDS + off) =
+            make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
+      }
+    } else {
+      tmem_st16(tS + (c0 >> 1), dd);
+    }
+  }
+}
+
+// End of a backward CTA.  After an abort, copies or MMAs may still be in
+// flight: wait for them (bounded, nothing raised) before TMEM is freed and
+// the CTA's shared memory released.
+__device__ __forceinline__ void bw_teardown(uint64_t* kv_bar, uint64_t* mma_bar, bool ok,
+                                            uint32_t nm, uint32_t tmem, uint32_t cols,
+                                            int warp) {
+  if (!ok && threadIdx.x == 0) {
+    mbar_wait_teardown(kv_bar, 0, 200000000ull);
+    mbar_wait_teardown(kv_bar, 1, 200000000ull);
+  }
+  if (warp == 0) {
+    // every MMA this CTA issued has completed once this commit arrives
+    tc_commit_warp(mma_bar);
+    if (threadIdx.x == 0) mbar_wait_teardown(mma_bar, nm & 1, 500000000ull);
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, cols);
+  }
+}
+
+// Bounded wait of the whole CTA on an mbarrier phase.
+__device__ __forceinline__ bool bw_wait(uint64_t* bar, uint32_t parity,
+                                        volatile uint32_t* abort_flag, uint32_t* st) {
+  return __syncthreads_and(mbar_wait(bar, parity, abort_flag, st) ? 1 : 0) != 0;
+}
+
+// dK / dV of one 128-key tile.
+//   routed: blockIdx.x = f * KT + kt over the pass's buckets f = u * NB + J;
+//           rows = the bucket's entries
+//   own:    blockIdx.x = f * KT + kt over (unit, block); rows = the block's
+//           tokens at or after the key tile, for every q head of the unit
+template <int D, int MODE>
+__global__ void __launch_bounds__(128, 1)
+    bw_kv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const BwArgs a) {
+  using C = BwCfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* kv_bar = bars + 0;
+  uint64_t* mma_bar = bars + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = threadIdx.x;
+
+  const int NB = a.P.totals[0];
+  const int KT = a.B / kTileN;
+  const int64_t f = blockIdx.x / KT;
+  const int kt = (int)(blockIdx.x % KT);
+  if (f >= (int64_t)a.nu * NB) return;
+  const int u = (int)(f / NB), J = (int)(f % NB);
+  const int g = a.u0 + u;
+  const int blen = a.P.blk_len[J];
+  const int nkeys = min(kTileN, blen - kt * kTileN);
+  if (nkeys <= 0) return;
+  const int64_t kstart = (int64_t)a.P.blk_tok[J] + (int64_t)kt * kTileN;
+  int64_t e0 = 0, e1 = 0;
+  int ntiles;
+  int own_tiles = 0;  // own: row tiles per q head
+  if (MODE == kBwRouted) {
+    e0 = a.entry_off[f];
+    e1 = a.entry_off[f + 1];
+    ntiles = (int)((e1 - e0 + kTileM - 1) / kTileM);
+  } else {
+    own_tiles = (blen - kt * kTileN + kTileM - 1) / kTileM;  // tiles from the key tile on
+    ntiles = own_tiles * a.G;
+  }
+  if (ntiles == 0) return;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_bar, 1);
+    mbar_init(mma_bar, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  unsigned char* sK = smem + C::kOffK;
+  unsigned char* sV = smem + C::kOffV;
+  unsigned char* sQ = smem + C::kOffQ;
+  unsigned char* sDO = smem + C::kOffDO;
+  unsigned char* sP = smem + C::kOffP;
+  unsigned char* sDS = smem + C::kOffDS;
+  uint32_t* st = a.status;
+  bool ok = true;
+  uint32_t nm = 0;  // mma_bar phases
+
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(kv_bar, 2 * C::kTile);
+#pragma unroll
+    for (int hx = 0; hx < D / 64; ++hx) {
+      tma_load_3d(sK + hx * C::kHalf, &tm_k, kv_bar, hx * 64, g, (int)kstart);
+      tma_load_3d(sV + hx * C::kHalf, &tm_v, kv_bar, hx * 64, g, (int)kstart);
+    }
+  }
+  ok = bw_wait(kv_bar, 0, abort_flag, st);
+
+  const uint32_t sQa = smem_u32(sQ), sDOa = smem_u32(sDO), sKa = smem_u32(sK),
+                 sVa = smem_u32(sV), sPa = smem_u32(sP), sDSa = smem_u32(sDS);
+  constexpr uint32_t idS = idesc_bf16_f32(kTileM, kTileN, false, false);
+  constexpr uint32_t idG = idesc_bf16_f32(kTileN, D, true, true);
+  for (int tile = 0; tile < ntiles && ok; ++tile) {
+    BwRow x{-1, 0};
+    if (MODE == kBwRouted) {
+      x = bw_row_routed(a, g, e0 + (int64_t)tile * kTileM, e1, r);
+    } else {
+      const int hh = tile / own_tiles, qt = tile % own_tiles;
+      const int64_t t = kstart + (int64_t)qt * kTileM + r;
+      if (t < (int64_t)a.P.blk_tok[J] + blen) {
+        x.t = t;
+        x.h = g * a.G + hh;
+      }
+    }
+    float lse2 = __int_as_float(0x7f800000), Dr = 0.f;
+    if (x.t >= 0) {
+      const float2 v = a.dl[(size_t)x.t * a.Hq + x.h];
+      Dr = v.x;
+      lse2 = v.y;
+    }
+    bw_load_row<D>(a, x, r, sQ, sDO);
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (warp == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::kHalf + (kk & 3) * 32;
+        tc_mma_ss_warp(tmem + C::kColS, sdesc_kmajor_sw128(sQa + off),
+                       sdesc_kmajor_sw128(sKa + off), idS, kk > 0 ? 1u : 0u);
+        tc_mma_ss_warp(tmem + C::kColDP, sdesc_kmajor_sw128(sDOa + off),
+                       sdesc_kmajor_sw128(sVa + off), idS, kk > 0 ? 1u : 0u);
+      }
+      tc_commit_warp(mma_bar);
+    }
+    ok = bw_wait(mma_bar, nm & 1, abort_flag, st);
+    ++nm;
+    if (!ok) break;
+    tc_fence_after();
+    bw_p_ds<D, true>(a, tmem + lane_off + C::kColS, tmem + lane_off + C::kColDP, r, lse2, Dr,
+                     nkeys, MODE == kBwOwn, x.t, kstart, sP, sDS);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < kTileM / 16; ++kk) {  // K = rows, 16 per step
+        const uint32_t acc = (tile > 0 || kk > 0) ? 1u : 0u;
+        tc_mma_ss_warp(tmem + C::kColA, sdesc_mnmajor_sw128(sPa + kk * 2048, C::kHalf, 1024),
+                       sdesc_mnmajor_sw128(sDOa + kk * 2048, C::kHalf, 1024), idG, acc);
+        tc_mma_ss_warp(tmem + C::kColB, sdesc_mnmajor_sw128(sDSa + kk * 2048, C::kHalf, 1024),
+                       sdesc_mnmajor_sw128(sQa + kk * 2048, C::kHalf, 1024), idG, acc);
+      }
+      tc_commit_warp(mma_bar);
+    }
+    ok = bw_wait(mma_bar, nm & 1, abort_flag, st);
+    ++nm;
+  }
+  if (ok) {
+    tc_fence_after();
+    // row r of the accumulators = key kstart + r; every lane takes part in
+    // the (warp-collective) TMEM loads, only lanes of real keys store
+    float* dv = a.dv32 + ((size_t)(kstart + r) * a.Hkv + g) * D;
+    float* dk = a.dk32 + ((size_t)(kstart + r) * a.Hkv + g) * D;
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t va[32], vb[32];
+      tmem_ld32(tmem + lane_off + C::kColA + c0, va);
+      tmem_ld32(tmem + lane_off + C::kColB + c0, vb);
+      tc_wait_ld();
+      if (r < nkeys) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          atomicAdd(dv + c0 + e, __uint_as_float(va[e]));
+          atomicAdd(dk + c0 + e, __uint_as_float(vb[e]) * a.scale);
+        }
+      }
+    }
+  }
+  bw_teardown(kv_bar, mma_bar, ok, nm, tmem, C::kTmemCols, warp);
+}
+
+// dQ of one 128-row tile.
+//   routed: blockIdx.x = item over the pass's 128-row items (tile_off);
+//           keys = all of the bucket's block
+//   own:    blockIdx.x = (unit head, query tile); keys = the tile's block up
+//           to and including the tile's own 128 keys (causal)
+template <int D, int MODE>
+__global__ void __launch_bounds__(128, 1)
+    bw_q_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                const BwArgs a) {
+  using C = BwCfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* kv_bar = bars + 0;
+  uint64_t* mma_bar = bars + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  const int warp = threadIdx.x >> 5, r = threadIdx.x;
+  const int NB = a.P.totals[0];
+
+  int g, J;
+  int nkt;             // key tiles to visit
+  int64_t kblock;      // first token of the block
+  int blen;
+  BwRow x{-1, 0};
+  if (MODE == kBwRouted) {
+    const int64_t nitems = a.tile_off[a.nu * NB];
+    if (blockIdx.x >= nitems) return;
+    const int f = upper_index(a.tile_off, a.nu * NB + 1, blockIdx.x);
+    const int u = f / NB;
+    J = f % NB;
+    g = a.u0 + u;
+    const int64_t e0 = a.entry_off[f] + (int64_t)(blockIdx.x - a.tile_off[f]) * kTileM;
+    x = bw_row_routed(a, g, e0, a.entry_off[f + 1], r);
+    blen = a.P.blk_len[J];
+    kblock = a.P.blk_tok[J];
+    nkt = (blen + kTileN - 1) / kTileN;
+  } else {
+    // (head of the unit, query tile)
+    const int NQT = a.P.totals[1];
+    const int64_t idx = blockIdx.x;
+    const int hl = (int)(idx / NQT);
+    const int qt = (int)(idx % NQT);
+    if (hl >= a.nu * a.G) return;
+    const int s = upper_index(a.P.qt_off, a.L.nseq + 1, qt);
+    const int64_t st0 = seq_start(a.L, s), len = seq_len(a.L, s);
+    const int64_t p0 = (int64_t)(qt - a.P.qt_off[s]) * kTileM;
+    const int i = (int)(p0 / a.B);
+    J = a.P.blk_off[s] + i;
+    g = a.u0 + hl / a.G;
+    blen = a.P.blk_len[J];
+    kblock = a.P.blk_tok[J];
+    nkt = (int)((p0 - (int64_t)i * a.B) / kTileN) + 1;  // up to the diagonal tile
+    if (p0 + r < len) {
+      x.t = st0 + p0 + r;
+      x.h = g * a.G + hl % a.G;
+    }
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_bar, 1);
+    mbar_init(mma_bar, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  unsigned char* sK = smem + C::kOffK;
+  unsigned char* sV = smem + C::kOffV;
+  unsigned char* sQ = smem + C::kOffQ;
+  unsigned char* sDO = smem + C::kOffDO;
+  uint32_t* st = a.status;
+
+  float lse2 = __int_as_float(0x7f800000), Dr = 0.f;
+  if (x.t >= 0) {
+    const float2 v = a.dl[(size_t)x.t * a.Hq + x.h];
+    Dr = v.x;
+    lse2 = v.y;
+  }
+  bw_load_row<D>(a, x, r, sQ, sDO);
+  cp_async_wait_all();
+  fence_proxy_async_smem();
+  __syncthreads();
+
+  const uint32_t sQa = smem_u32(sQ), sDOa = smem_u32(sDO), sKa = smem_u32(sK),
+                 sVa = smem_u32(sV);
+  constexpr uint32_t idS = idesc_bf16_f32(kTileM, kTileN, false, false);
+  constexpr uint32_t idQ = idesc_bf16_f32(kTileM, D, false, true);
+  bool ok = true;
+  uint32_t nm = 0;
+  for (int kt = 0; kt < nkt && ok; ++kt) {
+    const int64_t kbase = kblock + (int64_t)kt * kTileN;
+    const int nkeys = min(kTileN, blen - kt * kTileN);
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(kv_bar, 2 * C::kTile);
+#pragma unroll
+      for (int hx = 0; hx < D / 64; ++hx) {
+        tma_load_3d(sK + hx * C::kHalf, &tm_k, kv_bar, hx * 64, g, (int)kbase);
+        tma_load_3d(sV + hx * C::kHalf, &tm_v, kv_bar, hx * 64, g, (int)kbase);
+      }
+    }
+    ok = bw_wait(kv_bar, kt & 1, abort_flag, st);
+    if (!ok) break;
+    if (warp == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * C::kHalf + (kk & 3) * 32;
+        tc_mma_ss_warp(tmem + C::kColS, sdesc_kmajor_sw128(sQa + off),
+                       sdesc_kmajor_sw128(sKa + off), idS, kk > 0 ? 1u : 0u);
+        tc_mma_ss_warp(tmem + C::kColDP, sdesc_kmajor_sw128(sDOa + off),
+                       sdesc_kmajor_sw128(sVa + off), idS, kk > 0 ? 1u : 0u);
+      }
+      tc_commit_warp(mma_bar);
+    }
+    ok = bw_wait(mma_bar, nm & 1, abort_flag, st);
+    ++nm;
+    if (!ok) break;
+    tc_fence_after();
+    bw_p_ds<D, false>(a, tmem + lane_off + C::kColS, tmem + lane_off + C::kColDP, r, lse2, Dr,
+                      nkeys, MODE == kBwOwn, x.t, kbase, nullptr, nullptr);
+    tc_wait_st();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < kTileN / 16; ++kk)  // K = keys, 16 per step
+        tc_mma_ts_warp(tmem + C::kColA, tmem + C::kColS + kk * 8,
+                       sdesc_mnmajor_sw128(sKa + kk * 2048, C::kHalf, 1024), idQ,
+                       (kt > 0 || kk > 0) ? 1u : 0u);
+      tc_commit_warp(mma_bar);
+    }
+    // the next K / V load and S MMA overwrite what this MMA reads
+    ok = bw_wait(mma_bar, nm & 1, abort_flag, st);
+    ++nm;
+  }
+  if (ok) {
+    tc_fence_after();
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t va[32];
+      tmem_ld32(tmem + lane_off + C::kColA + c0, va);
+      tc_wait_ld();
+      if (x.t >= 0) {
+        float* dq = a.dq32 + ((size_t)x.t * a.Hq + x.h) * D + c0;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) atomicAdd(dq + e, __uint_as_float(va[e]) * a.scale);
+      }
+    }
+  }
+  bw_teardown(kv_bar, mma_bar, ok, nm, tmem, C::kTmemCols, warp);
+}
+
+// fp32 accumulators -> bf16 gradients.
+__global__ void bw_finish_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                                 int64_t n) {
+  const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i + 3 < n) {
+    const float4 v = *reinterpret_cast<const float4*>(src + i);
+    *reinterpret_cast<uint2*>(dst + i) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  } else {
+    for (int64_t j = i; j < n; ++j) dst[j] = __float2bfloat16_rn(src[j]);
+  }
+}
+
+}  // namespace moba

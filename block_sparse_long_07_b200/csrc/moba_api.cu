@@ -26,6 +26,8 @@
 #include "attn_tc2.cuh"
 #include "gate_tc.cuh"
 #include "decode.cuh"
+#include "variants.cuh"
+#include "backward.cuh"
 #include "common.cuh"
 #include "layout.cuh"
 
@@ -36,12 +38,14 @@ namespace {
 // ------------------------------------------------------------ kernel timer
 enum KernelClass {
   kKPlan, kKPool, kKGate, kKGateCount, kKScan, kKScatter, kKRouted, kKOwn, kKMerge, kKDense,
-  kKKbarCache, kKDecGate, kKDecAttn, kKDecMerge, kKNum
+  kKKbarCache, kKDecGate, kKDecAttn, kKDecMerge, kKMinmaxPool, kKGateMinmax, kKStaticSel,
+  kKBwPrep, kKBwKv, kKBwQ, kKBwFinish, kKNum
 };
 const char* const kKernelNames[kKNum] = {
-    "plan",        "pool",     "gate",       "gate_count",  "bucket_scan",
-    "bucket_scatter", "attn_routed", "attn_own", "merge",    "attn_dense",
-    "kbar_cache",  "decode_gate", "decode_attn", "decode_merge"};
+    "plan",        "pool",        "gate",         "gate_count",  "bucket_scan",
+    "bucket_scatter", "attn_routed", "attn_own",  "merge",       "attn_dense",
+    "kbar_cache",  "decode_gate", "decode_attn",  "decode_merge", "minmax_pool",
+    "gate_minmax", "static_select", "bw_prep", "bw_kv", "bw_q", "bw_finish"};
 struct TimedLaunch {
   int cls;
   cudaEvent_t a, b;
@@ -447,6 +451,76 @@ moba_status run_plan_pool(const Problem& pr, const void* k, const Ws& w, cudaStr
   return MOBA_OK;
 }
 
+// How a forward obtains its selection.
+enum Routing { kRouteMeanGate = 0, kRouteMinmaxGate = 1, kRouteGiven = 2 };
+
+moba_status run_plan(const Problem& pr, const Ws& w, cudaStream_t st) {
+  SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
+  Timed tm(kKPlan, st);
+  plan_kernel<<<1, 1024, 0, st>>>(L, pr.B, w.P, (int)pr.NBmax, (int)pr.NQTmax, w.status);
+  return cuda_status(cudaGetLastError());
+}
+
+// Block max / min (bf16 pairs) into the block-mean buffer, which has exactly
+// the room: 2 x 2 bytes per element against 4.
+moba_status run_minmax_pool(const Problem& pr, const void* k, const Ws& w, cudaStream_t st) {
+  dim3 grid((unsigned)pr.NBmax, (unsigned)pr.Hkv);
+  __nv_bfloat16* mm = reinterpret_cast<__nv_bfloat16*>(w.kbar);
+  Timed tm(kKMinmaxPool, st);
+  if (pr.D == 128)
+    minmax_pool_kernel<128><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(k),
+                                                  pr.Hkv, w.P, (int)pr.NBmax, mm);
+  else
+    minmax_pool_kernel<64><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(k),
+                                                 pr.Hkv, w.P, (int)pr.NBmax, mm);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int D, int KM>
+moba_status launch_gate_minmax_km(const Problem& pr, const void* q, const Ws& w, int32_t* sel,
+                                  uint32_t* counts, cudaStream_t st) {
+  const size_t smem =
+      sizeof(float) * kMinmaxChunk * 2 * D + sizeof(uint32_t) * kMaxBlocksPerSeq;
+  auto kern = gate_minmax_kernel<D, KM>;
+  MOBA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
+  dim3 grid((unsigned)pr.NQTmax, (unsigned)pr.Hq);
+  Timed tm(kKGateMinmax, st);
+  kern<<<grid, 128, smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(q), pr.Hq, pr.G, pr.B,
+                                pr.topk, L, w.P, (int)pr.NBmax,
+                                reinterpret_cast<const __nv_bfloat16*>(w.kbar), sel, pr.R,
+                                counts, w.status);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int D>
+moba_status launch_gate_minmax(const Problem& pr, const void* q, const Ws& w, int32_t* sel,
+                               uint32_t* counts, cudaStream_t st) {
+  const int64_t npast = pr.topk - 1;
+  const int64_t need = (npast >= pr.max_blocks_per_seq - 1) ? 1 : npast;
+  switch (pow2_at_least(need)) {
+    case 1: return launch_gate_minmax_km<D, 1>(pr, q, w, sel, counts, st);
+    case 2: return launch_gate_minmax_km<D, 2>(pr, q, w, sel, counts, st);
+    case 4: return launch_gate_minmax_km<D, 4>(pr, q, w, sel, counts, st);
+    case 8: return launch_gate_minmax_km<D, 8>(pr, q, w, sel, counts, st);
+    case 16: return launch_gate_minmax_km<D, 16>(pr, q, w, sel, counts, st);
+    case 32: return launch_gate_minmax_km<D, 32>(pr, q, w, sel, counts, st);
+    case 64: return launch_gate_minmax_km<D, 64>(pr, q, w, sel, counts, st);
+    default: return MOBA_ERR_UNSUPPORTED;
+  }
+}
+
+// Bucket sizes from a selection written by someone else.
+moba_status launch_count(const Problem& pr, const Ws& w, const int32_t* sel, uint32_t* counts,
+                         cudaStream_t st) {
+  SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
+  dim3 grid((unsigned)pr.NQTmax, (unsigned)pr.Hkv);
+  Timed tm(kKGateCount, st);
+  gate_count_kernel<<<grid, 128, sizeof(uint32_t) * kMaxBlocksPerSeq, st>>>(
+      sel, pr.R, pr.topk, pr.B, pr.G, L, w.P, (int)pr.NBmax, counts, w.status);
+  return cuda_status(cudaGetLastError());
+}
+
 moba_status gate_impl(const Problem& pr, const void* q, const void* k, int32_t* sel, void* ws,
                       size_t ws_bytes, cudaStream_t st) {
   if (!q || !k || !sel || !aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(sel) & 3))
@@ -464,14 +538,19 @@ moba_status gate_impl(const Problem& pr, const void* q, const void* k, int32_t* 
 template <int D>
 moba_status forward_passes(const Problem& pr, const void* q, const void* k, const void* v,
                            void* o, float* lse, const Ws& w, int32_t* sel, int nu_max,
-                           cudaStream_t st) {
+                           int route, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, pr.Hq, pr.T, D) || !make_tmap(&tk, k, pr.Hkv, pr.T, D) ||
       !make_tmap(&tv, v, pr.Hkv, pr.T, D))
     return MOBA_ERR_CUDA;
   SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
   MOBA_CUDA(cudaMemsetAsync(w.counts, 0, sizeof(uint32_t) * (size_t)pr.Hkv * pr.NBmax, st));
-  MOBA_TRY(launch_gate<D>(pr, q, w, sel, w.counts, st));
+  if (route == kRouteMeanGate)
+    MOBA_TRY(launch_gate<D>(pr, q, w, sel, w.counts, st));
+  else if (route == kRouteMinmaxGate)
+    MOBA_TRY(launch_gate_minmax<D>(pr, q, w, sel, w.counts, st));
+  else if (pr.topk > 1)
+    MOBA_TRY(launch_count(pr, w, sel, w.counts, st));
   AttnArgs a;
   memset(&a, 0, sizeof a);
   a.q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -526,7 +605,7 @@ moba_status forward_passes(const Problem& pr, const void* q, const void* k, cons
 
 moba_status forward_impl(const Problem& pr, const void* q, const void* k, const void* v, void* o,
                          float* lse, int32_t* sel_out, void* ws, size_t ws_bytes,
-                         cudaStream_t st) {
+                         cudaStream_t st, int route = kRouteMeanGate) {
   if (!q || !k || !v || !o || !lse) return MOBA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(lse) & 3) || (reinterpret_cast<uintptr_t>(sel_out) & 3))
@@ -544,9 +623,17 @@ moba_status forward_impl(const Problem& pr, const void* q, const void* k, const 
     ++nu;
   const Ws w = carve(pr, nu, static_cast<char*>(ws));
   int32_t* sel = sel_out ? sel_out : w.sel;
-  MOBA_TRY(run_plan_pool(pr, k, w, st));
-  return pr.D == 128 ? forward_passes<128>(pr, q, k, v, o, lse, w, sel, nu, st)
-                     : forward_passes<64>(pr, q, k, v, o, lse, w, sel, nu, st);
+  if (route == kRouteGiven && !sel_out) return MOBA_ERR_INVALID_ARG;
+  if (route == kRouteMeanGate)
+    MOBA_TRY(run_plan_pool(pr, k, w, st));
+  else if (route == kRouteMinmaxGate) {
+    MOBA_TRY(run_plan(pr, w, st));
+    MOBA_TRY(run_minmax_pool(pr, k, w, st));
+  } else {
+    MOBA_TRY(run_plan(pr, w, st));
+  }
+  return pr.D == 128 ? forward_passes<128>(pr, q, k, v, o, lse, w, sel, nu, route, st)
+                     : forward_passes<64>(pr, q, k, v, o, lse, w, sel, nu, route, st);
 }
 
 size_t dense_ws_bytes(int64_t T, int nseq) {
@@ -624,6 +711,179 @@ __global__ void wait_selftest_kernel(uint32_t* status, long long limit_cycles) {
   abort_flag = 0u;
   fence_barrier_init();
   mbar_wait(&bar, 0, &abort_flag, status, limit_cycles);
+}
+
+// ---------------------------------------------------------------- backward
+struct BwWs {
+  Ws w;  // status, plan, counts, buckets and entries, as the forward's
+  float2* dl;
+  float* dq32;
+  float* dk32;
+  float* dv32;
+  size_t bytes;
+};
+
+BwWs carve_bw(const Problem& pr, int nu, char* base) {
+  BwWs b;
+  memset(&b, 0, sizeof b);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + bytes);
+    return p;
+  };
+  const int64_t NB = pr.NBmax;
+  const int64_t np = pr.topk > 1 ? pr.topk - 1 : 0;
+  Ws& w = b.w;
+  w.status = reinterpret_cast<uint32_t*>(take(kAlign));
+  w.P.totals = reinterpret_cast<int32_t*>(take(4 * sizeof(int32_t)));
+  w.P.blk_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (pr.nseq + 1)));
+  w.P.qt_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (pr.nseq + 1)));
+  w.P.pair_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (pr.nseq + 1)));
+  w.P.blk_tok = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * NB));
+  w.P.blk_len = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * NB));
+  w.counts = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * (size_t)pr.Hkv * NB));
+  w.entry_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * ((size_t)nu * NB + 1)));
+  w.tile_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * ((size_t)nu * NB + 1)));
+  w.cursor = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * (size_t)nu * NB));
+  w.entries = reinterpret_cast<uint2*>(take(sizeof(uint2) * (size_t)nu * pr.T * pr.G * np));
+  b.dl = reinterpret_cast<float2*>(take(sizeof(float2) * (size_t)pr.T * pr.Hq));
+  b.dq32 = reinterpret_cast<float*>(take(sizeof(float) * (size_t)pr.T * pr.Hq * pr.D));
+  b.dk32 = reinterpret_cast<float*>(take(sizeof(float) * (size_t)pr.T * pr.Hkv * pr.D));
+  b.dv32 = reinterpret_cast<float*>(take(sizeof(float) * (size_t)pr.T * pr.Hkv * pr.D));
+  b.bytes = off;
+  return b;
+}
+
+template <int D>
+moba_status backward_passes(const Problem& pr, const void* q, const void* k, const void* v,
+                            const void* o, const float* lse, const void* dO, const int32_t* sel,
+                            void* dq, void* dk, void* dv, const BwWs& b, int nu_max,
+                            cudaStream_t st) {
+  using C = BwCfg<D>;
+  const Ws& w = b.w;
+  SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
+  MOBA_TRY(run_plan(pr, w, st));
+  if (pr.topk > 1) {
+    MOBA_CUDA(cudaMemsetAsync(w.counts, 0, sizeof(uint32_t) * (size_t)pr.Hkv * pr.NBmax, st));
+    MOBA_TRY(launch_count(pr, w, sel, w.counts, st));
+  }
+  MOBA_CUDA(cudaMemsetAsync(b.dq32, 0, sizeof(float) * (size_t)pr.T * pr.Hq * D, st));
+  MOBA_CUDA(cudaMemsetAsync(b.dk32, 0, sizeof(float) * (size_t)pr.T * pr.Hkv * D, st));
+  MOBA_CUDA(cudaMemsetAsync(b.dv32, 0, sizeof(float) * (size_t)pr.T * pr.Hkv * D, st));
+  {
+    Timed tm(kKBwPrep, st);
+    const int64_t rows = pr.T * pr.Hq;
+    bw_prep_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dO),
+        lse, pr.Hq, L, pr.R, b.dl);
+    MOBA_CUDA(cudaGetLastError());
+  }
+  CUtensorMap tk, tv;
+  if (!make_tmap(&tk, k, pr.Hkv, pr.T, D) || !make_tmap(&tv, v, pr.Hkv, pr.T, D))
+    return MOBA_ERR_CUDA;
+  MOBA_CUDA(cudaFuncSetAttribute(bw_kv_kernel<D, kBwRouted>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
+  MOBA_CUDA(cudaFuncSetAttribute(bw_kv_kernel<D, kBwOwn>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
+  MOBA_CUDA(cudaFuncSetAttribute(bw_q_kernel<D, kBwRouted>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
+  MOBA_CUDA(cudaFuncSetAttribute(bw_q_kernel<D, kBwOwn>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
+  BwArgs a;
+  memset(&a, 0, sizeof a);
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.dO = reinterpret_cast<const __nv_bfloat16*>(dO);
+  a.dl = b.dl;
+  a.dq32 = b.dq32;
+  a.dk32 = b.dk32;
+  a.dv32 = b.dv32;
+  a.entry_off = w.entry_off;
+  a.tile_off = w.tile_off;
+  a.entries = w.entries;
+  a.Hq = pr.Hq;
+  a.Hkv = pr.Hkv;
+  a.G = pr.G;
+  a.B = pr.B;
+  a.NBmax = (int)pr.NBmax;
+  a.scale = pr.scale;
+  a.scale_log2 = pr.scale * 1.4426950408889634f;
+  a.L = L;
+  a.P = w.P;
+  a.status = w.status;
+  const int64_t KT = pr.B / kTileN;
+  const int64_t np = pr.topk > 1 ? pr.topk - 1 : 0;
+  for (int u0 = 0; u0 < pr.Hkv; u0 += nu_max) {
+    const int nu = (pr.Hkv - u0) < nu_max ? (pr.Hkv - u0) : nu_max;
+    a.u0 = u0;
+    a.nu = nu;
+    if (pr.topk > 1) {
+      {
+        Timed tm(kKScan, st);
+        bucket_scan_kernel<<<1, 1024, 0, st>>>(w.counts, u0, nu, kTileM, w.P, (int)pr.NBmax,
+                                               w.entry_off, w.tile_off, w.cursor);
+      }
+      MOBA_CUDA(cudaGetLastError());
+      MOBA_TRY(launch_scatter(pr, w, sel, u0, nu, st));
+      {
+        Timed tm(kKBwKv, st);
+        bw_kv_kernel<D, kBwRouted><<<(unsigned)(nu * pr.NBmax * KT), 128, C::kSmemBytes, st>>>(
+            tk, tv, a);
+        MOBA_CUDA(cudaGetLastError());
+      }
+      {
+        const int64_t items = (int64_t)nu * pr.T * pr.G * np / kTileM + (int64_t)nu * pr.NBmax;
+        Timed tm(kKBwQ, st);
+        bw_q_kernel<D, kBwRouted><<<(unsigned)items, 128, C::kSmemBytes, st>>>(tk, tv, a);
+        MOBA_CUDA(cudaGetLastError());
+      }
+    }
+    {
+      Timed tm(kKBwKv, st);
+      bw_kv_kernel<D, kBwOwn><<<(unsigned)(nu * pr.NBmax * KT), 128, C::kSmemBytes, st>>>(tk, tv,
+                                                                                       a);
+      MOBA_CUDA(cudaGetLastError());
+    }
+    {
+      Timed tm(kKBwQ, st);
+      bw_q_kernel<D, kBwOwn><<<(unsigned)(nu * pr.G * pr.NQTmax), 128, C::kSmemBytes, st>>>(
+          tk, tv, a);
+      MOBA_CUDA(cudaGetLastError());
+    }
+  }
+  Timed tm(kKBwFinish, st);
+  const int64_t nq = pr.T * pr.Hq * D, nk = pr.T * pr.Hkv * D;
+  bw_finish_kernel<<<(unsigned)((nq / 4 + 255) / 256 + 1), 256, 0, st>>>(
+      b.dq32, static_cast<__nv_bfloat16*>(dq), nq);
+  bw_finish_kernel<<<(unsigned)((nk / 4 + 255) / 256 + 1), 256, 0, st>>>(
+      b.dk32, static_cast<__nv_bfloat16*>(dk), nk);
+  bw_finish_kernel<<<(unsigned)((nk / 4 + 255) / 256 + 1), 256, 0, st>>>(
+      b.dv32, static_cast<__nv_bfloat16*>(dv), nk);
+  return cuda_status(cudaGetLastError());
+}
+
+moba_status backward_impl(const Problem& pr, const void* q, const void* k, const void* v,
+                          const void* o, const float* lse, const void* dO, const int32_t* sel,
+                          void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                          cudaStream_t st) {
+  if (!q || !k || !v || !o || !lse || !dO || !sel || !dq || !dk || !dv)
+    return MOBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3) || (reinterpret_cast<uintptr_t>(sel) & 3))
+    return MOBA_ERR_INVALID_ARG;
+  if (!topk_supported(pr)) return MOBA_ERR_UNSUPPORTED;
+  if ((int64_t)pr.T * pr.G * (pr.topk > 1 ? pr.topk - 1 : 1) >= INT32_MAX)
+    return MOBA_ERR_UNSUPPORTED;
+  MOBA_TRY(check_ws(ws, ws_bytes, carve_bw(pr, 1, nullptr).bytes));
+  if (pr.T == 0) return MOBA_OK;
+  int nu = 1;
+  while (nu < pr.Hkv && carve_bw(pr, nu + 1, nullptr).bytes <= ws_bytes &&
+         (int64_t)(nu + 1) * pr.T * pr.G * (pr.topk > 1 ? pr.topk - 1 : 1) < INT32_MAX)
+    ++nu;
+  const BwWs b = carve_bw(pr, nu, static_cast<char*>(ws));
+  return pr.D == 128 ? backward_passes<128>(pr, q, k, v, o, lse, dO, sel, dq, dk, dv, b, nu, st)
+                     : backward_passes<64>(pr, q, k, v, o, lse, dO, sel, dq, dk, dv, b, nu, st);
 }
 
 // ---------------------------------------------------------------- decode
@@ -906,6 +1166,77 @@ int moba_profile_read(moba_kernel_time* out, int max_entries) {
     ++n;
   }
   return n;
+}
+
+// ---------------------------------------------------------------- routing variants
+moba_status moba_gate_minmax(const void* q, const void* k, int32_t* sel, const moba_params* p,
+                             void* ws, size_t ws_bytes, moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  if (!q || !k || !sel || !aligned16(q) || !aligned16(k) ||
+      (reinterpret_cast<uintptr_t>(sel) & 3))
+    return MOBA_ERR_INVALID_ARG;
+  if (!topk_supported(pr)) return MOBA_ERR_UNSUPPORTED;
+  MOBA_TRY(check_ws(ws, ws_bytes, carve(pr, 1, nullptr).bytes));
+  if (pr.T == 0) return MOBA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const Ws w = carve(pr, 1, static_cast<char*>(ws));
+  MOBA_TRY(run_plan(pr, w, st));
+  MOBA_TRY(run_minmax_pool(pr, k, w, st));
+  return pr.D == 128 ? launch_gate_minmax<128>(pr, q, w, sel, nullptr, st)
+                     : launch_gate_minmax<64>(pr, q, w, sel, nullptr, st);
+}
+
+moba_status moba_static_selection(int32_t* sel, int mode, const moba_params* p,
+                                  moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  if (!sel || (reinterpret_cast<uintptr_t>(sel) & 3)) return MOBA_ERR_INVALID_ARG;
+  if (mode != MOBA_ROUTE_WINDOW && mode != MOBA_ROUTE_SINK) return MOBA_ERR_INVALID_ARG;
+  const int64_t rows = (int64_t)pr.nseq * pr.Hq * pr.N;
+  if (rows == 0) return MOBA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Timed tm(kKStaticSel, st);
+  static_select_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(
+      sel, rows, pr.N, pr.Hq, pr.B, pr.topk, mode == MOBA_ROUTE_SINK ? kRouteSink : kRouteWindow);
+  return cuda_status(cudaGetLastError());
+}
+
+moba_status moba_forward_selected(const void* q, const void* k, const void* v, void* o,
+                                  float* lse, const int32_t* sel, const moba_params* p,
+                                  void* ws, size_t ws_bytes, moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  if (!sel) return MOBA_ERR_INVALID_ARG;
+  return forward_impl(pr, q, k, v, o, lse, const_cast<int32_t*>(sel), ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), kRouteGiven);
+}
+
+moba_status moba_forward_minmax(const void* q, const void* k, const void* v, void* o,
+                                float* lse, int32_t* sel_out, const moba_params* p, void* ws,
+                                size_t ws_bytes, moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  return forward_impl(pr, q, k, v, o, lse, sel_out, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), kRouteMinmaxGate);
+}
+
+// ---------------------------------------------------------------- backward
+size_t moba_backward_workspace_size(const moba_params* p, int heads_per_pass) {
+  Problem pr;
+  if (make_problem(p, false, nullptr, 0, 0, true, &pr) != MOBA_OK) return 0;
+  int nu = (heads_per_pass <= 0 || heads_per_pass > pr.Hkv) ? pr.Hkv : heads_per_pass;
+  return carve_bw(pr, nu, nullptr).bytes;
+}
+
+moba_status moba_backward(const void* q, const void* k, const void* v, const void* o,
+                          const float* lse, const void* dO, const int32_t* sel, void* dq,
+                          void* dk, void* dv, const moba_params* p, void* ws, size_t ws_bytes,
+                          moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  return backward_impl(pr, q, k, v, o, lse, dO, sel, dq, dk, dv, ws, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------- decode

@@ -130,6 +130,66 @@ moba_status moba_forward_varlen(const void *q, const void *k, const void *v,
                                 void *o, float *lse, int32_t *sel_out, const moba_params *p,
                                 void *ws, size_t ws_bytes, moba_stream_t stream);
 
+/* ----------------------------------------------------------------- backward
+ * Gradients of the forward's attention for an output gradient dO, over the
+ * selection the forward used (batch layout).  No gradient passes through the
+ * hard top-k gate (wispaper.ai blog, "The Change": the gradient does not flow
+ * through the discrete selection), so sel is an input: for every row and
+ * head, with P the attention probabilities over the chosen keys (from q, k
+ * and the forward's lse) and D = dO . o,
+ *   dS_u = P_u (dO . v_u - D),  dq = scale sum_u dS_u k_u,
+ *   dk_u += scale dS_u q,       dv_u += P_u dO.
+ * Inputs: q, k, v, o, dO as the forward's layouts (bf16), lse [batch][Hq][seqlen]
+ * fp32 and sel [batch][Hq][seqlen][top_k] exactly as moba_forward wrote them.
+ * Outputs dq [batch][seqlen][Hq][d], dk / dv [batch][seqlen][Hkv][d], bf16.
+ * The workspace holds the fp32 accumulators (moba_backward_workspace_size;
+ * heads_per_pass as for the forward). */
+size_t moba_backward_workspace_size(const moba_params *p, int heads_per_pass);
+moba_status moba_backward(const void *q, const void *k, const void *v, const void *o,
+                          const float *lse, const void *dO, const int32_t *sel, void *dq,
+                          void *dk, void *dv, const moba_params *p, void *ws, size_t ws_bytes,
+                          moba_stream_t stream);
+
+/* ------------------------------------------------------- routing variants
+ * The pages present the gate as one member of a family (batch layout only
+ * here): sliding-window attention is a gate that always selects the most
+ * recent blocks, sink attention one that always selects the initial and the
+ * most recent blocks (wispaper.ai blog, "Why the Change Is Plausible"), and
+ * Quest is MoBA with smaller blocks and min/max pooling (elamur summary
+ * card, "Key points").  A selection written by any of these has the gate's
+ * format: for a row in block i, exactly min(top_k - 1, i) past blocks
+ * ascending, then i, then -1 padding. */
+typedef enum moba_route_mode {
+  MOBA_ROUTE_WINDOW = 0, /* the own block and the top_k - 1 most recent past blocks */
+  MOBA_ROUTE_SINK = 1    /* block 0, the top_k - 2 most recent past blocks, the own block */
+} moba_route_mode;
+
+/* Static selection (no scores) into sel [batch][num_q_heads][seqlen][top_k];
+ * with fewer than top_k blocks every block is kept.  No workspace. */
+moba_status moba_static_selection(int32_t *sel, int mode, const moba_params *p,
+                                  moba_stream_t stream);
+
+/* Gate with min/max-pooled blocks: the elementwise max M_j and min m_j of
+ * each block's keys, score s_j = sum_c max(q_c M_jc, q_c m_jc) (Quest's bound
+ * on q . k over the block), then the same top-k, causality and tie rules as
+ * moba_gate.  Workspace: moba_workspace_size(p, 1). */
+moba_status moba_gate_minmax(const void *q, const void *k, int32_t *sel, const moba_params *p,
+                             void *ws, size_t ws_bytes, moba_stream_t stream);
+
+/* Forward over a caller-given selection sel [batch][num_q_heads][seqlen][top_k]
+ * in the gate's format (e.g. from moba_static_selection or moba_gate_minmax):
+ * no scoring; the attention, merge and outputs as moba_forward.  Entries that
+ * break the format (a past block >= the own block, a -1 among the first
+ * min(top_k - 1, i)) latch MOBA_ERR_DEVICE_CHECK. */
+moba_status moba_forward_selected(const void *q, const void *k, const void *v, void *o,
+                                  float *lse, const int32_t *sel, const moba_params *p,
+                                  void *ws, size_t ws_bytes, moba_stream_t stream);
+
+/* moba_gate_minmax followed by moba_forward_selected, in one call. */
+moba_status moba_forward_minmax(const void *q, const void *k, const void *v, void *o,
+                                float *lse, int32_t *sel_out, const moba_params *p, void *ws,
+                                size_t ws_bytes, moba_stream_t stream);
+
 /* Dense causal attention over every earlier token of each sequence: the
  * k = n limit of the method (wispaper.ai blog, "The Change": k = n
  * recovers full attention).  block_size and top_k are not used. */
@@ -214,7 +274,8 @@ moba_status moba_last_device_status(void *ws, moba_stream_t stream);
  * moba_profile_read synchronises those events and returns, per kernel class
  * (plan, pool, gate, gate_count, bucket_scan, bucket_scatter, attn_routed,
  * attn_own, merge, attn_dense, kbar_cache, decode_gate, decode_attn,
- * decode_merge), the launch count and summed device milliseconds since the
+ * decode_merge, minmax_pool, gate_minmax, static_select, bw_prep, bw_kv,
+ * bw_q, bw_finish), the launch count and summed device milliseconds since the
  * last reset.  Returns the number of classes written (<= max_entries).
  * Not thread safe; meant for one benchmarking thread. */
 typedef struct moba_kernel_time {
