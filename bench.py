@@ -378,13 +378,20 @@ def run_moba(args, w):
             h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh))
             d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
 
-            def estep():
-                q.copy_(qh, non_blocking=True)
-                k.copy_(kh, non_blocking=True)
-                v.copy_(vh, non_blocking=True)
-                step()
-                oh.copy_(o, non_blocking=True)
-                lh.copy_(lse, non_blocking=True)
+            if not varlen and route == "gate":
+                # the library's host-buffer call: copies inside, overlapped with the work
+                hbuf = moba.alloc_workspace(moba.forward_host_buffer_size(p, hp), dev)
+
+                def estep():
+                    moba.forward_host(qh, kh, vh, w.B, w.k, oh, lh, dev_buf=hbuf)
+            else:
+                def estep():
+                    q.copy_(qh, non_blocking=True)
+                    k.copy_(kh, non_blocking=True)
+                    v.copy_(vh, non_blocking=True)
+                    step()
+                    oh.copy_(o, non_blocking=True)
+                    lh.copy_(lse, non_blocking=True)
 
             estep()
             torch.cuda.synchronize()
@@ -397,7 +404,13 @@ def run_moba(args, w):
             torch.cuda.synchronize()
             ems = max_over_ranks(e0.elapsed_time(e1) / n_e)
             e2e = {"value": world * flops / (ems / 1e3) / 1e12, "unit": "TFLOP/s",
-                   "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+                   "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                   "call": ("moba_forward_host (copies inside the call)"
+                            if not varlen and route == "gate" else
+                            "host copies + moba_forward")}
+            e2e_status = moba.last_device_status(hbuf) if (not varlen and route == "gate") else 0
+            if e2e_status != 0:
+                e2e["device_status"] = e2e_status
             del qh, kh, vh, oh, lh
         except RuntimeError as exc:  # pinned allocation refused
             e2e = {"value": None, "unit": "TFLOP/s", "error": str(exc)[:200]}

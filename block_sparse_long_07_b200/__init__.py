@@ -30,7 +30,8 @@ EXPORTS = ("moba_workspace_size", "moba_workspace_size_varlen", "moba_gate", "mo
            "moba_profile_read", "moba_selftest_wait_timeout", "moba_decode_workspace_size",
            "moba_kbar_cache_size", "moba_kbar_cache_update", "moba_decode",
            "moba_static_selection", "moba_gate_minmax", "moba_forward_selected",
-           "moba_forward_minmax", "moba_backward_workspace_size", "moba_backward")
+           "moba_forward_minmax", "moba_backward_workspace_size", "moba_backward",
+           "moba_forward_host_buffer_size", "moba_forward_host")
 
 ROUTE_WINDOW, ROUTE_SINK = 0, 1
 
@@ -119,6 +120,10 @@ def load_library(path=None):
     lib.moba_forward_selected.argtypes = [vp, vp, vp, vp, vp, vp, pp, vp, sz, vp]
     lib.moba_forward_minmax.restype = i32
     lib.moba_forward_minmax.argtypes = [vp, vp, vp, vp, vp, vp, pp, vp, sz, vp]
+    lib.moba_forward_host_buffer_size.restype = sz
+    lib.moba_forward_host_buffer_size.argtypes = [pp, i32]
+    lib.moba_forward_host.restype = i32
+    lib.moba_forward_host.argtypes = [vp, vp, vp, vp, vp, vp, pp, vp, sz, vp]
     lib.moba_backward_workspace_size.restype = sz
     lib.moba_backward_workspace_size.argtypes = [pp, i32]
     lib.moba_backward.restype = i32
@@ -497,3 +502,30 @@ def backward(q, k, v, o, lse, dO, sel, block_size, top_k, softmax_scale=0.0, ws=
                                         ctypes.byref(p), _ptr(ws), ws.numel(), _stream(stream)),
            "moba_backward")
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------- host-buffer forward
+def forward_host_buffer_size(params, heads_per_pass=0):
+    return int(load_library().moba_forward_host_buffer_size(ctypes.byref(params),
+                                                            int(heads_per_pass)))
+
+
+def forward_host(q, k, v, block_size, top_k, out, lse, dev_buf=None, heads_per_pass=0,
+                 softmax_scale=0.0, sel_out=None, stream=None):
+    """MoBA forward on host (preferably pinned) tensors q [b,N,Hq,d], k/v
+    [b,N,Hkv,d]; writes the host tensors out [b,N,Hq,d] and lse [b,Hq,N].
+    The copies run inside the call, overlapped with the work of other kv-head
+    groups; synchronise the stream before reading out."""
+    torch = _torch()
+    for t in (q, k, v, out):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("expected contiguous bf16 host tensors")
+    b, N, Hq, d = q.shape
+    p = make_params(b, N, Hq, k.shape[2], d, block_size, top_k, softmax_scale)
+    if dev_buf is None:
+        dev_buf = alloc_workspace(forward_host_buffer_size(p, heads_per_pass))
+    _check(load_library().moba_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                            _ptr(sel_out), ctypes.byref(p), _ptr(dev_buf),
+                                            dev_buf.numel(), _stream(stream)),
+           "moba_forward_host")
+    return out, lse

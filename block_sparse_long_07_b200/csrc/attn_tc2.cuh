@@ -59,7 +59,7 @@ struct AttnArgs {
   const int32_t* tile_off;   // routed: [nu*NB + 1] work items per bucket, prefix
   const int32_t* entry_off;  // routed: [nu*NB + 1] bucket entries, prefix
   const uint2* entries;
-  __nv_bfloat16* part_O;     // [nu][T][G][topk-1][D]
+  __half* part_O;            // [nu][T][G][topk-1][D], fp16 (see the epilogue)
   float* part_lse;           // [nu][T][G][topk-1]
   float* own_O;              // [nu][T][G][D]
   float* own_lse;            // [nu][T][G]
@@ -563,8 +563,9 @@ __global__ void __launch_bounds__(352, 1)
       const float inv = 1.f / l_run;
       const float lse2 = m_run + lg2_approx(l_run);
       // destination of this row
-      int kind = 0;  // 0 skip, 1 bf16 partial, 2 fp32 partial, 3 final
+      int kind = 0;  // 0 skip, 1 fp16 partial, 2 fp32 partial, 3 final (bf16)
       __nv_bfloat16* dst16 = nullptr;
+      __half* dsth = nullptr;
       float* dst32 = nullptr;
       float* lse_dst = nullptr;
       float lse_val = lse2;
@@ -576,7 +577,7 @@ __global__ void __launch_bounds__(352, 1)
             const int64_t prow =
                 (((int64_t)it.u * a.L.T + e.x) * a.G + hh) * (a.topk - 1) + sl;
             kind = 1;
-            dst16 = a.part_O + prow * D;
+            dsth = a.part_O + prow * D;
             lse_dst = a.part_lse + prow;
           } else {
             atomicOr(a.status, MOBA_DEV_BAD_INDEX);
@@ -602,7 +603,7 @@ __global__ void __launch_bounds__(352, 1)
         uint32_t ov[32];
         tmem_ld32(tO + c4 * 32, ov);
         tc_wait_ld();
-        if (kind == 1 || kind == 3) {
+        if (kind == 3) {
           uint4* d4 = reinterpret_cast<uint4*>(dst16 + c4 * 32);
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
@@ -612,6 +613,24 @@ __global__ void __launch_bounds__(352, 1)
                                 pack_bf16x2(f[4] * inv, f[5] * inv),
                                 pack_bf16x2(f[6] * inv, f[7] * inv));
           }
+        } else if (kind == 1) {
+          // Routed partial O in fp16: a convex combination of V rows, so
+          // |O| <= max |v|; 8x finer than bf16, for the second rounding
+          // the merge adds before the final bf16 output.  Beyond the fp16
+          // range (|v| > 65504) the status word records it.
+          uint4* d4 = reinterpret_cast<uint4*>(dsth + c4 * 32);
+          float mx = 0.f;
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            const float* f = reinterpret_cast<const float*>(&ov[q8 * 8]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e] * inv));
+            d4[q8] = make_uint4(pack_half2(f[0] * inv, f[1] * inv),
+                                pack_half2(f[2] * inv, f[3] * inv),
+                                pack_half2(f[4] * inv, f[5] * inv),
+                                pack_half2(f[6] * inv, f[7] * inv));
+          }
+          if (!(mx <= 65504.f)) atomicOr(a.status, MOBA_DEV_CAPACITY);
         } else if (kind == 2) {
           float4* d4 = reinterpret_cast<float4*>(dst32 + c4 * 32);
 #pragma unroll

@@ -112,11 +112,12 @@ __global__ void plan_kernel(SeqLayout L, int B, Plan P, int NBmax, int NQTmax,
 // Grid (NBmax, Hkv), 256 threads; 16-byte loads, fixed summation order.
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ k, int Hkv,
-                                                   Plan P, int NBmax, float* __restrict__ kbar) {
+                                                   Plan P, int NBmax, float* __restrict__ kbar,
+                                                   int g0 = 0) {
   constexpr int CH = D / 8;          // 16-byte chunks per row
   constexpr int RPI = 256 / CH;      // rows per iteration
   __shared__ float red[RPI][D + 4];
-  const int J = blockIdx.x, g = blockIdx.y;
+  const int J = blockIdx.x, g = g0 + blockIdx.y;  // kv heads g0 .. g0 + gridDim.y - 1
   if (J >= P.totals[0]) return;
   const int64_t t0 = P.blk_tok[J];
   const int len = P.blk_len[J];
@@ -177,11 +178,11 @@ template <int D, int KM>
 __global__ void __launch_bounds__(128) gate_kernel(
     const __nv_bfloat16* __restrict__ q, int Hq, int G, int B, int topk, SeqLayout L, Plan P,
     int NBmax, const float* __restrict__ kbar, int32_t* __restrict__ sel, RowLayout R,
-    uint32_t* __restrict__ count_out, uint32_t* __restrict__ status) {
+    uint32_t* __restrict__ count_out, uint32_t* __restrict__ status, int h0 = 0) {
   extern __shared__ __align__(16) unsigned char gate_smem[];
   float* kb = reinterpret_cast<float*>(gate_smem);                             // [chunk][D]
   uint32_t* cnt = reinterpret_cast<uint32_t*>(kb + kGateChunk * D);           // [blocks]
-  const int qt = blockIdx.x, h = blockIdx.y;
+  const int qt = blockIdx.x, h = h0 + blockIdx.y;  // q heads h0 .. h0 + gridDim.y - 1
   if (qt >= P.totals[1]) return;
   const int s = upper_index(P.qt_off, L.nseq + 1, qt);
   const int64_t st = seq_start(L, s), len = seq_len(L, s);
@@ -464,7 +465,7 @@ __global__ void __launch_bounds__(128) bucket_scatter_kernel(
 // order.
 template <int D>
 __global__ void __launch_bounds__(256) merge_kernel(
-    const __nv_bfloat16* __restrict__ part_O, const float* __restrict__ part_lse,
+    const __half* __restrict__ part_O, const float* __restrict__ part_lse,
     const float* __restrict__ own_O, const float* __restrict__ own_lse, int topk, int B, int G,
     int Hq, int u0, int nu, SeqLayout L, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
     RowLayout R) {
@@ -520,10 +521,10 @@ __global__ void __launch_bounds__(256) merge_kernel(
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       den += w[q];
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[q]);
+      const __half2* h2 = reinterpret_cast<const __half2*>(&v[q]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h2[e]);
+        const float2 f = __half22float2(h2[e]);
         acc[2 * e] = fmaf(w[q], f.x, acc[2 * e]);
         acc[2 * e + 1] = fmaf(w[q], f.y, acc[2 * e + 1]);
       }
@@ -533,10 +534,10 @@ __global__ void __launch_bounds__(256) merge_kernel(
     const uint4 v = orow[sl * kStride];
     const float w = ex2_approx(lrow[sl] - m);
     den += w;
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+    const __half2* h2 = reinterpret_cast<const __half2*>(&v);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(h2[e]);
+      const float2 f = __half22float2(h2[e]);
       acc[2 * e] = fmaf(w, f.x, acc[2 * e]);
       acc[2 * e + 1] = fmaf(w, f.y, acc[2 * e + 1]);
     }

@@ -9,6 +9,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -314,11 +315,11 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1) 
 
 // 2^x for a pair on the FMA pipe, to take load off the special-function unit.
 // Range reduction x = j + f with j = round(x) (the 1.5 * 2^23 rounding
-// constant), |f| <= 1/2; 2^f by a degree-3 minimax polynomial fitted on
-// [-1/2, 1/2] (linear program on 4001 points, relative error 7.5e-5); j is
-// added into the exponent field.  x is clamped below at -126, so the result
-// stays finite (below 2^-125 there).  The caller rounds the result to bf16
-// (relative step 2^-8), far coarser than the polynomial's error.
+// constant), |f| <= 1/2; 2^f by a degree-4 minimax polynomial fitted on
+// [-1/2, 1/2] (linear program on 4001 points, relative error 2.6e-6, so that
+// the bf16 rounding of P the caller applies next almost never differs from
+// that of the exact value); j is added into the exponent field.  x is clamped
+// below at -126, so the result stays finite (below 2^-125 there).
 __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
   x0 = fmaxf(x0, -126.f);
   x1 = fmaxf(x1, -126.f);
@@ -329,10 +330,11 @@ __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float
   float f0 = x0, f1 = x1;
   fadd2(f0, f1, -j0, -j1);
   float p0, p1;
-  ffma2(p0, p1, 0.0551716685295105f, 0.0551716685295105f, f0, f1, 0.2426111251115799f,
-        0.2426111251115799f);
-  ffma2(p0, p1, p0, p1, f0, f1, 0.6932609677314758f, 0.6932609677314758f);
-  ffma2(p0, p1, p0, p1, f0, f1, 0.9999280571937561f, 0.9999280571937561f);
+  ffma2(p0, p1, 0.009569705463945866f, 0.009569705463945866f, f0, f1, 0.05591819807887077f,
+        0.05591819807887077f);
+  ffma2(p0, p1, p0, p1, f0, f1, 0.24024765193462372f, 0.24024765193462372f);
+  ffma2(p0, p1, p0, p1, f0, f1, 0.6931217312812805f, 0.6931217312812805f);
+  ffma2(p0, p1, p0, p1, f0, f1, 0.9999992251396179f, 0.9999992251396179f);
   y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
   y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
@@ -355,6 +357,10 @@ __device__ __forceinline__ float fmax3f(float a, float b, float c) {
 }
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 

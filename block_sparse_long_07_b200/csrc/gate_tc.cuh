@@ -61,6 +61,7 @@ struct GateTcArgs {
   RowLayout R;
   int32_t* sel;
   uint32_t* status;
+  int g0, ng;  // kv heads g0 .. g0 + ng - 1 (their items are contiguous)
 };
 
 template <int D>
@@ -192,8 +193,9 @@ __global__ void __launch_bounds__(352, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int64_t items = (int64_t)a.P.totals[1] * a.Hq;
-  const int64_t first = blockIdx.x, step = gridDim.x;
+  const int64_t per_g = (int64_t)a.P.totals[1] * a.G;
+  const int64_t items = (int64_t)(a.g0 + a.ng) * per_g;
+  const int64_t first = (int64_t)a.g0 * per_g + blockIdx.x, step = gridDim.x;
   uint32_t* st = a.status;
   const int npast = a.topk - 1;
 
@@ -488,9 +490,9 @@ __global__ void __launch_bounds__(352, 1)
 // kv head g.  One CTA per (query tile, kv head), counters in shared memory.
 __global__ void __launch_bounds__(128) gate_count_kernel(
     const int32_t* __restrict__ sel, RowLayout R, int topk, int B, int G, SeqLayout L, Plan P,
-    int NBmax, uint32_t* __restrict__ counts, uint32_t* __restrict__ status) {
+    int NBmax, uint32_t* __restrict__ counts, uint32_t* __restrict__ status, int g0 = 0) {
   extern __shared__ uint32_t ccnt[];  // [blocks of the sequence]
-  const int qt = blockIdx.x, g = blockIdx.y;
+  const int qt = blockIdx.x, g = g0 + blockIdx.y;  // kv heads g0 .. g0 + gridDim.y - 1
   if (qt >= P.totals[1]) return;
   const int s = upper_index(P.qt_off, L.nseq + 1, qt);
   const int64_t st = seq_start(L, s), len = seq_len(L, s);

@@ -125,7 +125,7 @@ struct Ws {
   int32_t* tile_off;
   uint32_t* cursor;
   uint2* entries;
-  __nv_bfloat16* part_O;
+  __half* part_O;  // routed partial O, fp16
   float* part_lse;
   float* own_O;
   float* own_lse;
@@ -161,7 +161,7 @@ Ws carve(const Problem& pr, int nu, char* base) {
   w.cursor = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * (size_t)nu * NB));
   const size_t prow = (size_t)nu * pr.T * pr.G;  // partial rows per pass
   w.entries = reinterpret_cast<uint2*>(take(sizeof(uint2) * prow * np));
-  w.part_O = reinterpret_cast<__nv_bfloat16*>(take(2 * prow * np * pr.D));
+  w.part_O = reinterpret_cast<__half*>(take(2 * prow * np * pr.D));
   w.part_lse = reinterpret_cast<float*>(take(sizeof(float) * prow * np));
   w.own_O = reinterpret_cast<float*>(take(sizeof(float) * prow * pr.D));
   w.own_lse = reinterpret_cast<float*>(take(sizeof(float) * prow));
@@ -299,17 +299,17 @@ moba_status launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
 
 template <int D, int KM>
 moba_status launch_gate_km(const Problem& pr, const void* q, const Ws& w, int32_t* sel,
-                           uint32_t* counts, cudaStream_t st) {
+                           uint32_t* counts, cudaStream_t st, int g0, int ng) {
   const size_t smem = sizeof(float) * kGateChunk * D + sizeof(uint32_t) * kMaxBlocksPerSeq;
   auto kern = gate_kernel<D, KM>;
   if (smem > 48 * 1024)
     MOBA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
-  dim3 grid((unsigned)pr.NQTmax, (unsigned)pr.Hq);
+  dim3 grid((unsigned)pr.NQTmax, (unsigned)(ng * pr.G));
   Timed tm(kKGate, st);
   kern<<<grid, 128, smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(q), pr.Hq, pr.G, pr.B,
                                 pr.topk, L, w.P, (int)pr.NBmax, w.kbar, sel, pr.R, counts,
-                                w.status);
+                                w.status, g0 * pr.G);
   return cuda_status(cudaGetLastError());
 }
 
@@ -317,7 +317,7 @@ moba_status launch_gate_km(const Problem& pr, const void* q, const Ws& w, int32_
 // the bucket sizes from the written selections.
 template <int D, int KM>
 moba_status launch_gate_tc_km(const Problem& pr, const void* q, const Ws& w, int32_t* sel,
-                              uint32_t* counts, cudaStream_t st) {
+                              uint32_t* counts, cudaStream_t st, int g0, int ng) {
   using C = GateTcCfg<D>;
   CUtensorMap tq;
   if (!make_tmap(&tq, q, pr.Hq, pr.T, D)) return MOBA_ERR_CUDA;
@@ -339,6 +339,8 @@ moba_status launch_gate_tc_km(const Problem& pr, const void* q, const Ws& w, int
   a.R = pr.R;
   a.sel = sel;
   a.status = w.status;
+  a.g0 = g0;
+  a.ng = ng;
   {
     Timed tm(kKGate, st);
     kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, a);
@@ -346,10 +348,10 @@ moba_status launch_gate_tc_km(const Problem& pr, const void* q, const Ws& w, int
   }
   if (counts) {
     const size_t smem = sizeof(uint32_t) * kMaxBlocksPerSeq;
-    dim3 cgrid((unsigned)pr.NQTmax, (unsigned)pr.Hkv);
+    dim3 cgrid((unsigned)pr.NQTmax, (unsigned)ng);
     Timed tm(kKGateCount, st);
     gate_count_kernel<<<cgrid, 128, smem, st>>>(sel, pr.R, pr.topk, pr.B, pr.G, L, w.P,
-                                                (int)pr.NBmax, counts, w.status);
+                                                (int)pr.NBmax, counts, w.status, g0);
     MOBA_CUDA(cudaGetLastError());
   }
   return MOBA_OK;
@@ -362,30 +364,32 @@ bool gate_tc_fits(const Problem& pr) {
          pr.max_blocks_per_seq - 1 <= kGateTcMaxPast;
 }
 
+// The gate for the q heads of kv heads g0 .. g0 + ng - 1 (default: all).
 template <int D>
 moba_status launch_gate(const Problem& pr, const void* q, const Ws& w, int32_t* sel,
-                        uint32_t* counts, cudaStream_t st) {
+                        uint32_t* counts, cudaStream_t st, int g0 = 0, int ng = -1) {
+  if (ng < 0) ng = pr.Hkv;
   const int64_t npast = pr.topk - 1;
   if (gate_tc_fits(pr)) {
     switch (pow2_at_least(npast)) {
-      case 1: return launch_gate_tc_km<D, 1>(pr, q, w, sel, counts, st);
-      case 2: return launch_gate_tc_km<D, 2>(pr, q, w, sel, counts, st);
-      case 4: return launch_gate_tc_km<D, 4>(pr, q, w, sel, counts, st);
-      case 8: return launch_gate_tc_km<D, 8>(pr, q, w, sel, counts, st);
+      case 1: return launch_gate_tc_km<D, 1>(pr, q, w, sel, counts, st, g0, ng);
+      case 2: return launch_gate_tc_km<D, 2>(pr, q, w, sel, counts, st, g0, ng);
+      case 4: return launch_gate_tc_km<D, 4>(pr, q, w, sel, counts, st, g0, ng);
+      case 8: return launch_gate_tc_km<D, 8>(pr, q, w, sel, counts, st, g0, ng);
       default:
-        if (npast <= 12) return launch_gate_tc_km<D, 12>(pr, q, w, sel, counts, st);
-        return launch_gate_tc_km<D, 16>(pr, q, w, sel, counts, st);
+        if (npast <= 12) return launch_gate_tc_km<D, 12>(pr, q, w, sel, counts, st, g0, ng);
+        return launch_gate_tc_km<D, 16>(pr, q, w, sel, counts, st, g0, ng);
     }
   }
   const int64_t need = (npast >= pr.max_blocks_per_seq - 1) ? 1 : npast;
   switch (pow2_at_least(need)) {
-    case 1: return launch_gate_km<D, 1>(pr, q, w, sel, counts, st);
-    case 2: return launch_gate_km<D, 2>(pr, q, w, sel, counts, st);
-    case 4: return launch_gate_km<D, 4>(pr, q, w, sel, counts, st);
-    case 8: return launch_gate_km<D, 8>(pr, q, w, sel, counts, st);
-    case 16: return launch_gate_km<D, 16>(pr, q, w, sel, counts, st);
-    case 32: return launch_gate_km<D, 32>(pr, q, w, sel, counts, st);
-    case 64: return launch_gate_km<D, 64>(pr, q, w, sel, counts, st);
+    case 1: return launch_gate_km<D, 1>(pr, q, w, sel, counts, st, g0, ng);
+    case 2: return launch_gate_km<D, 2>(pr, q, w, sel, counts, st, g0, ng);
+    case 4: return launch_gate_km<D, 4>(pr, q, w, sel, counts, st, g0, ng);
+    case 8: return launch_gate_km<D, 8>(pr, q, w, sel, counts, st, g0, ng);
+    case 16: return launch_gate_km<D, 16>(pr, q, w, sel, counts, st, g0, ng);
+    case 32: return launch_gate_km<D, 32>(pr, q, w, sel, counts, st, g0, ng);
+    case 64: return launch_gate_km<D, 64>(pr, q, w, sel, counts, st, g0, ng);
     default: return MOBA_ERR_UNSUPPORTED;
   }
 }
@@ -432,6 +436,20 @@ moba_status check_ws(void* ws, size_t ws_bytes, size_t need) {
   return MOBA_OK;
 }
 
+// Block means of kv heads g0 .. g0 + ng - 1.
+moba_status run_pool(const Problem& pr, const void* k, const Ws& w, cudaStream_t st, int g0,
+                     int ng) {
+  dim3 grid((unsigned)pr.NBmax, (unsigned)ng);
+  Timed tm(kKPool, st);
+  if (pr.D == 128)
+    pool_kernel<128><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(k), pr.Hkv,
+                                           w.P, (int)pr.NBmax, w.kbar, g0);
+  else
+    pool_kernel<64><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(k), pr.Hkv,
+                                          w.P, (int)pr.NBmax, w.kbar, g0);
+  return cuda_status(cudaGetLastError());
+}
+
 moba_status run_plan_pool(const Problem& pr, const void* k, const Ws& w, cudaStream_t st) {
   SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
   {
@@ -439,16 +457,7 @@ moba_status run_plan_pool(const Problem& pr, const void* k, const Ws& w, cudaStr
     plan_kernel<<<1, 1024, 0, st>>>(L, pr.B, w.P, (int)pr.NBmax, (int)pr.NQTmax, w.status);
   }
   MOBA_CUDA(cudaGetLastError());
-  dim3 grid((unsigned)pr.NBmax, (unsigned)pr.Hkv);
-  Timed tm(kKPool, st);
-  if (pr.D == 128)
-    pool_kernel<128><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(k), pr.Hkv,
-                                           w.P, (int)pr.NBmax, w.kbar);
-  else
-    pool_kernel<64><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(k), pr.Hkv,
-                                          w.P, (int)pr.NBmax, w.kbar);
-  MOBA_CUDA(cudaGetLastError());
-  return MOBA_OK;
+  return run_pool(pr, k, w, st, 0, pr.Hkv);
 }
 
 // How a forward obtains its selection.
@@ -535,23 +544,19 @@ moba_status gate_impl(const Problem& pr, const void* q, const void* k, int32_t* 
                      : launch_gate<64>(pr, q, w, sel, nullptr, st);
 }
 
-template <int D>
-moba_status forward_passes(const Problem& pr, const void* q, const void* k, const void* v,
-                           void* o, float* lse, const Ws& w, int32_t* sel, int nu_max,
-                           int route, cudaStream_t st) {
+// Attention arguments and tensor maps of one forward call.
+struct FwdCtx {
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, pr.Hq, pr.T, D) || !make_tmap(&tk, k, pr.Hkv, pr.T, D) ||
-      !make_tmap(&tv, v, pr.Hkv, pr.T, D))
-    return MOBA_ERR_CUDA;
-  SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
-  MOBA_CUDA(cudaMemsetAsync(w.counts, 0, sizeof(uint32_t) * (size_t)pr.Hkv * pr.NBmax, st));
-  if (route == kRouteMeanGate)
-    MOBA_TRY(launch_gate<D>(pr, q, w, sel, w.counts, st));
-  else if (route == kRouteMinmaxGate)
-    MOBA_TRY(launch_gate_minmax<D>(pr, q, w, sel, w.counts, st));
-  else if (pr.topk > 1)
-    MOBA_TRY(launch_count(pr, w, sel, w.counts, st));
   AttnArgs a;
+};
+
+template <int D>
+moba_status forward_setup(const Problem& pr, const void* q, const void* k, const void* v,
+                          void* o, float* lse, const Ws& w, FwdCtx* c) {
+  if (!make_tmap(&c->tq, q, pr.Hq, pr.T, D) || !make_tmap(&c->tk, k, pr.Hkv, pr.T, D) ||
+      !make_tmap(&c->tv, v, pr.Hkv, pr.T, D))
+    return MOBA_ERR_CUDA;
+  AttnArgs& a = c->a;
   memset(&a, 0, sizeof a);
   a.q = reinterpret_cast<const __nv_bfloat16*>(q);
   a.Hq = pr.Hq;
@@ -560,7 +565,7 @@ moba_status forward_passes(const Problem& pr, const void* q, const void* k, cons
   a.B = pr.B;
   a.topk = pr.topk;
   a.scale_log2 = pr.scale * 1.4426950408889634f;
-  a.L = L;
+  a.L = SeqLayout{pr.cu, pr.nseq, pr.N, pr.T};
   a.P = w.P;
   a.R = pr.R;
   a.tile_off = w.tile_off;
@@ -573,34 +578,191 @@ moba_status forward_passes(const Problem& pr, const void* q, const void* k, cons
   a.o = reinterpret_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.status = w.status;
-  for (int u0 = 0; u0 < pr.Hkv; u0 += nu_max) {
-    const int nu = (pr.Hkv - u0) < nu_max ? (pr.Hkv - u0) : nu_max;
-    a.u0 = u0;
-    a.nu = nu;
-    if (pr.topk > 1) {
-      {
-        Timed tm(kKScan, st);
-        bucket_scan_kernel<<<1, 1024, 0, st>>>(w.counts, u0, nu, 2 * kTileM, w.P,
-                                               (int)pr.NBmax, w.entry_off, w.tile_off,
-                                               w.cursor);
-      }
-      MOBA_CUDA(cudaGetLastError());
-      MOBA_TRY(launch_scatter(pr, w, sel, u0, nu, st));
-      MOBA_TRY((launch_attn<D, kRouted>(tq, tk, tv, a, 1, st)));
+  return MOBA_OK;
+}
+
+// Bucketing, routed and own-block attention and merge for kv heads u0 .. u0 + nu - 1
+// (their selection and bucket sizes already written).
+template <int D>
+moba_status forward_one_pass(const Problem& pr, FwdCtx& c, const Ws& w, const int32_t* sel,
+                             void* o, float* lse, int u0, int nu, cudaStream_t st) {
+  AttnArgs& a = c.a;
+  a.u0 = u0;
+  a.nu = nu;
+  if (pr.topk > 1) {
+    {
+      Timed tm(kKScan, st);
+      bucket_scan_kernel<<<1, 1024, 0, st>>>(w.counts, u0, nu, 2 * kTileM, w.P, (int)pr.NBmax,
+                                             w.entry_off, w.tile_off, w.cursor);
     }
-    MOBA_TRY((launch_attn<D, kOwn>(tq, tk, tv, a, pr.B % (2 * kTileM) == 0 ? 1 : 0, st)));
-    if (pr.topk > 1) {
-      const int64_t rows = pr.T * nu * pr.G;
-      const int64_t rows_per_block = 8 * (32 / (D / 8));
-      const unsigned blocks = (unsigned)((rows + rows_per_block - 1) / rows_per_block);
-      Timed tm(kKMerge, st);
-      merge_kernel<D><<<blocks, 256, 0, st>>>(w.part_O, w.part_lse, w.own_O, w.own_lse, pr.topk,
-                                              pr.B, pr.G, pr.Hq, u0, nu, L,
-                                              reinterpret_cast<__nv_bfloat16*>(o), lse, pr.R);
-      MOBA_CUDA(cudaGetLastError());
-    }
+    MOBA_CUDA(cudaGetLastError());
+    MOBA_TRY(launch_scatter(pr, w, sel, u0, nu, st));
+    MOBA_TRY((launch_attn<D, kRouted>(c.tq, c.tk, c.tv, a, 1, st)));
+  }
+  MOBA_TRY((launch_attn<D, kOwn>(c.tq, c.tk, c.tv, a, pr.B % (2 * kTileM) == 0 ? 1 : 0, st)));
+  if (pr.topk > 1) {
+    SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
+    const int64_t rows = pr.T * nu * pr.G;
+    const int64_t rows_per_block = 8 * (32 / (D / 8));
+    const unsigned blocks = (unsigned)((rows + rows_per_block - 1) / rows_per_block);
+    Timed tm(kKMerge, st);
+    merge_kernel<D><<<blocks, 256, 0, st>>>(w.part_O, w.part_lse, w.own_O, w.own_lse, pr.topk,
+                                            pr.B, pr.G, pr.Hq, u0, nu, L,
+                                            reinterpret_cast<__nv_bfloat16*>(o), lse, pr.R);
+    MOBA_CUDA(cudaGetLastError());
   }
   return MOBA_OK;
+}
+
+template <int D>
+moba_status forward_passes(const Problem& pr, const void* q, const void* k, const void* v,
+                           void* o, float* lse, const Ws& w, int32_t* sel, int nu_max,
+                           int route, cudaStream_t st) {
+  FwdCtx c;
+  MOBA_TRY(forward_setup<D>(pr, q, k, v, o, lse, w, &c));
+  MOBA_CUDA(cudaMemsetAsync(w.counts, 0, sizeof(uint32_t) * (size_t)pr.Hkv * pr.NBmax, st));
+  if (route == kRouteMeanGate)
+    MOBA_TRY(launch_gate<D>(pr, q, w, sel, w.counts, st));
+  else if (route == kRouteMinmaxGate)
+    MOBA_TRY(launch_gate_minmax<D>(pr, q, w, sel, w.counts, st));
+  else if (pr.topk > 1)
+    MOBA_TRY(launch_count(pr, w, sel, w.counts, st));
+  for (int u0 = 0; u0 < pr.Hkv; u0 += nu_max) {
+    const int nu = (pr.Hkv - u0) < nu_max ? (pr.Hkv - u0) : nu_max;
+    MOBA_TRY(forward_one_pass<D>(pr, c, w, sel, o, lse, u0, nu, st));
+  }
+  return MOBA_OK;
+}
+
+// ---------------------------------------------------------------- host-buffer forward
+// Device buffer of a forward on host buffers: the forward's workspace first
+// (its status word at offset 0, as for every workspace), then staging for
+// q, k, v, o, lse and sel.
+struct HostBufs {
+  char *q, *k, *v, *o;
+  float* lse;
+  int32_t* sel;
+  size_t staged;  // staging bytes
+};
+
+HostBufs carve_host(const Problem& pr, char* base, size_t ws_bytes) {
+  HostBufs h;
+  memset(&h, 0, sizeof h);
+  size_t off = align_up(ws_bytes);
+  auto take = [&](size_t bytes) -> char* {
+    char* p = base ? base + off : nullptr;
+    off = align_up(off + bytes);
+    return p;
+  };
+  const size_t qb = (size_t)pr.T * pr.Hq * pr.D * 2, kb = (size_t)pr.T * pr.Hkv * pr.D * 2;
+  h.q = take(qb);
+  h.k = take(kb);
+  h.v = take(kb);
+  h.o = take(qb);
+  h.lse = reinterpret_cast<float*>(take(sizeof(float) * (size_t)pr.T * pr.Hq));
+  h.sel = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)pr.T * pr.Hq * pr.topk));
+  h.staged = off - align_up(ws_bytes);
+  return h;
+}
+
+// Two copy streams per device (host -> device, device -> host), created on
+// first use.
+cudaStream_t copy_stream(int which) {
+  static std::mutex mu;
+  static cudaStream_t streams[64][2] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev][which] &&
+      cudaStreamCreateWithFlags(&streams[dev][which], cudaStreamNonBlocking) != cudaSuccess)
+    streams[dev][which] = nullptr;
+  return streams[dev][which];
+}
+
+// Columns [c0, c0 + nc) of a row-major [rows][ncols] array of `esz`-byte elements.
+cudaError_t copy_cols(void* dst, const void* src, int64_t rows, int64_t ncols, int64_t c0,
+                      int64_t nc, size_t esz, cudaMemcpyKind kind, cudaStream_t st) {
+  const size_t pitch = (size_t)ncols * esz;
+  return cudaMemcpy2DAsync(static_cast<char*>(dst) + c0 * esz, pitch,
+                           static_cast<const char*>(src) + c0 * esz, pitch, (size_t)nc * esz,
+                           (size_t)rows, kind, st);
+}
+
+// One pass per group of kv heads: its q / k / v columns go in on one copy
+// stream while the previous pass computes, its o / lse / sel come back on the
+// other while the next pass computes.
+template <int D>
+moba_status forward_host_passes(const Problem& pr, const void* q_h, const void* k_h,
+                                const void* v_h, void* o_h, float* lse_h, int32_t* sel_h,
+                                const HostBufs& hb, const Ws& w, int nu_max, cudaStream_t st) {
+  cudaStream_t h2d = copy_stream(0), d2h = copy_stream(1);
+  if (!h2d || !d2h) return MOBA_ERR_CUDA;
+  const int npass = (pr.Hkv + nu_max - 1) / nu_max;
+  std::vector<cudaEvent_t> ev((size_t)2 * npass + 1, nullptr);
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      for (auto& x : ev)
+        if (x) cudaEventDestroy(x);
+      return MOBA_ERR_CUDA;
+    }
+  cudaEvent_t start = ev[2 * npass];
+  auto fail = [&](moba_status s) {
+    for (auto& x : ev) cudaEventDestroy(x);  // released once any pending record completes
+    return s;
+  };
+  auto in_ready = [&](int p) { return ev[p]; };
+  auto done = [&](int p) { return ev[npass + p]; };
+  const int64_t rows_b = pr.nseq;                      // batch rows of lse / sel
+  const int64_t per_head_lse = pr.N, per_head_sel = (int64_t)pr.N * pr.topk;
+  if (cudaEventRecord(start, st) != cudaSuccess || cudaStreamWaitEvent(h2d, start, 0) != cudaSuccess)
+    return fail(MOBA_ERR_CUDA);
+  // inputs of every pass, in pass order, on the copy stream
+  for (int p = 0; p < npass; ++p) {
+    const int g0 = p * nu_max, ng = (pr.Hkv - g0) < nu_max ? (pr.Hkv - g0) : nu_max;
+    if (copy_cols(hb.k, k_h, pr.T, (int64_t)pr.Hkv * D, (int64_t)g0 * D, (int64_t)ng * D, 2,
+                  cudaMemcpyHostToDevice, h2d) != cudaSuccess ||
+        copy_cols(hb.q, q_h, pr.T, (int64_t)pr.Hq * D, (int64_t)g0 * pr.G * D,
+                  (int64_t)ng * pr.G * D, 2, cudaMemcpyHostToDevice, h2d) != cudaSuccess ||
+        copy_cols(hb.v, v_h, pr.T, (int64_t)pr.Hkv * D, (int64_t)g0 * D, (int64_t)ng * D, 2,
+                  cudaMemcpyHostToDevice, h2d) != cudaSuccess ||
+        cudaEventRecord(in_ready(p), h2d) != cudaSuccess)
+      return fail(MOBA_ERR_CUDA);
+  }
+  FwdCtx c;
+  moba_status r = forward_setup<D>(pr, hb.q, hb.k, hb.v, hb.o, hb.lse, w, &c);
+  if (r != MOBA_OK) return fail(r);
+  {
+    SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
+    Timed tm(kKPlan, st);
+    plan_kernel<<<1, 1024, 0, st>>>(L, pr.B, w.P, (int)pr.NBmax, (int)pr.NQTmax, w.status);
+  }
+  if (cudaMemsetAsync(w.counts, 0, sizeof(uint32_t) * (size_t)pr.Hkv * pr.NBmax, st) !=
+      cudaSuccess)
+    return fail(MOBA_ERR_CUDA);
+  for (int p = 0; p < npass; ++p) {
+    const int g0 = p * nu_max, ng = (pr.Hkv - g0) < nu_max ? (pr.Hkv - g0) : nu_max;
+    if (cudaStreamWaitEvent(st, in_ready(p), 0) != cudaSuccess) return fail(MOBA_ERR_CUDA);
+    if ((r = run_pool(pr, hb.k, w, st, g0, ng)) != MOBA_OK) return fail(r);
+    if ((r = launch_gate<D>(pr, hb.q, w, hb.sel, w.counts, st, g0, ng)) != MOBA_OK) return fail(r);
+    if ((r = forward_one_pass<D>(pr, c, w, hb.sel, hb.o, hb.lse, g0, ng, st)) != MOBA_OK)
+      return fail(r);
+    if (cudaEventRecord(done(p), st) != cudaSuccess ||
+        cudaStreamWaitEvent(d2h, done(p), 0) != cudaSuccess)
+      return fail(MOBA_ERR_CUDA);
+    const int64_t h0 = (int64_t)g0 * pr.G, nh = (int64_t)ng * pr.G;
+    if (copy_cols(o_h, hb.o, pr.T, (int64_t)pr.Hq * D, h0 * D, nh * D, 2,
+                  cudaMemcpyDeviceToHost, d2h) != cudaSuccess ||
+        copy_cols(lse_h, hb.lse, rows_b, (int64_t)pr.Hq * per_head_lse, h0 * per_head_lse,
+                  nh * per_head_lse, 4, cudaMemcpyDeviceToHost, d2h) != cudaSuccess ||
+        (sel_h && copy_cols(sel_h, hb.sel, rows_b, (int64_t)pr.Hq * per_head_sel,
+                            h0 * per_head_sel, nh * per_head_sel, 4, cudaMemcpyDeviceToHost,
+                            d2h) != cudaSuccess))
+      return fail(MOBA_ERR_CUDA);
+  }
+  // the caller's stream covers the output copies
+  if (cudaEventRecord(start, d2h) != cudaSuccess || cudaStreamWaitEvent(st, start, 0) != cudaSuccess)
+    return fail(MOBA_ERR_CUDA);
+  return fail(MOBA_OK);
 }
 
 moba_status forward_impl(const Problem& pr, const void* q, const void* k, const void* v, void* o,
@@ -1219,6 +1381,40 @@ moba_status moba_forward_minmax(const void* q, const void* k, const void* v, voi
   MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
   return forward_impl(pr, q, k, v, o, lse, sel_out, ws, ws_bytes,
                       reinterpret_cast<cudaStream_t>(stream), kRouteMinmaxGate);
+}
+
+// ---------------------------------------------------------------- host-buffer forward
+size_t moba_forward_host_buffer_size(const moba_params* p, int heads_per_pass) {
+  Problem pr;
+  if (make_problem(p, false, nullptr, 0, 0, true, &pr) != MOBA_OK) return 0;
+  int nu = (heads_per_pass <= 0 || heads_per_pass > pr.Hkv) ? pr.Hkv : heads_per_pass;
+  const size_t ws = carve(pr, nu, nullptr).bytes;
+  return align_up(ws) + carve_host(pr, nullptr, ws).staged;
+}
+
+moba_status moba_forward_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int32_t* sel_out, const moba_params* p, void* dev_buf,
+                              size_t dev_bytes, moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  if (!q || !k || !v || !o || !lse) return MOBA_ERR_INVALID_ARG;
+  if (!topk_supported(pr)) return MOBA_ERR_UNSUPPORTED;
+  if ((int64_t)pr.T * pr.G * (pr.topk > 1 ? pr.topk - 1 : 1) >= INT32_MAX)
+    return MOBA_ERR_UNSUPPORTED;
+  if (!dev_buf || (reinterpret_cast<uintptr_t>(dev_buf) % kAlign)) return MOBA_ERR_WORKSPACE;
+  const size_t staged = carve_host(pr, nullptr, 0).staged;
+  auto need = [&](int n) { return align_up(carve(pr, n, nullptr).bytes) + staged; };
+  if (dev_bytes < need(1)) return MOBA_ERR_WORKSPACE;
+  if (pr.T == 0) return MOBA_OK;
+  int nu = 1;
+  while (nu < pr.Hkv && need(nu + 1) <= dev_bytes &&
+         (int64_t)(nu + 1) * pr.T * pr.G * (pr.topk > 1 ? pr.topk - 1 : 1) < INT32_MAX)
+    ++nu;
+  const Ws w = carve(pr, nu, static_cast<char*>(dev_buf));
+  const HostBufs hb = carve_host(pr, static_cast<char*>(dev_buf), w.bytes);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return pr.D == 128 ? forward_host_passes<128>(pr, q, k, v, o, lse, sel_out, hb, w, nu, st)
+                     : forward_host_passes<64>(pr, q, k, v, o, lse, sel_out, hb, w, nu, st);
 }
 
 // ---------------------------------------------------------------- backward

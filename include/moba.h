@@ -130,6 +130,22 @@ moba_status moba_forward_varlen(const void *q, const void *k, const void *v,
                                 void *o, float *lse, int32_t *sel_out, const moba_params *p,
                                 void *ws, size_t ws_bytes, moba_stream_t stream);
 
+/* ------------------------------------------------- forward on host buffers
+ * moba_forward with q, k, v, o, lse and sel_out (nullable) in HOST memory
+ * (batch layout; page-locked memory lets the copies overlap the work).  The
+ * call copies each group of kv heads' q / k / v columns in while the previous
+ * group computes, and that group's o / lse / sel rows back while the next
+ * computes, on two internal copy streams ordered against `stream`.  dev_buf is
+ * device memory of moba_forward_host_buffer_size(p, heads_per_pass) bytes (or
+ * more: the largest group of kv heads that fits is used); its first 256 bytes
+ * are the status word of a workspace (zero them before first use;
+ * moba_last_device_status(dev_buf) reads them).  Results equal moba_forward's.
+ * Returns when the work is queued; synchronise `stream` before reading o. */
+size_t moba_forward_host_buffer_size(const moba_params *p, int heads_per_pass);
+moba_status moba_forward_host(const void *q, const void *k, const void *v, void *o, float *lse,
+                              int32_t *sel_out, const moba_params *p, void *dev_buf,
+                              size_t dev_bytes, moba_stream_t stream);
+
 /* ----------------------------------------------------------------- backward
  * Gradients of the forward's attention for an output gradient dO, over the
  * selection the forward used (batch layout).  No gradient passes through the

@@ -253,3 +253,25 @@ def test_workload_dense_sampled_rows(moba, name):
     rows = S.sample_rows(w, 256, seed=99)
     Og, Lg, _ = gather_rows_packed(o, lse, None, rows, w.Hq, False, N)
     print(name, compare_dense(orc, rows, Og, Lg, label=name))
+
+
+def test_forward_host_matches_forward(moba):
+    """The host-buffer call (copies inside, pipelined by kv-head group) gives
+    the device call's o, lse and selection bit for bit."""
+    b, N, Hq, Hkv, d, B, k = 2, 4096, 8, 2, 128, 256, 4
+    w = S.Workload("host", [N] * b, Hq, Hkv, d, B, k, seed=4242)
+    q, kk, v = S.make_qkv(w, "cuda")
+    q4, k4, v4 = (x.view(b, N, x.shape[1], d) for x in (q, kk, v))
+    sel = torch.empty(b, Hq, N, k, dtype=torch.int32, device="cuda")
+    o, lse = moba.forward(q4, k4, v4, B, k, sel_out=sel)
+    pin = lambda x: x.cpu().pin_memory()
+    qh, kh, vh = pin(q4), pin(k4), pin(v4)
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    sh = torch.empty(sel.shape, dtype=sel.dtype, pin_memory=True)
+    p = moba.make_params(b, N, Hq, Hkv, d, B, k)
+    buf = moba.alloc_workspace(moba.forward_host_buffer_size(p, 1))  # one kv head per pass
+    moba.forward_host(qh, kh, vh, B, k, oh, lh, dev_buf=buf, sel_out=sh)
+    torch.cuda.synchronize()
+    assert moba.last_device_status(buf) == 0
+    assert torch.equal(oh, o.cpu()) and torch.equal(lh, lse.cpu()) and torch.equal(sh, sel.cpu())
