@@ -206,16 +206,40 @@ __device__ __forceinline__ float tile_row_max(uint32_t tS, int r) {
   return fmaxf(fmax3f(mp[0], mp[1], mp[2]), fmax3f(fmax3f(mp[3], mp[4], mp[5]), mp[6], mp[7]));
 }
 
+// 2^x of score pair e of a 16-pair group: one pair in eight on the FMA
+// pipe, the rest on the special-function unit, whose throughput otherwise
+// bounds the softmax.  Deterministic, so a second evaluation of the same
+// pair reproduces the first bit for bit.
+__device__ __forceinline__ void pair_exp2(float& p0, float& p1, float s0, float s1,
+                                          float scale_log2, float m_use, int e) {
+  float x0, x1;
+  ffma2(x0, x1, s0, s1, scale_log2, scale_log2, -m_use, -m_use);
+  if ((e & 7) == 7) {
+    exp2_poly2(p0, p1, x0, x1);
+  } else {
+    p0 = ex2_approx(x0);
+    p1 = ex2_approx(x1);
+  }
+}
+
 // P = 2^(s * scale_log2 - m) for one score tile, written back as packed bf16
 // pairs into the tile's first 64 TMEM columns (chunk h2 of 64 scores becomes
 // 32 packed columns, which never overlap scores still to be read).  Returns
 // the row sum of the fp32 probabilities.  Scale-and-shift and the sums run
-// as packed pairs; one pair in eight takes 2^x from a polynomial on the FMA
-// pipe, the rest from the special-function unit, whose throughput otherwise
-// bounds this loop.
+// as packed pairs.
+//
+// lo_mode (warp-uniform, diagonal tiles only) serves the first tile of a
+// block, whose first rows have a handful of keys: there the 2^-9 relative
+// rounding of each bf16 weight does not average out.  Rows 0..63 (lo_mode 1)
+// also write the residual P - bf16(P), as bf16, into columns 64..95; their
+// keys 64..127 are all masked, so the scores held there are never needed.
+// Rows 64..127 (lo_mode 2) write zeros there once they have read those
+// scores.  A second set of PV MMAs over columns 64..95 then gives rows 0..63
+// about 16 bits of each weight.
 template <bool MASK>
 __device__ __forceinline__ float tile_exp_to_p(uint32_t tS, int r, float scale_log2,
-                                               float m_use, uint64_t* half_bar, int lane) {
+                                               float m_use, uint64_t* half_bar, int lane,
+                                               int lo_mode) {
   float sp[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) sp[e] = 0.f;
@@ -229,26 +253,35 @@ __device__ __forceinline__ float tile_exp_to_p(uint32_t tS, int r, float scale_l
 #pragma unroll
       for (int c = 0; c < 64; ++c)
         if (h2 * 64 + c > r) sv[c] = -INFINITY;
+      if (h2 == 1 && lo_mode == 2) {
+        uint32_t z[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) z[e] = 0u;
+        tmem_st16(tS + 64, z);
+        tmem_st16(tS + 80, z);
+      }
     }
 #pragma unroll
     for (int q2 = 0; q2 < 2; ++q2) {
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        float x0, x1;
-        ffma2(x0, x1, sv[q2 * 32 + 2 * e], sv[q2 * 32 + 2 * e + 1], scale_log2, scale_log2,
-              -m_use, -m_use);
         float p0, p1;
-        if ((e & 7) == 7) {  // one pair in eight on the FMA pipe
-          exp2_poly2(p0, p1, x0, x1);
-        } else {
-          p0 = ex2_approx(x0);
-          p1 = ex2_approx(x1);
-        }
+        pair_exp2(p0, p1, sv[q2 * 32 + 2 * e], sv[q2 * 32 + 2 * e + 1], scale_log2, m_use, e);
         fadd2(sp[2 * (e & 3)], sp[2 * (e & 3) + 1], p0, p1);
         pk[e] = pack_bf16x2(p0, p1);
       }
       tmem_st16(tS + h2 * 32 + q2 * 16, pk);
+      if (MASK && h2 == 0 && lo_mode == 1) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float p0, p1;
+          pair_exp2(p0, p1, sv[q2 * 32 + 2 * e], sv[q2 * 32 + 2 * e + 1], scale_log2, m_use, e);
+          const __nv_bfloat162 hi = __floats2bfloat162_rn(p0, p1);
+          pk[e] = pack_bf16x2(p0 - __low2float(hi), p1 - __high2float(hi));
+        }
+        tmem_st16(tS + 64 + q2 * 16, pk);
+      }
     }
     if (h2 == 0) {  // P of keys 0..63 is in TMEM: the first half of PV may start
       tc_wait_st();
@@ -463,6 +496,15 @@ __global__ void __launch_bounds__(352, 1)
       if (!wait(&p_full[x], (nsx - 1) & 1)) return false;  // all of P_X(j)
       tc_fence_after();
       issue_pv(x, vs, true, kTileN / 32, kTileN / 16);
+      if (MODE != kRouted && it.nkv_x[x] == 1) {
+        // residual weights of keys 0..63 in columns 64..95 (first tile of a block)
+        const uint32_t vbase = sKVa + vs * C::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTileN / 32; ++kk)
+          tc_mma_ts_warp(tmem + C::col_o(x), tmem + C::col_s(x) + 64 + kk * 8,
+                         sdesc_mnmajor_sw128(vbase + kk * 2048, C::kHalfBytes, 1024), C::kIdescPV,
+                         1u);
+      }
       if (j == it.nkv_x[x] - 1) {
         tc_commit_warp(&o_full[x]);
         if (x == 0) ++no0; else ++no1;
@@ -541,9 +583,11 @@ __global__ void __launch_bounds__(352, 1)
             tmem_st32(tO + c4 * 32, ov);
           }
         }
-        const float sum = diag_tile
-                              ? tile_exp_to_p<true>(tS, r, a.scale_log2, m_use, &p_half[x], lane)
-                              : tile_exp_to_p<false>(tS, r, a.scale_log2, m_use, &p_half[x], lane);
+        // first tile of a block: residual weights for rows 0..63 (see tile_exp_to_p)
+        const int lo_mode = (diag_tile && nkv == 1) ? ((warp & 3) < 2 ? 1 : 2) : 0;
+        const float sum =
+            diag_tile ? tile_exp_to_p<true>(tS, r, a.scale_log2, m_use, &p_half[x], lane, lo_mode)
+                      : tile_exp_to_p<false>(tS, r, a.scale_log2, m_use, &p_half[x], lane, 0);
         l_run = l_run * alpha + sum;
         m_run = m_use;
         tc_wait_st();

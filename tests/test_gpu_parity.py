@@ -142,6 +142,42 @@ def test_full_causal_varlen_small(moba):
     compare_dense(orc, rows, Og, Lg, label="dense varlen")
 
 
+def _half_ulp_bf16(x):
+    """Half the spacing of bf16 numbers (8 significant bits) around |x|."""
+    _, e = np.frexp(np.abs(x))
+    return np.ldexp(1.0, e - 9)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_first_rows_of_a_block_round_once(moba, d):
+    # Rows 0..63 of a block's first tile attend to 1..64 keys, too few for the
+    # bf16 rounding of their softmax weights to average out.  The attention
+    # gives them the residual weights as well, so their output is the exact
+    # value rounded once to bf16: within half a bf16 step, plus 1e-4 for the
+    # fp32 arithmetic.  Own block only (k = 1) and the dense kernel.
+    N, Hq, Hkv, B = 2048, 4, 2, 256
+    w = S.Workload("first_rows", [N], Hq, Hkv, d, B, 1, seed=707)
+    q, k, v = S.make_qkv(w, "cuda")
+    q4, k4, v4 = (x.view(1, N, x.shape[1], d) for x in (q, k, v))
+    o1, _ = moba.forward(q4, k4, v4, B, 1)
+    o2, _ = moba.full_causal(q4, k4, v4)
+    torch.cuda.synchronize()
+    orc = Oracle(bf16_bits(q), bf16_bits(k), bf16_bits(v), w.cu, Hq, Hkv, d, B, 1)
+    rows = np.array([t for t in range(N) if t % B < 64], dtype=np.int64)
+    _, _, own = local_block_info(w.cu, rows, B)
+    sel = np.ascontiguousarray(np.broadcast_to(own[:, None, None], (len(rows), Hq, 1)), np.int32)
+    ref, _, _ = orc.attend(rows, sel)
+    got = o1[0].float().cpu().numpy()[rows].astype(np.float64)
+    err = np.abs(got - ref)
+    assert np.all(err <= _half_ulp_bf16(ref) + 1e-4), err.max()
+    dense_rows = rows[rows < 64]
+    sel_all = np.zeros((len(dense_rows), Hq, 1), np.int32)  # block 0 holds every earlier key
+    ref_d, _, _ = orc.attend(dense_rows, sel_all)
+    got_d = o2[0].float().cpu().numpy()[dense_rows].astype(np.float64)
+    err_d = np.abs(got_d - ref_d)
+    assert np.all(err_d <= _half_ulp_bf16(ref_d) + 1e-4), err_d.max()
+
+
 def test_k_equal_n_matches_full_causal_kernel(moba):
     # the method with every block selected is full attention: both CUDA paths agree
     w = S.Workload("kn", [2048], 8, 2, 128, 256, 8, seed=404)
