@@ -452,7 +452,7 @@ __global__ void __launch_bounds__(128) bucket_scatter_kernel(
 }
 
 // ------------------------------------------------------------------ merge
-// The row's partials -- one per routed past block (bf16 O, log2-domain lse)
+// The row's partials -- one per routed past block (fp16 O, log2-domain lse)
 // and the own-block partial (fp32 O, log2 lse) -- are combined by the
 // online-softmax rule
 //   m = max lse_s, w_s = 2^(lse_s - m), O = sum w_s O_s / sum w_s,
@@ -462,13 +462,16 @@ __global__ void __launch_bounds__(128) bucket_scatter_kernel(
 // four slots are loaded before any is used.  Rows whose selection is the own
 // block alone were finished by the own-block kernel and are skipped.  The
 // own-block partial is combined first, then the routed slots in ascending
-// order.
+// order.  A routed partial beyond the fp16 range (a value of 65520 or more,
+// possible only where the block's |v| exceeds it) was stored as inf; the
+// merged row is then not finite and the status word records
+// MOBA_DEV_CAPACITY.
 template <int D>
 __global__ void __launch_bounds__(256) merge_kernel(
     const __half* __restrict__ part_O, const float* __restrict__ part_lse,
     const float* __restrict__ own_O, const float* __restrict__ own_lse, int topk, int B, int G,
     int Hq, int u0, int nu, SeqLayout L, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
-    RowLayout R) {
+    RowLayout R, uint32_t* __restrict__ status) {
   constexpr int LPR = D / 8;       // lanes per row
   constexpr int RPW = 32 / LPR;    // rows per warp
   const int lane = threadIdx.x & 31;
@@ -542,6 +545,10 @@ __global__ void __launch_bounds__(256) merge_kernel(
       acc[2 * e + 1] = fmaf(w, f.y, acc[2 * e + 1]);
     }
   }
+  bool finite = true;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) finite = finite && fabsf(acc[e]) <= 3.4028234663852886e38f;
+  if (!finite) atomicOr(status, MOBA_DEV_CAPACITY);
   const float inv = 1.f / den;
   uint4 out;
   out.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);

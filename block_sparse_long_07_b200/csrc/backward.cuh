@@ -23,8 +23,8 @@
 // operands (S, dP) and as MN-major B operands (dK, dV); K / V tiles likewise.
 // Gradients are summed in fp32 buffers with atomic adds (each key gets one
 // routed and one own contribution per kv head; each row one per chosen
-// block) and converted to bf16 at the end.  This first version runs each
-// tile's MMAs and elementwise work in turn (no cross-tile pipelining).
+// block) and converted to bf16 at the end.  Within a CTA, a tile's MMAs and
+// elementwise work run in turn; bw_q_kernel double-buffers its K / V tiles.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -393,18 +393,26 @@ __global__ void __launch_bounds__(128, 1)
 //           keys = all of the bucket's block
 //   own:    blockIdx.x = (unit head, query tile); keys = the tile's block up
 //           to and including the tile's own 128 keys (causal)
+// K / V tiles are double-buffered (the second pair of buffers sits where the
+// key-tile kernel keeps its P and dS tiles): tile kt + 1 is loaded once the
+// dQ MMA of tile kt - 1, the last reader of its buffer, has completed, so the
+// load overlaps tile kt's S / dP MMAs, elementwise pass and dQ MMA.  The dQ
+// MMA of a tile is not waited for: the tensor pipe runs the next tile's S MMA,
+// which overwrites the dS columns it reads, after it.
 template <int D, int MODE>
 __global__ void __launch_bounds__(128, 1)
     bw_q_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const BwArgs a) {
   using C = BwCfg<D>;
+  static_assert(C::kTile <= C::kPT, "the second K / V buffers must fit the P / dS tiles");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* kv_bar = bars + 0;
-  uint64_t* mma_bar = bars + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  uint64_t* kv_full = bars + 0;  // [2] K / V tile landed in buffer b
+  uint64_t* mma_bar = bars + 2;  // S / dP MMAs of a tile (and all earlier MMAs) done
+  uint64_t* dq_bar = bars + 3;   // dQ MMA of a tile done: its K / V buffer is free
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   const int warp = threadIdx.x >> 5, r = threadIdx.x;
   const int NB = a.P.totals[0];
@@ -449,8 +457,10 @@ __global__ void __launch_bounds__(128, 1)
   }
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_bar, 1);
+    mbar_init(&kv_full[0], 1);
+    mbar_init(&kv_full[1], 1);
     mbar_init(mma_bar, 1);
+    mbar_init(dq_bar, 1);
     *abort_flag = 0u;
     fence_barrier_init();
   }
@@ -463,11 +473,25 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  unsigned char* sK = smem + C::kOffK;
-  unsigned char* sV = smem + C::kOffV;
+  auto sKb = [&](int b) { return smem + (b ? C::kOffP : C::kOffK); };
+  auto sVb = [&](int b) { return smem + (b ? C::kOffDS : C::kOffV); };
   unsigned char* sQ = smem + C::kOffQ;
   unsigned char* sDO = smem + C::kOffDO;
   uint32_t* st = a.status;
+  uint32_t nload0 = 0, nload1 = 0, nuse0 = 0, nuse1 = 0;  // K / V loads per buffer (thread 0)
+
+  auto load_kv = [&](int kt) {  // thread 0
+    const int b = kt & 1;
+    const int64_t kb = kblock + (int64_t)kt * kTileN;
+    mbar_arrive_expect_tx(&kv_full[b], 2 * C::kTile);
+#pragma unroll
+    for (int hx = 0; hx < D / 64; ++hx) {
+      tma_load_3d(sKb(b) + hx * C::kHalf, &tm_k, &kv_full[b], hx * 64, g, (int)kb);
+      tma_load_3d(sVb(b) + hx * C::kHalf, &tm_v, &kv_full[b], hx * 64, g, (int)kb);
+    }
+    if (b) ++nload1; else ++nload0;
+  };
+  if (threadIdx.x == 0) load_kv(0);  // overlaps the row gather below
 
   float lse2 = __int_as_float(0x7f800000), Dr = 0.f;
   if (x.t >= 0) {
@@ -480,25 +504,19 @@ __global__ void __launch_bounds__(128, 1)
   fence_proxy_async_smem();
   __syncthreads();
 
-  const uint32_t sQa = smem_u32(sQ), sDOa = smem_u32(sDO), sKa = smem_u32(sK),
-                 sVa = smem_u32(sV);
+  const uint32_t sQa = smem_u32(sQ), sDOa = smem_u32(sDO);
   constexpr uint32_t idS = idesc_bf16_f32(kTileM, kTileN, false, false);
   constexpr uint32_t idQ = idesc_bf16_f32(kTileM, D, false, true);
   bool ok = true;
-  uint32_t nm = 0;
+  uint32_t nm = 0, ndq = 0;  // mma_bar and dq_bar phases
   for (int kt = 0; kt < nkt && ok; ++kt) {
+    const int b = kt & 1;
     const int64_t kbase = kblock + (int64_t)kt * kTileN;
     const int nkeys = min(kTileN, blen - kt * kTileN);
-    if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(kv_bar, 2 * C::kTile);
-#pragma unroll
-      for (int hx = 0; hx < D / 64; ++hx) {
-        tma_load_3d(sK + hx * C::kHalf, &tm_k, kv_bar, hx * 64, g, (int)kbase);
-        tma_load_3d(sV + hx * C::kHalf, &tm_v, kv_bar, hx * 64, g, (int)kbase);
-      }
-    }
-    ok = bw_wait(kv_bar, kt & 1, abort_flag, st);
+    const uint32_t sKa = smem_u32(sKb(b)), sVa = smem_u32(sVb(b));
+    ok = bw_wait(&kv_full[b], (uint32_t)(kt >> 1) & 1u, abort_flag, st);
     if (!ok) break;
+    if (b) ++nuse1; else ++nuse0;
     if (warp == 0) {
       tc_fence_after();
 #pragma unroll
@@ -511,6 +529,12 @@ __global__ void __launch_bounds__(128, 1)
       }
       tc_commit_warp(mma_bar);
     }
+    if (threadIdx.x == 0 && kt + 1 < nkt) {
+      // buffer (kt + 1) & 1 was last read by the dQ MMA of tile kt - 1
+      const bool free_ok = kt == 0 || mbar_wait(dq_bar, (uint32_t)(kt - 1) & 1u, abort_flag, st);
+      if (free_ok) load_kv(kt + 1);
+    }
+    __syncwarp();  // warp 0 reconverges before the block-wide wait
     ok = bw_wait(mma_bar, nm & 1, abort_flag, st);
     ++nm;
     if (!ok) break;
@@ -527,9 +551,12 @@ __global__ void __launch_bounds__(128, 1)
         tc_mma_ts_warp(tmem + C::kColA, tmem + C::kColS + kk * 8,
                        sdesc_mnmajor_sw128(sKa + kk * 2048, C::kHalf, 1024), idQ,
                        (kt > 0 || kk > 0) ? 1u : 0u);
-      tc_commit_warp(mma_bar);
+      tc_commit_warp(dq_bar);
     }
-    // the next K / V load and S MMA overwrite what this MMA reads
+    ++ndq;
+  }
+  if (ok) {  // every dQ MMA done
+    if (warp == 0) tc_commit_warp(mma_bar);
     ok = bw_wait(mma_bar, nm & 1, abort_flag, st);
     ++nm;
   }
@@ -547,7 +574,25 @@ __global__ void __launch_bounds__(128, 1)
       }
     }
   }
-  bw_teardown(kv_bar, mma_bar, ok, nm, tmem, C::kTmemCols, warp);
+  // teardown: after an abort, loads and MMAs may still be in flight
+  if (!ok && threadIdx.x == 0) {
+    if (nload0 > nuse0) mbar_wait_teardown(&kv_full[0], (nload0 - 1u) & 1u, 200000000ull);
+    if (nload1 > nuse1) mbar_wait_teardown(&kv_full[1], (nload1 - 1u) & 1u, 200000000ull);
+  }
+  if (warp == 0) {
+    tc_commit_warp(mma_bar);  // arrives once every MMA of this CTA has completed
+    if (threadIdx.x == 0) {
+      mbar_wait_teardown(mma_bar, nm & 1, 500000000ull);
+      if (ndq > 0) mbar_wait_teardown(dq_bar, (ndq - 1u) & 1u, 500000000ull);
+    }
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
 }
 
 // fp32 accumulators -> bf16 gradients.

@@ -608,7 +608,8 @@ moba_status forward_one_pass(const Problem& pr, FwdCtx& c, const Ws& w, const in
     Timed tm(kKMerge, st);
     merge_kernel<D><<<blocks, 256, 0, st>>>(w.part_O, w.part_lse, w.own_O, w.own_lse, pr.topk,
                                             pr.B, pr.G, pr.Hq, u0, nu, L,
-                                            reinterpret_cast<__nv_bfloat16*>(o), lse, pr.R);
+                                            reinterpret_cast<__nv_bfloat16*>(o), lse, pr.R,
+                                            w.status);
     MOBA_CUDA(cudaGetLastError());
   }
   return MOBA_OK;

@@ -79,7 +79,14 @@ PREFILL_10M_SHARD = Workload("prefill_10m_shard", [10485760], 4, 1, 128, 40960, 
                              note="one kv-head group (4 q / 1 kv head) of the 32 q / 8 kv "
                                   "model at N=10485760, B=40960 (256 blocks), k=12")
 
-WORKLOADS = {w.name: w for w in (TINY, FINE_32K, LONG_128K, MILLION, VARLEN, PREFILL_10M_SHARD)}
+# long_128k's shape with a quarter of the heads (same N, B, k and per-head
+# bucket sizes): a case small enough on the device for multi-pass kernel
+# captures, with q (268 MB) still larger than L2.
+LONG_128K_H8 = Workload("long_128k_h8", [131072], 8, 2, 128, 4096, 12, seed=2,
+                        note="8 q / 2 kv heads, d=128, N=131072, B=4096 (32 blocks), k=12")
+
+WORKLOADS = {w.name: w for w in (TINY, FINE_32K, LONG_128K, MILLION, VARLEN, PREFILL_10M_SHARD,
+                                 LONG_128K_H8)}
 
 
 def block_ids(lengths: List[int], B: int) -> np.ndarray:

@@ -85,6 +85,9 @@ SMALL = [
     ([1280, 1280], 4, 2, 128, 256, 3),  # batch of 2
     ([129], 2, 1, 128, 128, 2),       # one row past the first block
     ([4096], 8, 2, 128, 128, 5),      # many blocks, top-k ranking
+    ([32896], 2, 1, 128, 128, 6),     # 257 blocks: 256 past, the tensor-core gate's limit
+    ([40000], 2, 1, 64, 128, 8),      # 313 blocks: beyond it, the SIMT gate
+    ([4096], 4, 1, 128, 128, 17),     # k - 1 = 16, the longest list the tensor-core gate ranks
 ]
 
 
@@ -176,6 +179,27 @@ def test_first_rows_of_a_block_round_once(moba, d):
     got_d = o2[0].float().cpu().numpy()[dense_rows].astype(np.float64)
     err_d = np.abs(got_d - ref_d)
     assert np.all(err_d <= _half_ulp_bf16(ref_d) + 1e-4), err_d.max()
+
+
+def test_routed_partial_beyond_fp16_range_is_reported(moba):
+    # Routed partials are stored in fp16.  Every row of block 1 routes to
+    # block 0, its only past block.  With block 0's V at 65280 (the largest
+    # bf16 value below the fp16 maximum) nothing is reported; at 65536 the
+    # partial rounds to inf in fp16 and the forward reports a device check.
+    N, Hq, Hkv, d, B, k = 1024, 2, 1, 128, 256, 3
+    w = S.Workload("fp16_range", [N], Hq, Hkv, d, B, k, seed=111)
+    q, kk, v = S.make_qkv(w, "cuda")
+    q4, k4 = (x.view(1, N, x.shape[1], d) for x in (q, kk))
+    p = moba.make_params(1, N, Hq, Hkv, d, B, k)
+    for val, want in ((65280.0, 0), (65536.0, 6)):  # 6 = MOBA_ERR_DEVICE_CHECK
+        v2 = v.clone()
+        v2[:B] = val
+        ws = moba.alloc_workspace(moba.workspace_size(p, 1))
+        o, _ = moba.forward(q4, k4, v2.view(1, N, Hkv, d), B, k, ws=ws)
+        torch.cuda.synchronize()
+        assert moba.last_device_status(ws) == want, val
+        if want == 0:
+            assert torch.isfinite(o.float()).all()
 
 
 def test_k_equal_n_matches_full_causal_kernel(moba):
