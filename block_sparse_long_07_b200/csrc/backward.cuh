@@ -12,19 +12,21 @@
 // meet J's keys; for the own part, each block's rows meet the same block's
 // keys, causally.  Two kernels per part, each recomputing S and P:
 //   bw_kv_kernel  one CTA per (bucket or own block, 128-key tile): loops over
-//                 the rows in tiles of 128; S = Q K^T and dP = dO V^T into
-//                 TMEM, P and dS into shared memory as [rows][keys] tiles,
-//                 which are the transposed (MN-major) A operands of
-//                 dV += P^T dO and dK += dS^T Q, accumulated in TMEM
+//                 the rows in tiles of 128; S^T = K Q^T and dP^T = V dO^T
+//                 (keys on the TMEM lanes), P^T and dS^T packed as bf16 over
+//                 them, which are the TMEM A operands of dV += P^T dO and
+//                 dK += dS^T Q, accumulated in TMEM
 //   bw_q_kernel   one CTA per tile of 128 rows (gathered or own): loops over
 //                 the block's key tiles; dS packed as bf16 into TMEM is the A
 //                 operand of dQ += dS K
-// The Q / dO tiles ([rows][d], 128-byte swizzled) serve both as K-major A
-// operands (S, dP) and as MN-major B operands (dK, dV); K / V tiles likewise.
+// The Q / dO tiles ([rows][d], 128-byte swizzled) serve both as K-major
+// operands (S, dP and their transposes) and as MN-major B operands (dK, dV);
+// K / V tiles likewise.
 // Gradients are summed in fp32 buffers with atomic adds (each key gets one
 // routed and one own contribution per kv head; each row one per chosen
 // block) and converted to bf16 at the end.  Within a CTA, a tile's MMAs and
-// elementwise work run in turn; bw_q_kernel double-buffers its K / V tiles.
+// elementwise work run in turn; the next tile's operands (bw_kv: gathered
+// Q / dO rows, bw_q: K / V) load into a second buffer meanwhile.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -58,14 +60,16 @@ template <int D>
 struct BwCfg {
   static constexpr int kHalf = kTileM * 128;   // 128 rows x 64 columns bf16
   static constexpr int kTile = kTileM * D * 2; // one [128][D] bf16 tile
-  static constexpr int kPT = kTileM * kTileN * 2;  // one [128 rows][128 keys] bf16 tile
+  // Six tile slots.  bw_kv: K, V, then two (Q, dO) buffers.  bw_q: K, V,
+  // Q, dO, then a second (K, V) buffer.
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kTile;
   static constexpr int kOffQ = kOffV + kTile;
   static constexpr int kOffDO = kOffQ + kTile;
-  static constexpr int kOffP = kOffDO + kTile;
-  static constexpr int kOffDS = kOffP + kPT;
-  static constexpr int kOffBar = kOffDS + kPT;
+  static constexpr int kOffX = kOffDO + kTile;   // slot 4
+  static constexpr int kOffY = kOffX + kTile;    // slot 5
+  static constexpr int kOffDL = kOffY + kTile;   // bw_kv: float2 (D, lse2) [2][128 rows]
+  static constexpr int kOffBar = kOffDL + 2 * kTileM * 8;
   static constexpr int kSmemBytes = kOffBar + 64 + 1024;
   static constexpr uint32_t kTmemCols = 512;
   // TMEM columns
@@ -142,27 +146,24 @@ __device__ __forceinline__ void bw_load_row(const BwArgs& a, BwRow x, int r, uns
   }
 }
 
-// P and dS of row r for key tile [kbase, kbase + 128): reads S and dP from
-// TMEM (this thread's lane), masks keys >= nkeys and, when causal, keys
-// after the row's token.  Writes P and dS as bf16 [rows][keys] tiles
-// (128-byte swizzled halves of 64 keys) when to_smem, or dS packed into
-// TMEM columns [kColS, kColS + 64) otherwise.
-template <int D, bool TO_SMEM>
-__device__ __forceinline__ void bw_p_ds(const BwArgs& a, uint32_t tS, uint32_t tDP, int r,
-                                        float lse2, float Dr, int nkeys, bool causal,
-                                        int64_t trow, int64_t kbase, unsigned char* sP,
-                                        unsigned char* sDS) {
-  using C = BwCfg<D>;
+// dS of row r for key tile [kbase, kbase + 128) (dQ kernel, rows on TMEM
+// lanes): reads S and dP from TMEM (this thread's lane), masks keys >= nkeys
+// and, when causal, keys after the row's token, and packs dS as bf16 pairs
+// into TMEM columns [kColS, kColS + 64).
+template <int D>
+__device__ __forceinline__ void bw_p_ds(const BwArgs& a, uint32_t tS, uint32_t tDP, float lse2,
+                                        float Dr, int nkeys, bool causal, int64_t trow,
+                                        int64_t kbase) {
 #pragma unroll 1
   for (int c0 = 0; c0 < kTileN; c0 += 32) {
     uint32_t sv[32], dv[32];
     tmem_ld32(tS + c0, sv);
     tmem_ld32(tDP + c0, dv);
     tc_wait_ld();
-    uint32_t pp[16], dd[16];
+    uint32_t dd[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-      float p2[2], d2[2];
+      float d2[2];
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
         const int j = c0 + 2 * e + x;
@@ -170,50 +171,52 @@ __device__ __forceinline__ void bw_p_ds(const BwArgs& a, uint32_t tS, uint32_t t
         if (causal) keep = keep && (kbase + j <= trow);
         const float p =
             keep ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + x]), a.scale_log2, -lse2)) : 0.f;
-        p2[x] = p;
         d2[x] = p * (__uint_as_float(dv[2 * e + x]) - Dr);
+      }
+      dd[e] = pack_bf16x2(d2[0], d2[1]);
+    }
+    tmem_st16(tS + (c0 >> 1), dd);
+  }
+}
+
+// P^T and dS^T of key lane r for one 128-row tile (dK / dV kernel, keys on
+// TMEM lanes): reads S^T and dP^T over the tile's row columns, with each
+// row's (D, lse2) from shared memory (a row past the tile's end has lse2 =
+// +inf, so its P is 0).  Masks the lane when its key is past the block end
+// (key_ok false) and, when causal, rows before the key's token.  Packs P^T as
+// bf16 pairs into [kColS, kColS + 64) and dS^T into [kColDP, kColDP + 64):
+// chunk c0 of 32 columns becomes 16 packed columns at c0 / 2, which this
+// thread has already read.
+__device__ __forceinline__ void bw_pt_dst(const BwArgs& a, uint32_t tS, uint32_t tDP,
+                                          const float2* __restrict__ dl, bool key_ok,
+                                          bool causal, int64_t key_tok, int64_t row_tok0) {
+#pragma unroll 1
+  for (int c0 = 0; c0 < kTileM; c0 += 32) {
+    uint32_t sv[32], dv[32];
+    tmem_ld32(tS + c0, sv);
+    tmem_ld32(tDP + c0, dv);
+    tc_wait_ld();
+    uint32_t pp[16], dd[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float4 l = *reinterpret_cast<const float4*>(dl + c0 + 2 * e);  // D, lse2 of 2 rows
+      float p2[2], d2[2];
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const int c = c0 + 2 * e + x;
+        bool keep = key_ok;
+        if (causal) keep = keep && (key_tok <= row_tok0 + c);
+        const float Dc = x ? l.z : l.x, lc = x ? l.w : l.y;
+        const float p =
+            keep ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + x]), a.scale_log2, -lc)) : 0.f;
+        p2[x] = p;
+        d2[x] = p * (__uint_as_float(dv[2 * e + x]) - Dc);
       }
       pp[e] = pack_bf16x2(p2[0], p2[1]);
       dd[e] = pack_bf16x2(d2[0], d2[1]);
     }
-    if (TO_SMEM) {
-      // keys c0..c0+31 = 64 bytes = 4 16-byte units of half c0 / 64
-      const uint32_t hoff = (uint32_t)(c0 >> 6) * C::kHalf;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t off = hoff + sw128_offset(r, ((c0 & 63) >> 3) + u);
-        *reinterpret_cast<uint4*>(sP + off) =
-            make_uint4(pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
-        *reinterpret_cast<uint4*>(sDS + off) =
-            make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
-      }
-    } else {
-      tmem_st16(tS + (c0 >> 1), dd);
-    }
-  }
-}
-
-// End of a backward CTA.  After an abort, copies or MMAs may still be in
-// flight: wait for them (bounded, nothing raised) before TMEM is freed and
-// the CTA's shared memory released.
-__device__ __forceinline__ void bw_teardown(uint64_t* kv_bar, uint64_t* mma_bar, bool ok,
-                                            uint32_t nm, uint32_t tmem, uint32_t cols,
-                                            int warp) {
-  if (!ok && threadIdx.x == 0) {
-    mbar_wait_teardown(kv_bar, 0, 200000000ull);
-    mbar_wait_teardown(kv_bar, 1, 200000000ull);
-  }
-  if (warp == 0) {
-    // every MMA this CTA issued has completed once this commit arrives
-    tc_commit_warp(mma_bar);
-    if (threadIdx.x == 0) mbar_wait_teardown(mma_bar, nm & 1, 500000000ull);
-    __syncwarp();
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, cols);
+    tmem_st16(tS + (c0 >> 1), pp);
+    tmem_st16(tDP + (c0 >> 1), dd);
   }
 }
 
@@ -223,11 +226,20 @@ __device__ __forceinline__ bool bw_wait(uint64_t* bar, uint32_t parity,
   return __syncthreads_and(mbar_wait(bar, parity, abort_flag, st) ? 1 : 0) != 0;
 }
 
-// dK / dV of one 128-key tile.
+// dK / dV of one 128-key tile, with the keys on the TMEM lanes.
 //   routed: blockIdx.x = f * KT + kt over the pass's buckets f = u * NB + J;
 //           rows = the bucket's entries
 //   own:    blockIdx.x = f * KT + kt over (unit, block); rows = the block's
 //           tokens at or after the key tile, for every q head of the unit
+// Per 128-row tile n: S^T = K Q^T and dP^T = V dO^T (M = keys, N = rows) go
+// to TMEM; the four warps (thread = key) form P^T and dS^T = P^T (dP^T - D)
+// and pack them as bf16 over the columns they came from; dV += P^T dO and
+// dK += dS^T Q take them as TMEM A operands (K = rows), with dO and Q as
+// MN-major B operands.  The rows are gathered into two (Q, dO) buffers: tile
+// n + 1 is gathered while tile n computes, once the dV / dK MMAs of tile
+// n - 1, the last readers of its buffer, are done.  The tensor pipe runs the
+// S^T MMA of tile n + 1 after the dV / dK MMAs of tile n that read the
+// columns it overwrites.
 template <int D, int MODE>
 __global__ void __launch_bounds__(128, 1)
     bw_kv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -237,11 +249,12 @@ __global__ void __launch_bounds__(128, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* kv_bar = bars + 0;
-  uint64_t* mma_bar = bars + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  uint64_t* kv_bar = bars + 0;   // K / V tile landed
+  uint64_t* s_bar = bars + 1;    // S^T / dP^T MMAs of a row tile done
+  uint64_t* mma_bar = bars + 2;  // dV / dK MMAs of a row tile (and every earlier MMA) done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = threadIdx.x;
+  const int warp = threadIdx.x >> 5, r = threadIdx.x;
 
   const int NB = a.P.totals[0];
   const int KT = a.B / kTileN;
@@ -269,6 +282,7 @@ __global__ void __launch_bounds__(128, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_bar, 1);
+    mbar_init(s_bar, 1);
     mbar_init(mma_bar, 1);
     *abort_flag = 0u;
     fence_barrier_init();
@@ -284,13 +298,37 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
   unsigned char* sK = smem + C::kOffK;
   unsigned char* sV = smem + C::kOffV;
-  unsigned char* sQ = smem + C::kOffQ;
-  unsigned char* sDO = smem + C::kOffDO;
-  unsigned char* sP = smem + C::kOffP;
-  unsigned char* sDS = smem + C::kOffDS;
+  auto sQb = [&](int b) { return smem + (b ? C::kOffX : C::kOffQ); };
+  auto sDOb = [&](int b) { return smem + (b ? C::kOffY : C::kOffDO); };
+  float2* sdl = reinterpret_cast<float2*>(smem + C::kOffDL);  // [2][128] (D, lse2)
   uint32_t* st = a.status;
-  bool ok = true;
-  uint32_t nm = 0;  // mma_bar phases
+
+  // row r of row tile n: routed -> the bucket's entry; own -> a token of the
+  // block at or after the key tile, for q head n / own_tiles
+  auto row_of = [&](int n) -> BwRow {
+    BwRow x{-1, 0};
+    if (MODE == kBwRouted) {
+      x = bw_row_routed(a, g, e0 + (int64_t)n * kTileM, e1, r);
+    } else {
+      const int hh = n / own_tiles, qt = n % own_tiles;
+      const int64_t t = kstart + (int64_t)qt * kTileM + r;
+      if (t < (int64_t)a.P.blk_tok[J] + blen) {
+        x.t = t;
+        x.h = g * a.G + hh;
+      }
+    }
+    return x;
+  };
+  // gather row tile n into buffer n & 1: q / dO rows by cp.async (one group),
+  // (D, lse2) by a plain load; a missing row gets lse2 = +inf (P = 0)
+  auto gather = [&](int n) {
+    const BwRow x = row_of(n);
+    float2 dlv = make_float2(0.f, __int_as_float(0x7f800000));
+    if (x.t >= 0) dlv = a.dl[(size_t)x.t * a.Hq + x.h];
+    sdl[(n & 1) * kTileM + r] = dlv;
+    bw_load_row<D>(a, x, r, sQb(n & 1), sDOb(n & 1));
+    cp_async_commit();
+  };
 
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx(kv_bar, 2 * C::kTile);
@@ -300,32 +338,19 @@ __global__ void __launch_bounds__(128, 1)
       tma_load_3d(sV + hx * C::kHalf, &tm_v, kv_bar, hx * 64, g, (int)kstart);
     }
   }
-  ok = bw_wait(kv_bar, 0, abort_flag, st);
+  gather(0);
+  bool ok = bw_wait(kv_bar, 0, abort_flag, st);
 
-  const uint32_t sQa = smem_u32(sQ), sDOa = smem_u32(sDO), sKa = smem_u32(sK),
-                 sVa = smem_u32(sV), sPa = smem_u32(sP), sDSa = smem_u32(sDS);
-  constexpr uint32_t idS = idesc_bf16_f32(kTileM, kTileN, false, false);
-  constexpr uint32_t idG = idesc_bf16_f32(kTileN, D, true, true);
-  for (int tile = 0; tile < ntiles && ok; ++tile) {
-    BwRow x{-1, 0};
-    if (MODE == kBwRouted) {
-      x = bw_row_routed(a, g, e0 + (int64_t)tile * kTileM, e1, r);
-    } else {
-      const int hh = tile / own_tiles, qt = tile % own_tiles;
-      const int64_t t = kstart + (int64_t)qt * kTileM + r;
-      if (t < (int64_t)a.P.blk_tok[J] + blen) {
-        x.t = t;
-        x.h = g * a.G + hh;
-      }
-    }
-    float lse2 = __int_as_float(0x7f800000), Dr = 0.f;
-    if (x.t >= 0) {
-      const float2 v = a.dl[(size_t)x.t * a.Hq + x.h];
-      Dr = v.x;
-      lse2 = v.y;
-    }
-    bw_load_row<D>(a, x, r, sQ, sDO);
-    cp_async_wait_all();
+  const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
+  constexpr uint32_t idS = idesc_bf16_f32(kTileN, kTileM, false, false);  // M = keys, N = rows
+  constexpr uint32_t idG = idesc_bf16_f32(kTileN, D, false, true);        // A in TMEM, B MN-major
+  const bool key_ok = r < nkeys;
+  const int64_t key_tok = kstart + r;
+  uint32_t ns = 0, nm = 0;  // s_bar and mma_bar phases
+  for (int n = 0; n < ntiles && ok; ++n) {
+    const int b = n & 1;
+    const uint32_t sQa = smem_u32(sQb(b)), sDOa = smem_u32(sDOb(b));
+    cp_async_wait_group<0>();  // this thread's rows of tile n (the only group pending)
     fence_proxy_async_smem();
     __syncthreads();
     if (warp == 0) {
@@ -333,34 +358,48 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * C::kHalf + (kk & 3) * 32;
-        tc_mma_ss_warp(tmem + C::kColS, sdesc_kmajor_sw128(sQa + off),
-                       sdesc_kmajor_sw128(sKa + off), idS, kk > 0 ? 1u : 0u);
-        tc_mma_ss_warp(tmem + C::kColDP, sdesc_kmajor_sw128(sDOa + off),
-                       sdesc_kmajor_sw128(sVa + off), idS, kk > 0 ? 1u : 0u);
+        tc_mma_ss_warp(tmem + C::kColS, sdesc_kmajor_sw128(sKa + off),
+                       sdesc_kmajor_sw128(sQa + off), idS, kk > 0 ? 1u : 0u);
+        tc_mma_ss_warp(tmem + C::kColDP, sdesc_kmajor_sw128(sVa + off),
+                       sdesc_kmajor_sw128(sDOa + off), idS, kk > 0 ? 1u : 0u);
       }
-      tc_commit_warp(mma_bar);
+      tc_commit_warp(s_bar);
     }
-    ok = bw_wait(mma_bar, nm & 1, abort_flag, st);
-    ++nm;
+    ++ns;
+    if (n + 1 < ntiles) {
+      // buffer (n + 1) & 1 was last read by the dV / dK MMAs of tile n - 1
+      if (n > 0) {
+        ok = bw_wait(mma_bar, (nm - 1) & 1, abort_flag, st);
+        if (!ok) break;
+      }
+      gather(n + 1);
+    }
+    ok = bw_wait(s_bar, (ns - 1) & 1, abort_flag, st);
     if (!ok) break;
     tc_fence_after();
-    bw_p_ds<D, true>(a, tmem + lane_off + C::kColS, tmem + lane_off + C::kColDP, r, lse2, Dr,
-                     nkeys, MODE == kBwOwn, x.t, kstart, sP, sDS);
-    fence_proxy_async_smem();
+    int64_t row_tok0 = 0;
+    if (MODE == kBwOwn) row_tok0 = kstart + (int64_t)(n % own_tiles) * kTileM;
+    bw_pt_dst(a, tmem + lane_off + C::kColS, tmem + lane_off + C::kColDP, sdl + b * kTileM,
+              key_ok, MODE == kBwOwn, key_tok, row_tok0);
+    tc_wait_st();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < kTileM / 16; ++kk) {  // K = rows, 16 per step
-        const uint32_t acc = (tile > 0 || kk > 0) ? 1u : 0u;
-        tc_mma_ss_warp(tmem + C::kColA, sdesc_mnmajor_sw128(sPa + kk * 2048, C::kHalf, 1024),
+        const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
+        tc_mma_ts_warp(tmem + C::kColA, tmem + C::kColS + kk * 8,
                        sdesc_mnmajor_sw128(sDOa + kk * 2048, C::kHalf, 1024), idG, acc);
-        tc_mma_ss_warp(tmem + C::kColB, sdesc_mnmajor_sw128(sDSa + kk * 2048, C::kHalf, 1024),
+        tc_mma_ts_warp(tmem + C::kColB, tmem + C::kColDP + kk * 8,
                        sdesc_mnmajor_sw128(sQa + kk * 2048, C::kHalf, 1024), idG, acc);
       }
       tc_commit_warp(mma_bar);
     }
+    ++nm;
+  }
+  if (ok) {  // every dV / dK MMA done
+    if (warp == 0) tc_commit_warp(mma_bar);
     ok = bw_wait(mma_bar, nm & 1, abort_flag, st);
     ++nm;
   }
@@ -376,7 +415,7 @@ __global__ void __launch_bounds__(128, 1)
       tmem_ld32(tmem + lane_off + C::kColA + c0, va);
       tmem_ld32(tmem + lane_off + C::kColB + c0, vb);
       tc_wait_ld();
-      if (r < nkeys) {
+      if (key_ok) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           atomicAdd(dv + c0 + e, __uint_as_float(va[e]));
@@ -385,7 +424,24 @@ __global__ void __launch_bounds__(128, 1)
       }
     }
   }
-  bw_teardown(kv_bar, mma_bar, ok, nm, tmem, C::kTmemCols, warp);
+  // teardown: after an abort, row gathers, the K / V load and MMAs may still
+  // be in flight; wait for them (bounded) before TMEM and shared memory go
+  cp_async_wait_all();
+  if (!ok && threadIdx.x == 0) mbar_wait_teardown(kv_bar, 0, 200000000ull);
+  if (warp == 0) {
+    tc_commit_warp(mma_bar);  // arrives once every MMA of this CTA has completed
+    if (threadIdx.x == 0) {
+      mbar_wait_teardown(mma_bar, nm & 1, 500000000ull);
+      if (ns > 0) mbar_wait_teardown(s_bar, (ns - 1) & 1, 500000000ull);
+    }
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
 }
 
 // dQ of one 128-row tile.
@@ -393,8 +449,8 @@ __global__ void __launch_bounds__(128, 1)
 //           keys = all of the bucket's block
 //   own:    blockIdx.x = (unit head, query tile); keys = the tile's block up
 //           to and including the tile's own 128 keys (causal)
-// K / V tiles are double-buffered (the second pair of buffers sits where the
-// key-tile kernel keeps its P and dS tiles): tile kt + 1 is loaded once the
+// K / V tiles are double-buffered (the second pair in slots 4 and 5): tile
+// kt + 1 is loaded once the
 // dQ MMA of tile kt - 1, the last reader of its buffer, has completed, so the
 // load overlaps tile kt's S / dP MMAs, elementwise pass and dQ MMA.  The dQ
 // MMA of a tile is not waited for: the tensor pipe runs the next tile's S MMA,
@@ -404,7 +460,6 @@ __global__ void __launch_bounds__(128, 1)
     bw_q_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const BwArgs a) {
   using C = BwCfg<D>;
-  static_assert(C::kTile <= C::kPT, "the second K / V buffers must fit the P / dS tiles");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -473,8 +528,8 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  auto sKb = [&](int b) { return smem + (b ? C::kOffP : C::kOffK); };
-  auto sVb = [&](int b) { return smem + (b ? C::kOffDS : C::kOffV); };
+  auto sKb = [&](int b) { return smem + (b ? C::kOffX : C::kOffK); };
+  auto sVb = [&](int b) { return smem + (b ? C::kOffY : C::kOffV); };
   unsigned char* sQ = smem + C::kOffQ;
   unsigned char* sDO = smem + C::kOffDO;
   uint32_t* st = a.status;
@@ -539,8 +594,8 @@ __global__ void __launch_bounds__(128, 1)
     ++nm;
     if (!ok) break;
     tc_fence_after();
-    bw_p_ds<D, false>(a, tmem + lane_off + C::kColS, tmem + lane_off + C::kColDP, r, lse2, Dr,
-                      nkeys, MODE == kBwOwn, x.t, kbase, nullptr, nullptr);
+    bw_p_ds<D>(a, tmem + lane_off + C::kColS, tmem + lane_off + C::kColDP, lse2, Dr, nkeys,
+               MODE == kBwOwn, x.t, kbase);
     tc_wait_st();
     tc_fence_before();
     __syncthreads();
