@@ -128,34 +128,46 @@ __device__ __forceinline__ BwRow bw_row_routed(const BwArgs& a, int g, int64_t e
   return x;
 }
 
-// Copy row r's q and dO (128-byte swizzled halves of 64 columns) into the
-// tiles; a row with t < 0 copies token 0's data (finite; its P and dS are
-// forced to zero).
+// Copy half hg (columns hg * D / 2 .. + D / 2) of row r's q and dO into the
+// tiles (128-byte swizzled halves of 64 columns); two threads share a row.
+// A row with t < 0 copies token 0's data (finite; its P and dS are forced to
+// zero).
 template <int D>
-__device__ __forceinline__ void bw_load_row(const BwArgs& a, BwRow x, int r, unsigned char* sQ,
-                                            unsigned char* sDO) {
+__device__ __forceinline__ void bw_load_row(const BwArgs& a, BwRow x, int r, int hg,
+                                            unsigned char* sQ, unsigned char* sDO) {
   using C = BwCfg<D>;
   const int64_t t = x.t < 0 ? 0 : x.t;
   const __nv_bfloat16* qs = a.q + ((size_t)t * a.Hq + x.h) * D;
   const __nv_bfloat16* gs = a.dO + ((size_t)t * a.Hq + x.h) * D;
 #pragma unroll
-  for (int c = 0; c < D / 8; ++c) {
+  for (int c = hg * (D / 16); c < (hg + 1) * (D / 16); ++c) {
     const uint32_t off = (uint32_t)(c >> 3) * C::kHalf + sw128_offset(r, c & 7);
     cp_async_16(sQ + off, qs + c * 8);
     cp_async_16(sDO + off, gs + c * 8);
   }
 }
 
-// dS of row r for key tile [kbase, kbase + 128) (dQ kernel, rows on TMEM
-// lanes): reads S and dP from TMEM (this thread's lane), masks keys >= nkeys
-// and, when causal, keys after the row's token, and packs dS as bf16 pairs
-// into TMEM columns [kColS, kColS + 64).
+// Eight warps share the elementwise work of a 128 x 128 score tile: warp w
+// takes TMEM lanes 32 * (w % 4) .. + 31 and columns 64 * (w / 4) .. + 63.
+// Its 32-column chunks are packed as bf16 pairs over columns it has already
+// read: column c of the tile lands in packed column c / 2 (c < 64) or
+// 64 + c / 2 (c >= 64; that half walks its chunks from the top down).  The
+// MMA over tile columns 16 kk .. 16 kk + 15 reads its A operand there.
+__host__ __device__ constexpr uint32_t bw_packed_col(int kk) {
+  return kk < 4 ? 8u * kk : 64u + 8u * kk;
+}
+
+// dS of a row for its half hc of key tile [kbase, kbase + 128) (dQ kernel,
+// rows on TMEM lanes): reads S and dP from TMEM (this thread's lane), masks
+// keys >= nkeys and, when causal, keys after the row's token, and packs dS
+// as bf16 pairs (see bw_packed_col) from TMEM column kColS.
 template <int D>
 __device__ __forceinline__ void bw_p_ds(const BwArgs& a, uint32_t tS, uint32_t tDP, float lse2,
                                         float Dr, int nkeys, bool causal, int64_t trow,
-                                        int64_t kbase) {
+                                        int64_t kbase, int hc) {
 #pragma unroll 1
-  for (int c0 = 0; c0 < kTileN; c0 += 32) {
+  for (int i = 0; i < 2; ++i) {
+    const int c0 = hc ? 96 - 32 * i : 32 * i;
     uint32_t sv[32], dv[32];
     tmem_ld32(tS + c0, sv);
     tmem_ld32(tDP + c0, dv);
@@ -175,23 +187,24 @@ __device__ __forceinline__ void bw_p_ds(const BwArgs& a, uint32_t tS, uint32_t t
       }
       dd[e] = pack_bf16x2(d2[0], d2[1]);
     }
-    tmem_st16(tS + (c0 >> 1), dd);
+    tmem_st16(tS + (hc ? 64 : 0) + (c0 >> 1), dd);
   }
 }
 
-// P^T and dS^T of key lane r for one 128-row tile (dK / dV kernel, keys on
-// TMEM lanes): reads S^T and dP^T over the tile's row columns, with each
-// row's (D, lse2) from shared memory (a row past the tile's end has lse2 =
-// +inf, so its P is 0).  Masks the lane when its key is past the block end
-// (key_ok false) and, when causal, rows before the key's token.  Packs P^T as
-// bf16 pairs into [kColS, kColS + 64) and dS^T into [kColDP, kColDP + 64):
-// chunk c0 of 32 columns becomes 16 packed columns at c0 / 2, which this
-// thread has already read.
+// P^T and dS^T of a key lane for half hc of one 128-row tile (dK / dV
+// kernel, keys on TMEM lanes): reads S^T and dP^T over the half's row
+// columns, with each row's (D, lse2) from shared memory (a row past the
+// tile's end has lse2 = +inf, so its P is 0).  Masks the lane when its key
+// is past the block end (key_ok false) and, when causal, rows before the
+// key's token.  Packs P^T as bf16 pairs from column kColS and dS^T from
+// kColDP (see bw_packed_col).
 __device__ __forceinline__ void bw_pt_dst(const BwArgs& a, uint32_t tS, uint32_t tDP,
                                           const float2* __restrict__ dl, bool key_ok,
-                                          bool causal, int64_t key_tok, int64_t row_tok0) {
+                                          bool causal, int64_t key_tok, int64_t row_tok0,
+                                          int hc) {
 #pragma unroll 1
-  for (int c0 = 0; c0 < kTileM; c0 += 32) {
+  for (int i = 0; i < 2; ++i) {
+    const int c0 = hc ? 96 - 32 * i : 32 * i;
     uint32_t sv[32], dv[32];
     tmem_ld32(tS + c0, sv);
     tmem_ld32(tDP + c0, dv);
@@ -215,8 +228,9 @@ __device__ __forceinline__ void bw_pt_dst(const BwArgs& a, uint32_t tS, uint32_t
       pp[e] = pack_bf16x2(p2[0], p2[1]);
       dd[e] = pack_bf16x2(d2[0], d2[1]);
     }
-    tmem_st16(tS + (c0 >> 1), pp);
-    tmem_st16(tDP + (c0 >> 1), dd);
+    const uint32_t pc = (hc ? 64 : 0) + (c0 >> 1);
+    tmem_st16(tS + pc, pp);
+    tmem_st16(tDP + pc, dd);
   }
 }
 
@@ -239,9 +253,10 @@ __device__ __forceinline__ bool bw_wait(uint64_t* bar, uint32_t parity,
 // n + 1 is gathered while tile n computes, once the dV / dK MMAs of tile
 // n - 1, the last readers of its buffer, are done.  The tensor pipe runs the
 // S^T MMA of tile n + 1 after the dV / dK MMAs of tile n that read the
-// columns it overwrites.
+// columns it overwrites.  Eight warps: two per TMEM lane quarter, each taking
+// half of the row columns (see bw_packed_col); two threads gather each row.
 template <int D, int MODE>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
     bw_kv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const BwArgs a) {
   using C = BwCfg<D>;
@@ -254,7 +269,9 @@ __global__ void __launch_bounds__(128, 1)
   uint64_t* mma_bar = bars + 2;  // dV / dK MMAs of a row tile (and every earlier MMA) done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  const int warp = threadIdx.x >> 5, r = threadIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int r = threadIdx.x & 127;  // TMEM lane (key) and gathered row of this thread
+  const int hc = warp >> 2;         // column half (elementwise) / row half (gather)
 
   const int NB = a.P.totals[0];
   const int KT = a.B / kTileN;
@@ -295,7 +312,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   unsigned char* sK = smem + C::kOffK;
   unsigned char* sV = smem + C::kOffV;
   auto sQb = [&](int b) { return smem + (b ? C::kOffX : C::kOffQ); };
@@ -325,8 +342,8 @@ __global__ void __launch_bounds__(128, 1)
     const BwRow x = row_of(n);
     float2 dlv = make_float2(0.f, __int_as_float(0x7f800000));
     if (x.t >= 0) dlv = a.dl[(size_t)x.t * a.Hq + x.h];
-    sdl[(n & 1) * kTileM + r] = dlv;
-    bw_load_row<D>(a, x, r, sQb(n & 1), sDOb(n & 1));
+    if (hc == 0) sdl[(n & 1) * kTileM + r] = dlv;
+    bw_load_row<D>(a, x, r, hc, sQb(n & 1), sDOb(n & 1));
     cp_async_commit();
   };
 
@@ -380,7 +397,7 @@ __global__ void __launch_bounds__(128, 1)
     int64_t row_tok0 = 0;
     if (MODE == kBwOwn) row_tok0 = kstart + (int64_t)(n % own_tiles) * kTileM;
     bw_pt_dst(a, tmem + lane_off + C::kColS, tmem + lane_off + C::kColDP, sdl + b * kTileM,
-              key_ok, MODE == kBwOwn, key_tok, row_tok0);
+              key_ok, MODE == kBwOwn, key_tok, row_tok0, hc);
     tc_wait_st();
     tc_fence_before();
     __syncthreads();
@@ -389,9 +406,9 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
       for (int kk = 0; kk < kTileM / 16; ++kk) {  // K = rows, 16 per step
         const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-        tc_mma_ts_warp(tmem + C::kColA, tmem + C::kColS + kk * 8,
+        tc_mma_ts_warp(tmem + C::kColA, tmem + C::kColS + bw_packed_col(kk),
                        sdesc_mnmajor_sw128(sDOa + kk * 2048, C::kHalf, 1024), idG, acc);
-        tc_mma_ts_warp(tmem + C::kColB, tmem + C::kColDP + kk * 8,
+        tc_mma_ts_warp(tmem + C::kColB, tmem + C::kColDP + bw_packed_col(kk),
                        sdesc_mnmajor_sw128(sQa + kk * 2048, C::kHalf, 1024), idG, acc);
       }
       tc_commit_warp(mma_bar);
@@ -405,12 +422,13 @@ __global__ void __launch_bounds__(128, 1)
   }
   if (ok) {
     tc_fence_after();
-    // row r of the accumulators = key kstart + r; every lane takes part in
-    // the (warp-collective) TMEM loads, only lanes of real keys store
+    // row r of the accumulators = key kstart + r, columns of half hc; every
+    // lane takes part in the (warp-collective) TMEM loads, only lanes of real
+    // keys store
     float* dv = a.dv32 + ((size_t)(kstart + r) * a.Hkv + g) * D;
     float* dk = a.dk32 + ((size_t)(kstart + r) * a.Hkv + g) * D;
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
+    for (int c0 = hc * (D / 2); c0 < (hc + 1) * (D / 2); c0 += 32) {
       uint32_t va[32], vb[32];
       tmem_ld32(tmem + lane_off + C::kColA + c0, va);
       tmem_ld32(tmem + lane_off + C::kColB + c0, vb);
@@ -454,9 +472,11 @@ __global__ void __launch_bounds__(128, 1)
 // dQ MMA of tile kt - 1, the last reader of its buffer, has completed, so the
 // load overlaps tile kt's S / dP MMAs, elementwise pass and dQ MMA.  The dQ
 // MMA of a tile is not waited for: the tensor pipe runs the next tile's S MMA,
-// which overwrites the dS columns it reads, after it.
+// which overwrites the dS columns it reads, after it.  Eight warps: two per
+// TMEM lane quarter (row), each taking half of the key columns (see
+// bw_packed_col); two threads gather each row.
 template <int D, int MODE>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
     bw_q_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const BwArgs a) {
   using C = BwCfg<D>;
@@ -469,7 +489,9 @@ __global__ void __launch_bounds__(128, 1)
   uint64_t* dq_bar = bars + 3;   // dQ MMA of a tile done: its K / V buffer is free
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  const int warp = threadIdx.x >> 5, r = threadIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int r = threadIdx.x & 127;  // TMEM lane and row of this thread
+  const int hc = warp >> 2;         // column half (elementwise) / row half (gather)
   const int NB = a.P.totals[0];
 
   int g, J;
@@ -527,7 +549,7 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   auto sKb = [&](int b) { return smem + (b ? C::kOffX : C::kOffK); };
   auto sVb = [&](int b) { return smem + (b ? C::kOffY : C::kOffV); };
   unsigned char* sQ = smem + C::kOffQ;
@@ -554,7 +576,7 @@ __global__ void __launch_bounds__(128, 1)
     Dr = v.x;
     lse2 = v.y;
   }
-  bw_load_row<D>(a, x, r, sQ, sDO);
+  bw_load_row<D>(a, x, r, hc, sQ, sDO);
   cp_async_wait_all();
   fence_proxy_async_smem();
   __syncthreads();
@@ -595,7 +617,7 @@ __global__ void __launch_bounds__(128, 1)
     if (!ok) break;
     tc_fence_after();
     bw_p_ds<D>(a, tmem + lane_off + C::kColS, tmem + lane_off + C::kColDP, lse2, Dr, nkeys,
-               MODE == kBwOwn, x.t, kbase);
+               MODE == kBwOwn, x.t, kbase, hc);
     tc_wait_st();
     tc_fence_before();
     __syncthreads();
@@ -603,7 +625,7 @@ __global__ void __launch_bounds__(128, 1)
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < kTileN / 16; ++kk)  // K = keys, 16 per step
-        tc_mma_ts_warp(tmem + C::kColA, tmem + C::kColS + kk * 8,
+        tc_mma_ts_warp(tmem + C::kColA, tmem + C::kColS + bw_packed_col(kk),
                        sdesc_mnmajor_sw128(sKa + kk * 2048, C::kHalf, 1024), idQ,
                        (kt > 0 || kk > 0) ? 1u : 0u);
       tc_commit_warp(dq_bar);
@@ -618,7 +640,7 @@ __global__ void __launch_bounds__(128, 1)
   if (ok) {
     tc_fence_after();
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
+    for (int c0 = hc * (D / 2); c0 < (hc + 1) * (D / 2); c0 += 32) {
       uint32_t va[32];
       tmem_ld32(tmem + lane_off + C::kColA + c0, va);
       tc_wait_ld();

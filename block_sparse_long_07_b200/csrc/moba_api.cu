@@ -990,26 +990,26 @@ moba_status backward_passes(const Problem& pr, const void* q, const void* k, con
       MOBA_TRY(launch_scatter(pr, w, sel, u0, nu, st));
       {
         Timed tm(kKBwKv, st);
-        bw_kv_kernel<D, kBwRouted><<<(unsigned)(nu * pr.NBmax * KT), 128, C::kSmemBytes, st>>>(
+        bw_kv_kernel<D, kBwRouted><<<(unsigned)(nu * pr.NBmax * KT), 256, C::kSmemBytes, st>>>(
             tk, tv, a);
         MOBA_CUDA(cudaGetLastError());
       }
       {
         const int64_t items = (int64_t)nu * pr.T * pr.G * np / kTileM + (int64_t)nu * pr.NBmax;
         Timed tm(kKBwQ, st);
-        bw_q_kernel<D, kBwRouted><<<(unsigned)items, 128, C::kSmemBytes, st>>>(tk, tv, a);
+        bw_q_kernel<D, kBwRouted><<<(unsigned)items, 256, C::kSmemBytes, st>>>(tk, tv, a);
         MOBA_CUDA(cudaGetLastError());
       }
     }
     {
       Timed tm(kKBwKv, st);
-      bw_kv_kernel<D, kBwOwn><<<(unsigned)(nu * pr.NBmax * KT), 128, C::kSmemBytes, st>>>(tk, tv,
+      bw_kv_kernel<D, kBwOwn><<<(unsigned)(nu * pr.NBmax * KT), 256, C::kSmemBytes, st>>>(tk, tv,
                                                                                        a);
       MOBA_CUDA(cudaGetLastError());
     }
     {
       Timed tm(kKBwQ, st);
-      bw_q_kernel<D, kBwOwn><<<(unsigned)(nu * pr.G * pr.NQTmax), 128, C::kSmemBytes, st>>>(
+      bw_q_kernel<D, kBwOwn><<<(unsigned)(nu * pr.G * pr.NQTmax), 256, C::kSmemBytes, st>>>(
           tk, tv, a);
       MOBA_CUDA(cudaGetLastError());
     }
