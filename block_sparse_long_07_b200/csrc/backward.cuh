@@ -320,12 +320,29 @@ __global__ void __launch_bounds__(256, 1)
   float2* sdl = reinterpret_cast<float2*>(smem + C::kOffDL);  // [2][128] (D, lse2)
   uint32_t* st = a.status;
 
-  // row r of row tile n: routed -> the bucket's entry; own -> a token of the
-  // block at or after the key tile, for q head n / own_tiles
-  auto row_of = [&](int n) -> BwRow {
+  // row r of row tile n: routed -> the bucket's entry, read one tile ahead
+  // (entry_of) so that no gather waits on it; own -> a token of the block at
+  // or after the key tile, for q head n / own_tiles
+  auto entry_of = [&](int n) -> uint2 {
+    uint2 en = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);  // no entry
+    if (MODE == kBwRouted) {
+      const int64_t e = e0 + (int64_t)n * kTileM + r;
+      if (e < e1) en = a.entries[e];
+    }
+    return en;
+  };
+  auto row_of = [&](int n, uint2 en) -> BwRow {
     BwRow x{-1, 0};
     if (MODE == kBwRouted) {
-      x = bw_row_routed(a, g, e0 + (int64_t)n * kTileM, e1, r);
+      if (en.y != 0xFFFFFFFFu) {
+        const int hh = (int)(en.y & 0xFFFFu);
+        if (en.x < (uint32_t)a.L.T && hh < a.G) {
+          x.t = en.x;
+          x.h = g * a.G + hh;
+        } else {
+          atomicOr(a.status, MOBA_DEV_BAD_INDEX);
+        }
+      }
     } else {
       const int hh = n / own_tiles, qt = n % own_tiles;
       const int64_t t = kstart + (int64_t)qt * kTileM + r;
@@ -336,13 +353,19 @@ __global__ void __launch_bounds__(256, 1)
     }
     return x;
   };
-  // gather row tile n into buffer n & 1: q / dO rows by cp.async (one group),
-  // (D, lse2) by a plain load; a missing row gets lse2 = +inf (P = 0)
+  // gather row tile n into buffer n & 1, all by cp.async in one group: the
+  // q / dO rows and (D, lse2); a missing row gets (0, +inf), so its P is 0
+  uint2 ent = entry_of(0);
   auto gather = [&](int n) {
-    const BwRow x = row_of(n);
-    float2 dlv = make_float2(0.f, __int_as_float(0x7f800000));
-    if (x.t >= 0) dlv = a.dl[(size_t)x.t * a.Hq + x.h];
-    if (hc == 0) sdl[(n & 1) * kTileM + r] = dlv;
+    const BwRow x = row_of(n, ent);
+    if (n + 1 < ntiles) ent = entry_of(n + 1);
+    if (hc == 0) {
+      float2* d = sdl + (n & 1) * kTileM + r;
+      if (x.t >= 0)
+        cp_async_8(d, a.dl + (size_t)x.t * a.Hq + x.h);
+      else
+        *d = make_float2(0.f, __int_as_float(0x7f800000));
+    }
     bw_load_row<D>(a, x, r, hc, sQb(n & 1), sDOb(n & 1));
     cp_async_commit();
   };

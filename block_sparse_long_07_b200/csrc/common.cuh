@@ -122,6 +122,11 @@ __device__ __forceinline__ void cp_async_16(void* dst_smem, const void* src_gmem
                "l"(src_gmem)
                : "memory");
 }
+__device__ __forceinline__ void cp_async_8(void* dst_smem, const void* src_gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst_smem)),
+               "l"(src_gmem)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
