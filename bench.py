@@ -124,20 +124,30 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def code_sha1(text):
+    """sha1 of C++ source with comments and blank lines removed: the counters
+    of a kernel stay valid across edits that touch only its comments."""
+    import hashlib
+    import re
+    t = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    t = re.sub(r"//[^\n]*", "", t)
+    lines = [ln.rstrip() for ln in t.splitlines() if ln.strip()]
+    return hashlib.sha1("\n".join(lines).encode()).hexdigest()
+
+
 def load_traffic(name, entries_per_launch):
     """DRAM bytes per launch of a kernel from the committed ncu summary, scaled
-    to this workload by work entries, or None when the kernel source changed
+    to this workload by work entries, or None when the kernel's code changed
     since the counters were taken."""
-    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             ent = json.load(f).get(name)
-        with open(os.path.join(ROOT, ent["source_file"]), "rb") as f:
-            sha = hashlib.sha1(f.read()).hexdigest()
+        with open(os.path.join(ROOT, ent["source_file"])) as f:
+            sha = code_sha1(f.read())
     except (OSError, ValueError, KeyError, TypeError):
         return None
-    if sha != ent.get("source_sha1"):
+    if sha != ent.get("source_code_sha1"):
         return None
     return float(ent["bytes_per_entry"]) * entries_per_launch
 

@@ -6,7 +6,7 @@
 // historical blocks, combined by online softmax):
 //   kRouted : up to 256 gathered (token, q-head) rows that chose the same past
 //             block J, against the B keys of J, no mask.  Each row writes a
-//             normalised partial O (bf16) and its log2-domain lse to its slot.
+//             normalised partial O (fp16) and its log2-domain lse to its slot.
 //   kOwn    : two consecutive 128-row query tiles of one head against their
 //             own block up to the diagonal, causal mask on the diagonal tile
 //             (wispaper.ai blog, "The Change": the current block is always
@@ -23,7 +23,9 @@
 //   warp  9     TMEM allocation and MMA issue (one elected lane per MMA)
 //   warp 10     Q row gather for routed items (cp.async into swizzled smem)
 // TMEM (512 columns): S_X at 128*X (fp32 scores; after the softmax the first
-// 64 columns hold P_X as packed bf16), O_X at 256 + D*X.
+// 64 columns hold P_X as packed bf16, and on the first tile of an own/dense
+// block columns 64..95 hold the residual weights of rows 0..63), O_X at
+// 256 + D*X.
 // Per KV tile j and sub-tile X: S_X = Q_X K_j^T (both operands in shared
 // memory); the softmax reads S_X, keeps a running max / sum, writes P_X back
 // into TMEM; O_X += P_X V_j takes P_X straight from TMEM, so P never touches
