@@ -61,7 +61,7 @@ struct BwCfg {
   static constexpr int kHalf = kTileM * 128;   // 128 rows x 64 columns bf16
   static constexpr int kTile = kTileM * D * 2; // one [128][D] bf16 tile
   // Six tile slots.  bw_kv: K, V, then two (Q, dO) buffers.  bw_q: K, V,
-  // Q, dO, then a second (K, V) buffer.
+  // Q, dO, a second (K, V) buffer and a third K buffer (kOffK3).
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kTile;
   static constexpr int kOffQ = kOffV + kTile;
@@ -71,6 +71,11 @@ struct BwCfg {
   static constexpr int kOffDL = kOffY + kTile;   // bw_kv: float2 (D, lse2) [2][128 rows]
   static constexpr int kOffBar = kOffDL + 2 * kTileM * 8;
   static constexpr int kSmemBytes = kOffBar + 64 + 1024;
+  // bw_q: a seventh slot (a third K buffer) from kOffDL on, then its barriers
+  static constexpr int kOffK3 = kOffDL;
+  static constexpr int kOffBarQ = kOffK3 + kTile;
+  static constexpr int kSmemBytesQ = kOffBarQ + 64 + 1024;
+  static_assert(kSmemBytesQ <= 232448, "bw_q shared memory beyond the per-CTA limit");
   static constexpr uint32_t kTmemCols = 512;
   // TMEM columns
   static constexpr uint32_t kColS = 0, kColDP = 128, kColA = 256, kColB = 256 + D;
@@ -160,14 +165,14 @@ __host__ __device__ constexpr uint32_t bw_packed_col(int kk) {
 // dS of a row for its half hc of key tile [kbase, kbase + 128) (dQ kernel,
 // rows on TMEM lanes): reads S and dP from TMEM (this thread's lane), masks
 // keys >= nkeys and, when causal, keys after the row's token, and packs dS
-// as bf16 pairs (see bw_packed_col) from TMEM column kColS.
+// as bf16 pairs into tOut: key column c at tOut + c / 2.
 template <int D>
-__device__ __forceinline__ void bw_p_ds(const BwArgs& a, uint32_t tS, uint32_t tDP, float lse2,
-                                        float Dr, int nkeys, bool causal, int64_t trow,
-                                        int64_t kbase, int hc) {
+__device__ __forceinline__ void bw_p_ds(const BwArgs& a, uint32_t tS, uint32_t tDP,
+                                        uint32_t tOut, float lse2, float Dr, int nkeys,
+                                        bool causal, int64_t trow, int64_t kbase, int hc) {
 #pragma unroll 1
   for (int i = 0; i < 2; ++i) {
-    const int c0 = hc ? 96 - 32 * i : 32 * i;
+    const int c0 = 64 * hc + 32 * i;
     uint32_t sv[32], dv[32];
     tmem_ld32(tS + c0, sv);
     tmem_ld32(tDP + c0, dv);
@@ -187,7 +192,7 @@ __device__ __forceinline__ void bw_p_ds(const BwArgs& a, uint32_t tS, uint32_t t
       }
       dd[e] = pack_bf16x2(d2[0], d2[1]);
     }
-    tmem_st16(tS + (hc ? 64 : 0) + (c0 >> 1), dd);
+    tmem_st16(tOut + (c0 >> 1), dd);
   }
 }
 
@@ -490,12 +495,14 @@ __global__ void __launch_bounds__(256, 1)
 //           keys = all of the bucket's block
 //   own:    blockIdx.x = (unit head, query tile); keys = the tile's block up
 //           to and including the tile's own 128 keys (causal)
-// K / V tiles are double-buffered (the second pair in slots 4 and 5): tile
-// kt + 1 is loaded once the
-// dQ MMA of tile kt - 1, the last reader of its buffer, has completed, so the
-// load overlaps tile kt's S / dP MMAs, elementwise pass and dQ MMA.  The dQ
-// MMA of a tile is not waited for: the tensor pipe runs the next tile's S MMA,
-// which overwrites the dS columns it reads, after it.  Eight warps: two per
+// K tiles have three buffers and V tiles two; dS is packed into two TMEM
+// regions from kColB on, which S, dP and the dQ accumulator leave free.  The
+// MMAs of tile kt go S / dP(kt), then dQ(kt - 1), so the elementwise pass of
+// tile kt overlaps the dQ MMA of tile kt - 1.  Tile kt + 1 loads at the start
+// of iteration kt: its K slot was last read by dQ(kt - 2), which ran during
+// the previous elementwise pass, and its V slot by dP(kt - 1).  The commit
+// after S / dP(kt) covers dQ(kt - 2), the last reader of the dS region that
+// tile kt writes.  Eight warps: two per
 // TMEM lane quarter (row), each taking half of the key columns (see
 // bw_packed_col); two threads gather each row.
 template <int D, int MODE>
@@ -506,11 +513,11 @@ __global__ void __launch_bounds__(256, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* kv_full = bars + 0;  // [2] K / V tile landed in buffer b
-  uint64_t* mma_bar = bars + 2;  // S / dP MMAs of a tile (and all earlier MMAs) done
-  uint64_t* dq_bar = bars + 3;   // dQ MMA of a tile done: its K / V buffer is free
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBarQ);
+  uint64_t* kv_full = bars + 0;  // [3] K / V of tile t landed (K slot t % 3)
+  uint64_t* mma_bar = bars + 3;  // S / dP MMAs of a tile (and all earlier MMAs) done
+  uint64_t* dq_bar = bars + 4;   // dQ MMA of a tile done: its K slot is free
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   const int warp = threadIdx.x >> 5;
   const int r = threadIdx.x & 127;  // TMEM lane and row of this thread
@@ -559,6 +566,7 @@ __global__ void __launch_bounds__(256, 1)
   if (threadIdx.x == 0) {
     mbar_init(&kv_full[0], 1);
     mbar_init(&kv_full[1], 1);
+    mbar_init(&kv_full[2], 1);
     mbar_init(mma_bar, 1);
     mbar_init(dq_bar, 1);
     *abort_flag = 0u;
@@ -573,23 +581,26 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  auto sKb = [&](int b) { return smem + (b ? C::kOffX : C::kOffK); };
-  auto sVb = [&](int b) { return smem + (b ? C::kOffY : C::kOffV); };
+  auto sKb = [&](int t) {  // K slot of tile t
+    const int m = t % 3;
+    return smem + (m == 0 ? C::kOffK : (m == 1 ? C::kOffX : C::kOffK3));
+  };
+  auto sVb = [&](int t) { return smem + ((t & 1) ? C::kOffY : C::kOffV); };  // V slot
   unsigned char* sQ = smem + C::kOffQ;
   unsigned char* sDO = smem + C::kOffDO;
   uint32_t* st = a.status;
-  uint32_t nload0 = 0, nload1 = 0, nuse0 = 0, nuse1 = 0;  // K / V loads per buffer (thread 0)
+  int nloaded = 0, nused = 0;  // K / V tiles loaded (thread 0) and consumed
 
   auto load_kv = [&](int kt) {  // thread 0
-    const int b = kt & 1;
+    uint64_t* bar = &kv_full[kt % 3];
     const int64_t kb = kblock + (int64_t)kt * kTileN;
-    mbar_arrive_expect_tx(&kv_full[b], 2 * C::kTile);
+    mbar_arrive_expect_tx(bar, 2 * C::kTile);
 #pragma unroll
     for (int hx = 0; hx < D / 64; ++hx) {
-      tma_load_3d(sKb(b) + hx * C::kHalf, &tm_k, &kv_full[b], hx * 64, g, (int)kb);
-      tma_load_3d(sVb(b) + hx * C::kHalf, &tm_v, &kv_full[b], hx * 64, g, (int)kb);
+      tma_load_3d(sKb(kt) + hx * C::kHalf, &tm_k, bar, hx * 64, g, (int)kb);
+      tma_load_3d(sVb(kt) + hx * C::kHalf, &tm_v, bar, hx * 64, g, (int)kb);
     }
-    if (b) ++nload1; else ++nload0;
+    ++nloaded;
   };
   if (threadIdx.x == 0) load_kv(0);  // overlaps the row gather below
 
@@ -609,14 +620,30 @@ __global__ void __launch_bounds__(256, 1)
   constexpr uint32_t idQ = idesc_bf16_f32(kTileM, D, false, true);
   bool ok = true;
   uint32_t nm = 0, ndq = 0;  // mma_bar and dq_bar phases
+  // dQ(t) += dS(t) K(t): A = dS(t) packed in region t & 1, B = K(t)
+  auto issue_dq = [&](int t) {  // warp 0
+    const uint32_t kb = smem_u32(sKb(t));
+    const uint32_t ds = tmem + C::kColB + 64u * (uint32_t)(t & 1);
+#pragma unroll
+    for (int kk = 0; kk < kTileN / 16; ++kk)  // K = keys, 16 per step
+      tc_mma_ts_warp(tmem + C::kColA, ds + kk * 8,
+                     sdesc_mnmajor_sw128(kb + kk * 2048, C::kHalf, 1024), idQ,
+                     (t > 0 || kk > 0) ? 1u : 0u);
+    tc_commit_warp(dq_bar);
+  };
   for (int kt = 0; kt < nkt && ok; ++kt) {
-    const int b = kt & 1;
     const int64_t kbase = kblock + (int64_t)kt * kTileN;
     const int nkeys = min(kTileN, blen - kt * kTileN);
-    const uint32_t sKa = smem_u32(sKb(b)), sVa = smem_u32(sVb(b));
-    ok = bw_wait(&kv_full[b], (uint32_t)(kt >> 1) & 1u, abort_flag, st);
+    const uint32_t sKa = smem_u32(sKb(kt)), sVa = smem_u32(sVb(kt));
+    if (threadIdx.x == 0 && kt + 1 < nkt) {
+      // K slot of tile kt + 1 was last read by dQ(kt - 2); its V slot by dP(kt - 1)
+      const bool free_ok = kt < 2 || mbar_wait(dq_bar, (uint32_t)(kt - 2) & 1u, abort_flag, st);
+      if (free_ok) load_kv(kt + 1);
+    }
+    __syncwarp();  // warp 0 reconverges before the block-wide wait
+    ok = bw_wait(&kv_full[kt % 3], (uint32_t)(kt / 3) & 1u, abort_flag, st);
     if (!ok) break;
-    if (b) ++nuse1; else ++nuse0;
+    ++nused;
     if (warp == 0) {
       tc_fence_after();
 #pragma unroll
@@ -628,30 +655,24 @@ __global__ void __launch_bounds__(256, 1)
                        sdesc_kmajor_sw128(sVa + off), idS, kk > 0 ? 1u : 0u);
       }
       tc_commit_warp(mma_bar);
+      if (kt > 0) issue_dq(kt - 1);
     }
-    if (threadIdx.x == 0 && kt + 1 < nkt) {
-      // buffer (kt + 1) & 1 was last read by the dQ MMA of tile kt - 1
-      const bool free_ok = kt == 0 || mbar_wait(dq_bar, (uint32_t)(kt - 1) & 1u, abort_flag, st);
-      if (free_ok) load_kv(kt + 1);
-    }
-    __syncwarp();  // warp 0 reconverges before the block-wide wait
+    if (kt > 0) ++ndq;
     ok = bw_wait(mma_bar, nm & 1, abort_flag, st);
     ++nm;
     if (!ok) break;
     tc_fence_after();
-    bw_p_ds<D>(a, tmem + lane_off + C::kColS, tmem + lane_off + C::kColDP, lse2, Dr, nkeys,
+    bw_p_ds<D>(a, tmem + lane_off + C::kColS, tmem + lane_off + C::kColDP,
+               tmem + lane_off + C::kColB + 64u * (uint32_t)(kt & 1), lse2, Dr, nkeys,
                MODE == kBwOwn, x.t, kbase, hc);
     tc_wait_st();
     tc_fence_before();
     __syncthreads();
+  }
+  if (ok) {  // the last tile's dQ MMA
     if (warp == 0) {
       tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kTileN / 16; ++kk)  // K = keys, 16 per step
-        tc_mma_ts_warp(tmem + C::kColA, tmem + C::kColS + bw_packed_col(kk),
-                       sdesc_mnmajor_sw128(sKa + kk * 2048, C::kHalf, 1024), idQ,
-                       (kt > 0 || kk > 0) ? 1u : 0u);
-      tc_commit_warp(dq_bar);
+      issue_dq(nkt - 1);
     }
     ++ndq;
   }
@@ -676,8 +697,9 @@ __global__ void __launch_bounds__(256, 1)
   }
   // teardown: after an abort, loads and MMAs may still be in flight
   if (!ok && threadIdx.x == 0) {
-    if (nload0 > nuse0) mbar_wait_teardown(&kv_full[0], (nload0 - 1u) & 1u, 200000000ull);
-    if (nload1 > nuse1) mbar_wait_teardown(&kv_full[1], (nload1 - 1u) & 1u, 200000000ull);
+    // at most two loads are unconsumed (tiles nused and nused + 1)
+    for (int t = nused; t < nloaded; ++t)
+      mbar_wait_teardown(&kv_full[t % 3], (uint32_t)(t / 3) & 1u, 200000000ull);
   }
   if (warp == 0) {
     tc_commit_warp(mma_bar);  // arrives once every MMA of this CTA has completed

@@ -950,9 +950,9 @@ moba_status backward_passes(const Problem& pr, const void* q, const void* k, con
   MOBA_CUDA(cudaFuncSetAttribute(bw_kv_kernel<D, kBwOwn>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
   MOBA_CUDA(cudaFuncSetAttribute(bw_q_kernel<D, kBwRouted>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytesQ));
   MOBA_CUDA(cudaFuncSetAttribute(bw_q_kernel<D, kBwOwn>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytesQ));
   BwArgs a;
   memset(&a, 0, sizeof a);
   a.q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -997,7 +997,7 @@ moba_status backward_passes(const Problem& pr, const void* q, const void* k, con
       {
         const int64_t items = (int64_t)nu * pr.T * pr.G * np / kTileM + (int64_t)nu * pr.NBmax;
         Timed tm(kKBwQ, st);
-        bw_q_kernel<D, kBwRouted><<<(unsigned)items, 256, C::kSmemBytes, st>>>(tk, tv, a);
+        bw_q_kernel<D, kBwRouted><<<(unsigned)items, 256, C::kSmemBytesQ, st>>>(tk, tv, a);
         MOBA_CUDA(cudaGetLastError());
       }
     }
@@ -1009,7 +1009,7 @@ moba_status backward_passes(const Problem& pr, const void* q, const void* k, con
     }
     {
       Timed tm(kKBwQ, st);
-      bw_q_kernel<D, kBwOwn><<<(unsigned)(nu * pr.G * pr.NQTmax), 256, C::kSmemBytes, st>>>(
+      bw_q_kernel<D, kBwOwn><<<(unsigned)(nu * pr.G * pr.NQTmax), 256, C::kSmemBytesQ, st>>>(
           tk, tv, a);
       MOBA_CUDA(cudaGetLastError());
     }
