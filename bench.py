@@ -152,6 +152,37 @@ def load_traffic(name, entries_per_launch):
     return float(ent["bytes_per_entry"]) * entries_per_launch
 
 
+class RankGroup:
+    """The processes of a multi-GPU run, one per GPU: a barrier and the max of
+    a scalar (the step time) over ranks through the given torch.distributed
+    module (NCCL here; any backend works), or no-ops for a single process."""
+
+    def __init__(self, pg=None, device="cpu"):
+        self.pg, self.device = pg, device
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x):
+        if self.pg is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+
+def rank_seed(w, rank):
+    """Each rank draws its own copy of the workload (independent problems)."""
+    return w.seed + 1000 * rank
+
+
+def whole_job_rate(world, units_per_rank_step, ms_max):
+    """Units per second over all ranks, each step timed by the slowest rank."""
+    return world * units_per_rank_step / (ms_max / 1e3)
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -246,18 +277,10 @@ def run_moba(args, w):
                                 device_id=dev)
         pg = dist
 
-    def barrier():
-        if pg is not None:
-            pg.barrier()
+    ranks = RankGroup(pg, dev)
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
-    def max_over_ranks(x):
-        if pg is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
-
-    q, k, v = S.make_qkv(w, dev, seed=w.seed + 1000 * rank)
+    q, k, v = S.make_qkv(w, dev, seed=rank_seed(w, rank))
     T = w.T
     varlen = not w.batch_mode
     if varlen:
@@ -331,7 +354,7 @@ def run_moba(args, w):
         print("device status %d after the timed steps" % status, file=sys.stderr)
     ms_local = e0.elapsed_time(e1) / args.steps
     ms = max_over_ranks(ms_local)
-    value = world * flops / (ms / 1e3) / 1e12
+    value = whole_job_rate(world, flops, ms) / 1e12
 
     peaks, peak_src = load_peaks()
     peak_tf = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -413,7 +436,7 @@ def run_moba(args, w):
             e1.record(stream)
             torch.cuda.synchronize()
             ems = max_over_ranks(e0.elapsed_time(e1) / n_e)
-            e2e = {"value": world * flops / (ems / 1e3) / 1e12, "unit": "TFLOP/s",
+            e2e = {"value": whole_job_rate(world, flops, ems) / 1e12, "unit": "TFLOP/s",
                    "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                    "call": ("moba_forward_host (copies inside the call)"
                             if not varlen and route == "gate" else
@@ -508,7 +531,7 @@ def run_decode(args, w):
         raise SystemExit("decode mode takes a batch workload")
     b, N = len(w.lengths), w.lengths[0]
     G = w.Hq // w.Hkv
-    q, k, v = S.make_qkv(w, dev, seed=w.seed + 1000 * rank)
+    q, k, v = S.make_qkv(w, dev, seed=rank_seed(w, rank))
     kc = k.view(b, N, w.Hkv, w.d)
     vc = v.view(b, N, w.Hkv, w.d)
     qd = q.view(b, N, w.Hq, w.d)[:, N - 1].contiguous()
@@ -526,16 +549,8 @@ def run_decode(args, w):
         moba.kbar_cache_update(kc, lens, kbar, w.B, only_last=True, ws=ws)
         moba.decode(qin, kc, vc, lens, kbar, w.B, w.k, ws=ws, out=o, lse=lse, sel_out=sel)
 
-    def barrier():
-        if pg is not None:
-            pg.barrier()
-
-    def max_over_ranks(x):
-        if pg is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+    ranks = RankGroup(pg, dev)
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     for _ in range(args.warmup):
         step()
@@ -566,7 +581,7 @@ def run_decode(args, w):
     if status != 0:
         print("device status %d after the timed steps" % status, file=sys.stderr)
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-    value = world * b / (ms / 1e3)
+    value = whole_job_rate(world, b, ms)
 
     peaks, peak_src = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
@@ -605,7 +620,7 @@ def run_decode(args, w):
         e1.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-        e2e = {"value": world * b / (ems / 1e3), "unit": "steps/s", "ms_per_step": ems,
+        e2e = {"value": whole_job_rate(world, b, ems), "unit": "steps/s", "ms_per_step": ems,
                "h2d_bytes_per_step": qh.numel() * qh.element_size(),
                "d2h_bytes_per_step": oh.numel() * oh.element_size() +
                lh.numel() * lh.element_size()}
