@@ -199,3 +199,63 @@ def test_decode_pointer_and_workspace_checks(lib):
                                       None) == WORKSPACE
     assert lib.moba_kbar_cache_update(None, fake, fake, 0, ctypes.byref(p), fake, need,
                                       None) == INVALID
+
+
+def test_backward_argument_checks(lib):
+    p = _p()
+    fake = ctypes.c_void_p(1 << 20)
+    need = moba.backward_workspace_size(p, 1)
+    assert need > 0 and moba.backward_workspace_size(p, 2) > need
+    args = [fake] * 10  # q, k, v, o, lse, dO, sel, dq, dk, dv
+    for bad in range(10):
+        a = list(args)
+        a[bad] = None
+        assert lib.moba_backward(*a, ctypes.byref(p), fake, need, None) == INVALID
+    a = list(args)
+    a[5] = ctypes.c_void_p((1 << 20) + 8)  # dO not 16-byte aligned
+    assert lib.moba_backward(*a, ctypes.byref(p), fake, need, None) == INVALID
+    a = list(args)
+    a[6] = ctypes.c_void_p((1 << 20) + 2)  # sel not 4-byte aligned
+    assert lib.moba_backward(*a, ctypes.byref(p), fake, need, None) == INVALID
+    assert lib.moba_backward(*args, ctypes.byref(p), fake, need - 1, None) == WORKSPACE
+    assert lib.moba_backward(*args, ctypes.byref(p), None, need, None) == WORKSPACE
+    bad = _p(d=96)
+    assert lib.moba_backward(*args, ctypes.byref(bad), fake, 1 << 40, None) == UNSUPPORTED
+
+
+def test_routing_variant_argument_checks(lib):
+    p = _p()
+    fake = ctypes.c_void_p(1 << 20)
+    need = moba.workspace_size(p, 1)
+    # static selections: a destination and one of the two modes
+    assert lib.moba_static_selection(None, 0, ctypes.byref(p), None) == INVALID
+    assert lib.moba_static_selection(ctypes.c_void_p((1 << 20) + 2), 0, ctypes.byref(p),
+                                     None) == INVALID
+    assert lib.moba_static_selection(fake, 7, ctypes.byref(p), None) == INVALID
+    # min/max gate: q, k, sel, then the workspace
+    assert lib.moba_gate_minmax(None, fake, fake, ctypes.byref(p), fake, need, None) == INVALID
+    assert lib.moba_gate_minmax(fake, fake, None, ctypes.byref(p), fake, need, None) == INVALID
+    assert lib.moba_gate_minmax(fake, fake, fake, ctypes.byref(p), fake, need - 1,
+                                None) == WORKSPACE
+    # forward over a given selection needs the selection
+    assert lib.moba_forward_selected(fake, fake, fake, fake, fake, None, ctypes.byref(p), fake,
+                                     need, None) == INVALID
+    assert lib.moba_forward_minmax(None, fake, fake, fake, fake, None, ctypes.byref(p), fake,
+                                   need, None) == INVALID
+
+
+def test_forward_host_argument_checks(lib):
+    p = _p()
+    host = ctypes.c_void_p(1 << 20)
+    dev = ctypes.c_void_p(1 << 24)  # kAlign-aligned
+    need = moba.forward_host_buffer_size(p, 1)
+    assert need > moba.workspace_size(p, 1)  # workspace plus the staging of one kv-head group
+    for bad in range(5):  # q, k, v, o, lse
+        a = [host] * 5
+        a[bad] = None
+        assert lib.moba_forward_host(*a, None, ctypes.byref(p), dev, need, None) == INVALID
+    a = [host] * 5
+    assert lib.moba_forward_host(*a, None, ctypes.byref(p), None, need, None) == WORKSPACE
+    assert lib.moba_forward_host(*a, None, ctypes.byref(p), ctypes.c_void_p((1 << 24) + 16),
+                                 need, None) == WORKSPACE
+    assert lib.moba_forward_host(*a, None, ctypes.byref(p), dev, need - 1, None) == WORKSPACE
