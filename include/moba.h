@@ -140,7 +140,10 @@ moba_status moba_forward_varlen(const void *q, const void *k, const void *v,
  * more: the largest group of kv heads that fits is used); its first 256 bytes
  * are the status word of a workspace (zero them before first use;
  * moba_last_device_status(dev_buf) reads them).  Results equal moba_forward's.
- * Returns when the work is queued; synchronise `stream` before reading o. */
+ * Returns when the work is queued; synchronise `stream` before reading o.
+ * Errors: a null q, k, v, o or lse -> MOBA_ERR_INVALID_ARG; dev_buf null, not
+ * 256-byte aligned or smaller than one kv head's share -> MOBA_ERR_WORKSPACE;
+ * parameters as for moba_forward. */
 size_t moba_forward_host_buffer_size(const moba_params *p, int heads_per_pass);
 moba_status moba_forward_host(const void *q, const void *k, const void *v, void *o, float *lse,
                               int32_t *sel_out, const moba_params *p, void *dev_buf,
@@ -159,7 +162,13 @@ moba_status moba_forward_host(const void *q, const void *k, const void *v, void 
  * fp32 and sel [batch][Hq][seqlen][top_k] exactly as moba_forward wrote them.
  * Outputs dq [batch][seqlen][Hq][d], dk / dv [batch][seqlen][Hkv][d], bf16.
  * The workspace holds the fp32 accumulators (moba_backward_workspace_size;
- * heads_per_pass as for the forward). */
+ * heads_per_pass as for the forward; its status word as for the forward).
+ * Errors: a null pointer, a tensor not 16-byte aligned, or lse / sel not
+ * 4-byte aligned -> MOBA_ERR_INVALID_ARG; parameters as for moba_forward
+ * (MOBA_ERR_UNSUPPORTED for d or top_k outside what the kernels take); a
+ * workspace that is null, misaligned or too small -> MOBA_ERR_WORKSPACE.  A
+ * selection entry out of range (a future or missing block) is skipped and
+ * latched in the status word (MOBA_ERR_DEVICE_CHECK). */
 size_t moba_backward_workspace_size(const moba_params *p, int heads_per_pass);
 moba_status moba_backward(const void *q, const void *k, const void *v, const void *o,
                           const float *lse, const void *dO, const int32_t *sel, void *dq,
