@@ -83,6 +83,40 @@ def test_one_token_blocks_minmax_equals_mean_gate():
     np.testing.assert_allclose(mb, ma, rtol=0, atol=1e-12)
 
 
+def test_minmax_score_is_a_dot_product_of_sign_split_queries():
+    # max(q_c M_c, q_c m_c) = max(q_c, 0) M_c + min(q_c, 0) m_c since M_c >= m_c:
+    # the min/max score is q+ . M + q- . m, two plain matrix products.  The
+    # oracle's selection must be the top-(k-1) of those scores (ties to the
+    # lower block) on every row whose (k-1)-th / k-th gap is not a rounding
+    # tie, at a size brute force cannot reach.
+    lengths, Hq, Hkv, d, B, k = [4096], 4, 2, 32, 64, 6
+    q, kb, v, cu = _problem(lengths, Hq, Hkv, d, B, k, seed=31)
+    orc = Oracle(q, kb, v, cu, Hq, Hkv, d, B, k)
+    kx, kn = orc.block_minmax()
+    qf = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).double().numpy()  # exact
+    rows = np.arange(0, 4096, 7)
+    sel, _, _ = orc.select_minmax(rows)
+    G = Hq // Hkv
+    checked = 0
+    for a, t in enumerate(rows):
+        i = t // B
+        if i == 0:
+            continue
+        for h in range(Hq):
+            g = h // G
+            qp, qn = np.maximum(qf[t, h], 0.0), np.minimum(qf[t, h], 0.0)
+            s = kx[g, :i] @ qp + kn[g, :i] @ qn
+            order = sorted(range(i), key=lambda j: (-s[j], j))
+            npast = min(k - 1, i)
+            if npast < i and abs(s[order[npast - 1]] - s[order[npast]]) < 1e-9 * np.abs(s).max():
+                continue
+            want = sorted(order[:npast]) + [i]
+            got = [int(x) for x in sel[a, h] if x >= 0]
+            assert got == want, (t, h)
+            checked += 1
+    assert checked > 1500
+
+
 def _tb(a):
     return bf16_bits(torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16))
 
