@@ -28,7 +28,7 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(moba_[a-z_]+)\s*\(", text)))
 
 
-def test_header_declares_the_survey_calls():
+def test_header_declares_the_prefill_calls():
     names = declared_functions()
     for n in ("moba_gate", "moba_forward", "moba_forward_varlen", "moba_full_causal",
               "moba_workspace_size", "moba_status_string"):
