@@ -135,3 +135,51 @@ def sample_rows(w: Workload, per_head_rows: int, seed: int = 1234) -> np.ndarray
         return np.arange(T, dtype=np.int64)
     rng = np.random.default_rng(seed)
     return np.sort(rng.choice(T, size=per_head_rows, replace=False)).astype(np.int64)
+
+
+# Inputs whose attention rows are peaky: keys planted late in every block
+# that outscore everything before them by far, and queries aligned with them.
+# They exist so that the running maximum of a row's scores jumps, after the
+# first 128-key tile of the keys it attends, by many powers of two (the
+# attention kernels rescale their accumulators only on such a jump).
+#
+# Recipe, on top of make_qkv's draws:
+#   * one unit direction u_g per kv head (N(0, I) normalised), drawn from a
+#     generator seeded with seed + 7919;
+#   * q heads with an even index get a * u_g added (their kv head's u);
+#   * in every block, for each (tile, c) of `plants`, the keys at positions
+#     tile * 128 + 37 and tile * 128 + 91 of the block (where they exist) get
+#     c * u_g added;
+#   * v is multiplied by v_scale (a power of two, so exactly).
+# The additions happen in fp32 on the bf16 draws and are rounded once more.
+PEAKY_PLANTS = ((1, 24.0), (3, 48.0))
+
+
+def make_peaky_qkv(w: Workload, device="cpu", a: float = 6.0, plants=PEAKY_PLANTS,
+                   v_scale: float = 0.25, seed: Optional[int] = None):
+    dev = torch.device(device)
+    q, k, v = make_qkv(w, dev, seed=seed)
+    g = torch.Generator(device=dev)
+    g.manual_seed((w.seed if seed is None else seed) + 7919)
+    u = torch.randn(w.Hkv, w.d, generator=g, device=dev, dtype=torch.float32)
+    u = u / u.norm(dim=1, keepdim=True)
+    G = w.Hq // w.Hkv
+    qf = q.float()
+    for h in range(0, w.Hq, 2):
+        qf[:, h] += a * u[h // G]
+    kf = k.float()
+    pos = []
+    base = 0
+    for L in w.lengths:
+        for b0 in range(0, L, w.B):
+            for tile, c in plants:
+                for off in (37, 91):
+                    p = b0 + tile * 128 + off
+                    if p < min(L, b0 + w.B):
+                        pos.append((base + p, c))
+        base += L
+    if pos:
+        idx = torch.tensor([p for p, _ in pos], device=dev, dtype=torch.long)
+        cs = torch.tensor([c for _, c in pos], device=dev, dtype=torch.float32)
+        kf[idx] += cs[:, None, None] * u[None, :, :]
+    return qf.to(torch.bfloat16), kf.to(torch.bfloat16), (v.float() * v_scale).to(torch.bfloat16)

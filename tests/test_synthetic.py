@@ -49,3 +49,27 @@ def test_block_ids_restart_with_each_sequence():
     ids = S.block_ids([300, 5, 256], 256)
     assert list(ids[:300:100]) == [0, 0, 0] and ids[256] == 1
     assert ids[300] == 2 and ids[305] == 3 and ids[-1] == 3
+
+
+def test_peaky_inputs_force_the_rescale_rule():
+    """The planted-key recipe makes a row's running score maximum jump past
+    the attention kernels' rescale threshold after the first key tile: in
+    the routed span of past blocks, in the own block and in the dense span
+    (replayed in fp64 on CPU-drawn inputs of the recipe)."""
+    import sys, os
+    sys.path.insert(0, os.path.dirname(__file__))
+    from oracle import Oracle, bf16_bits
+    from rescale_util import rescale_events
+    w = S.Workload("peaky", [4096], 4, 2, 128, 512, 3, seed=3131)
+    q, k, v = S.make_peaky_qkv(w, "cpu")
+    assert torch.equal(v.float() * 4, S.make_qkv(w, "cpu")[2].float())  # v scaled exactly
+    qb, kb, vb = bf16_bits(q), bf16_bits(k), bf16_bits(v)
+    rows = np.arange(w.T, dtype=np.int64)
+    sel, _, _ = Oracle(qb, kb, vb, w.cu, 4, 2, 128, 512, 3).select(rows)
+    ev_r, ev_o = rescale_events(qb, kb, w.cu, rows, 4, 2, 128, 512, sel=sel)
+    ev_d, _ = rescale_events(qb, kb, w.cu, rows, 4, 2, 128, 512, dense=True)
+    # the peaked (even) heads: every row with a past block rescales there
+    assert (ev_r[:, 0::2] > 0).mean() >= 0.85
+    assert (ev_o[:, 0::2] > 0).mean() >= 0.5
+    assert (ev_d[:, 0::2] > 0).mean() >= 0.9
+    assert (ev_r[:, 0::2] > 1).mean() >= 0.5 * (ev_r[:, 0::2] > 0).mean()  # tile 3 again
