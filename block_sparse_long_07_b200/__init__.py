@@ -23,7 +23,7 @@ _STATUS = {0: "MOBA_OK", 1: "MOBA_ERR_INVALID_ARG", 2: "MOBA_ERR_UNSUPPORTED",
            6: "MOBA_ERR_DEVICE_CHECK"}
 
 EXPORTS = ("moba_workspace_size", "moba_workspace_size_varlen", "moba_gate", "moba_gate_varlen",
-           "moba_gate_noalloc",
+           "moba_gate_noalloc", "moba_gate_noalloc_status",
            "moba_forward", "moba_forward_varlen", "moba_full_causal_workspace_size",
            "moba_full_causal", "moba_full_causal_varlen", "moba_last_device_status",
            "moba_status_string", "moba_version", "moba_last_error_string", "moba_profile_enable", "moba_profile_reset",
@@ -86,6 +86,8 @@ def load_library(path=None):
     lib.moba_gate_varlen.argtypes = [vp, vp, vp, i32, i64, vp, pp, vp, sz, vp]
     lib.moba_gate_noalloc.restype = i32
     lib.moba_gate_noalloc.argtypes = [vp, vp, vp, pp, vp]
+    lib.moba_gate_noalloc_status.restype = i32
+    lib.moba_gate_noalloc_status.argtypes = [vp]
     lib.moba_forward.restype = i32
     lib.moba_forward.argtypes = [vp, vp, vp, vp, vp, vp, pp, vp, sz, vp]
     lib.moba_forward_varlen.restype = i32

@@ -83,6 +83,9 @@ struct Timed {
 // Last CUDA runtime error seen by this thread inside the library.
 thread_local const char* g_last_cuda_error = "no error";
 
+// Device address of the allocation-free gate's scratch (defined with it).
+moba_status gate_scratch_address(void** out);
+
 moba_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return MOBA_OK;
   g_last_cuda_error = cudaGetErrorString(e);
@@ -1179,9 +1182,13 @@ extern "C" {
 
 moba_status moba_selftest_wait_timeout(void* ws, size_t ws_bytes, long long limit_cycles,
                                        moba_stream_t stream) {
-  if (!ws || (reinterpret_cast<uintptr_t>(ws) % kAlign) || ws_bytes < kAlign)
-    return MOBA_ERR_WORKSPACE;
   if (limit_cycles <= 0 || limit_cycles > MOBA_WAIT_LIMIT_CYCLES) return MOBA_ERR_INVALID_ARG;
+  if (!ws) {  // the allocation-free gate's status word
+    MOBA_TRY(gate_scratch_address(&ws));
+    ws_bytes = kAlign;
+  }
+  if ((reinterpret_cast<uintptr_t>(ws) % kAlign) || ws_bytes < kAlign)
+    return MOBA_ERR_WORKSPACE;
   wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<uint32_t*>(ws), limit_cycles);
   return cuda_status(cudaGetLastError());
@@ -1568,19 +1575,27 @@ extern "C" moba_status moba_gate_noalloc(const void* q, const void* k, int32_t* 
                                          const moba_params* p, moba_stream_t stream) {
   Problem pr;
   MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  if (!topk_supported(pr)) return MOBA_ERR_UNSUPPORTED;
+  // the scratch limit first: a shape it refuses never reaches the pointers
+  if (carve_gate_scratch(pr, nullptr).bytes > kGateScratchBytes) return MOBA_ERR_WORKSPACE;
   if (!q || !k || !sel || !aligned16(q) || !aligned16(k) ||
       (reinterpret_cast<uintptr_t>(sel) & 3))
     return MOBA_ERR_INVALID_ARG;
-  if (!topk_supported(pr)) return MOBA_ERR_UNSUPPORTED;
-  if (carve_gate_scratch(pr, nullptr).bytes > kGateScratchBytes) return MOBA_ERR_WORKSPACE;
   if (pr.T == 0) return MOBA_OK;
   void* base = nullptr;
   MOBA_TRY(gate_scratch_address(&base));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const Ws w = carve_gate_scratch(pr, static_cast<char*>(base));
-  // the status word is the only state a call reads before writing it
-  MOBA_CUDA(cudaMemsetAsync(w.status, 0, sizeof(uint32_t), st));
+  // The status word is not cleared here: device checks of every call latch
+  // in it until moba_gate_noalloc_status reads and clears it.  The kernels
+  // only ever OR bits into it, so a latched bit changes no later result.
   MOBA_TRY(run_plan_pool(pr, k, w, st));
   return pr.D == 128 ? launch_gate<128>(pr, q, w, sel, nullptr, st)
                      : launch_gate<64>(pr, q, w, sel, nullptr, st);
+}
+
+extern "C" moba_status moba_gate_noalloc_status(moba_stream_t stream) {
+  void* base = nullptr;
+  MOBA_TRY(gate_scratch_address(&base));
+  return moba_last_device_status(base, stream);
 }

@@ -116,9 +116,19 @@ moba_status moba_gate_varlen(const void *q, const void *k, const int32_t *cu_seq
  *     can overlap on the GPU race, and the caller must order them;
  *   - the first call on a device looks up the array's address with that
  *     device current; make that first call before any stream capture.
- * Results equal moba_gate's for the same inputs. */
+ * Results equal moba_gate's for the same inputs.  The size limit is checked
+ * before the pointers, so a refused shape launches nothing whatever the
+ * pointers are.  Device-side checks (a pipeline wait that ran out of time,
+ * a bad index) latch bits in the array's status word, which no call clears:
+ * moba_gate_noalloc_status reads them. */
 moba_status moba_gate_noalloc(const void *q, const void *k, int32_t *sel, const moba_params *p,
                               moba_stream_t stream);
+/* Status of the allocation-free gate's device checks on the current device:
+ * synchronises `stream`, reads the status word every moba_gate_noalloc call
+ * on this device latches into, clears it and returns MOBA_OK,
+ * MOBA_ERR_TIMEOUT or MOBA_ERR_DEVICE_CHECK (as moba_last_device_status does
+ * for a workspace).  Allocates nothing. */
+moba_status moba_gate_noalloc_status(moba_stream_t stream);
 
 /* Full MoBA prefill forward: o and lse; sel_out (nullable) receives the
  * selection. */
@@ -317,7 +327,9 @@ int moba_profile_read(moba_kernel_time *out, int max_entries);
  * barrier nothing arrives on.  The wait gives up and latches the timeout bit
  * in ws's status word; moba_last_device_status(ws) then returns
  * MOBA_ERR_TIMEOUT and the context stays usable.  Shows that a stuck pipeline
- * ends in an error status instead of a hang.  ws needs 256 bytes. */
+ * ends in an error status instead of a hang.  ws needs 256 bytes; a null ws
+ * targets the allocation-free gate's status word instead (read it back with
+ * moba_gate_noalloc_status). */
 moba_status moba_selftest_wait_timeout(void *ws, size_t ws_bytes, long long limit_cycles,
                                        moba_stream_t stream);
 

@@ -146,8 +146,11 @@ def test_binding_refuses_missing_library(tmp_path):
 
 
 def test_selftest_argument_checks(lib):
-    assert lib.moba_selftest_wait_timeout(None, 4096, 1000, None) == WORKSPACE
+    # the limit is checked first; a null ws would aim at the allocation-free
+    # gate's status word, which needs a device
+    assert lib.moba_selftest_wait_timeout(None, 4096, 0, None) == INVALID
     fake = ctypes.c_void_p(1 << 20)
+    assert lib.moba_selftest_wait_timeout(ctypes.c_void_p(1 << 20 | 8), 4096, 1000, None) == WORKSPACE
     assert lib.moba_selftest_wait_timeout(fake, 4096, 0, None) == INVALID
     assert lib.moba_selftest_wait_timeout(fake, 4096, 10**12, None) == INVALID
     assert lib.moba_selftest_wait_timeout(fake, 16, 1000, None) == WORKSPACE
