@@ -429,7 +429,7 @@ def run_moba(args, w):
             estep()
             torch.cuda.synchronize()
             barrier()
-            n_e = max(1, min(args.steps, 3))
+            n_e = args.steps  # the same number of timed steps as the device-resident value
             e0.record(stream)
             for _ in range(n_e):
                 estep()
@@ -437,7 +437,8 @@ def run_moba(args, w):
             torch.cuda.synchronize()
             ems = max_over_ranks(e0.elapsed_time(e1) / n_e)
             e2e = {"value": whole_job_rate(world, flops, ems) / 1e12, "unit": "TFLOP/s",
-                   "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                   "ms_per_step": ems, "steps": n_e, "h2d_bytes_per_step": h2d,
+                   "d2h_bytes_per_step": d2h,
                    "call": ("moba_forward_host (copies inside the call)"
                             if not varlen and route == "gate" else
                             "host copies + moba_forward")}

@@ -5,7 +5,8 @@
 // Every wait here is bounded.  A wait that runs out sets the CTA's abort
 // flag and the library's device status word (MOBA_DEV_TIMEOUT) and returns
 // false; callers then leave their loops and the kernel tears down cleanly
-// (see attn_tc.cuh).  No kernel traps or spins without a limit.
+// (as the attention kernels in attn_tc2.cuh do).  No kernel traps or
+// spins without a limit.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>

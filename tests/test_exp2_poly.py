@@ -85,3 +85,33 @@ def test_integer_points_and_rounding_ties():
 def test_below_the_clamp_stays_tiny_and_finite():
     v = exp2_poly_np(np.array([-1e4, -300.0, -126.5, -np.inf], np.float32))
     assert np.all(np.isfinite(v)) and np.all(v >= 0) and np.all(v < 2.0 ** -125)
+
+
+def _minimax_fit(deg, npts=4001):
+    """Coefficients c0..c_deg minimising max |p(f) / 2^f - 1| over npts
+    equispaced points of [-1/2, 1/2], as a linear program in (c, t):
+    minimise t subject to -t <= p(f_i) / 2^f_i - 1 <= t."""
+    from scipy.optimize import linprog
+    f = np.linspace(-0.5, 0.5, npts)
+    y = 2.0 ** f
+    V = np.vstack([f ** k for k in range(deg + 1)]).T / y[:, None]
+    n = deg + 1
+    ones = np.ones((len(f), 1))
+    A = np.vstack([np.hstack([V, -ones]), np.hstack([-V, -ones])])
+    b = np.concatenate([np.ones(len(f)), -np.ones(len(f))])
+    cost = np.zeros(n + 1)
+    cost[-1] = 1.0
+    res = linprog(cost, A_ub=A, b_ub=b, bounds=[(None, None)] * (n + 1), method="highs")
+    assert res.success
+    return res.x[:n], res.x[-1]
+
+
+def test_constants_come_from_the_minimax_fit():
+    """Refit the degree-4 polynomial and compare with the source's constants
+    (rounded to fp32), so the derivation of the constants is reproducible."""
+    _, _, (c4, c3, c2, c1, c0) = _constants()
+    coef, err = _minimax_fit(4)
+    assert err < 2.7e-6
+    got = np.array([c0, c1, c2, c3, c4], np.float64)
+    assert np.allclose(got, coef.astype(np.float32).astype(np.float64), rtol=0, atol=2e-7), \
+        (got, coef)
