@@ -31,7 +31,10 @@ EXPORTS = ("moba_workspace_size", "moba_workspace_size_varlen", "moba_gate", "mo
            "moba_kbar_cache_size", "moba_kbar_cache_update", "moba_decode",
            "moba_static_selection", "moba_gate_minmax", "moba_forward_selected",
            "moba_forward_minmax", "moba_backward_workspace_size", "moba_backward",
-           "moba_forward_host_buffer_size", "moba_forward_host")
+           "moba_forward_host_buffer_size", "moba_forward_host",
+           "moba_static_selection_varlen", "moba_gate_minmax_varlen",
+           "moba_forward_selected_varlen", "moba_forward_minmax_varlen",
+           "moba_backward_workspace_size_varlen", "moba_backward_varlen")
 
 ROUTE_WINDOW, ROUTE_SINK = 0, 1
 
@@ -130,6 +133,21 @@ def load_library(path=None):
     lib.moba_backward_workspace_size.argtypes = [pp, i32]
     lib.moba_backward.restype = i32
     lib.moba_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, pp, vp, sz, vp]
+    lib.moba_static_selection_varlen.restype = i32
+    lib.moba_static_selection_varlen.argtypes = [vp, i32, vp, i32, i64, pp, vp]
+    lib.moba_gate_minmax_varlen.restype = i32
+    lib.moba_gate_minmax_varlen.argtypes = [vp, vp, vp, i32, i64, vp, pp, vp, sz, vp]
+    lib.moba_forward_selected_varlen.restype = i32
+    lib.moba_forward_selected_varlen.argtypes = [vp, vp, vp, vp, i32, i64, vp, vp, vp, pp, vp,
+                                                 sz, vp]
+    lib.moba_forward_minmax_varlen.restype = i32
+    lib.moba_forward_minmax_varlen.argtypes = [vp, vp, vp, vp, i32, i64, vp, vp, vp, pp, vp,
+                                               sz, vp]
+    lib.moba_backward_workspace_size_varlen.restype = sz
+    lib.moba_backward_workspace_size_varlen.argtypes = [pp, i64, i32, i32]
+    lib.moba_backward_varlen.restype = i32
+    lib.moba_backward_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp,
+                                         pp, vp, sz, vp]
     dp = ctypes.POINTER(MobaDecodeParams)
     lib.moba_decode_workspace_size.restype = sz
     lib.moba_decode_workspace_size.argtypes = [dp]
@@ -476,6 +494,109 @@ def forward_minmax(q, k, v, block_size, top_k, softmax_scale=0.0, ws=None, out=N
                                               ws.numel(), _stream(stream)),
            "moba_forward_minmax")
     return out, lse
+
+
+def static_selection_varlen(cu_seqlens, total_tokens, Hq, block_size, top_k, mode, sel=None,
+                            stream=None):
+    """Window / sink selection sel [Hq, T, top_k] for packed sequences."""
+    torch = _torch()
+    nseq = cu_seqlens.numel() - 1
+    p = make_params(1, 0, Hq, Hq, 128, block_size, top_k)
+    if sel is None:
+        sel = torch.empty(Hq, total_tokens, top_k, dtype=torch.int32, device=cu_seqlens.device)
+    _check(load_library().moba_static_selection_varlen(_ptr(sel), int(mode), _ptr(cu_seqlens),
+                                                       nseq, int(total_tokens), ctypes.byref(p),
+                                                       _stream(stream)),
+           "moba_static_selection_varlen")
+    return sel
+
+
+def _varlen_common(q, k, v, cu_seqlens, block_size, top_k, softmax_scale, ws, out, lse):
+    torch = _torch()
+    _require_cuda_bf16(q, k, v)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    nseq = cu_seqlens.numel() - 1
+    p = make_params(1, 0, Hq, Hkv, d, block_size, top_k, softmax_scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(Hq, T, dtype=torch.float32, device=q.device)
+    if ws is None:
+        hp = pick_heads_per_pass(lambda n: workspace_size_varlen(p, T, nseq, n), Hkv)
+        ws = alloc_workspace(workspace_size_varlen(p, T, nseq, hp), q.device)
+    return p, nseq, T, out, lse, ws
+
+
+def gate_minmax_varlen(q, k, cu_seqlens, block_size, top_k, softmax_scale=0.0, ws=None,
+                       sel=None, stream=None):
+    """Min/max-pooled gate on packed sequences: sel [Hq, T, top_k]."""
+    torch = _torch()
+    _require_cuda_bf16(q, k)
+    T, Hq, d = q.shape
+    nseq = cu_seqlens.numel() - 1
+    p = make_params(1, 0, Hq, k.shape[1], d, block_size, top_k, softmax_scale)
+    if sel is None:
+        sel = torch.empty(Hq, T, top_k, dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(workspace_size_varlen(p, T, nseq, 1), q.device)
+    _check(load_library().moba_gate_minmax_varlen(_ptr(q), _ptr(k), _ptr(cu_seqlens), nseq, T,
+                                                  _ptr(sel), ctypes.byref(p), _ptr(ws),
+                                                  ws.numel(), _stream(stream)),
+           "moba_gate_minmax_varlen")
+    return sel
+
+
+def forward_selected_varlen(q, k, v, cu_seqlens, sel, block_size, top_k, softmax_scale=0.0,
+                            ws=None, out=None, lse=None, stream=None):
+    """Forward over a given selection sel [Hq, T, top_k] on packed sequences: (o, lse)."""
+    p, nseq, T, out, lse, ws = _varlen_common(q, k, v, cu_seqlens, block_size, top_k,
+                                              softmax_scale, ws, out, lse)
+    _check(load_library().moba_forward_selected_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, _ptr(out), _ptr(lse), _ptr(sel),
+        ctypes.byref(p), _ptr(ws), ws.numel(), _stream(stream)), "moba_forward_selected_varlen")
+    return out, lse
+
+
+def forward_minmax_varlen(q, k, v, cu_seqlens, block_size, top_k, softmax_scale=0.0, ws=None,
+                          out=None, lse=None, sel_out=None, stream=None):
+    """Min/max-gate forward on packed sequences: (o, lse [Hq, T])."""
+    p, nseq, T, out, lse, ws = _varlen_common(q, k, v, cu_seqlens, block_size, top_k,
+                                              softmax_scale, ws, out, lse)
+    _check(load_library().moba_forward_minmax_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, _ptr(out), _ptr(lse),
+        _ptr(sel_out), ctypes.byref(p), _ptr(ws), ws.numel(), _stream(stream)),
+        "moba_forward_minmax_varlen")
+    return out, lse
+
+
+# ---------------------------------------------------------------- backward
+def backward_workspace_size_varlen(params, total_tokens, num_seqs, heads_per_pass=0):
+    return int(load_library().moba_backward_workspace_size_varlen(
+        ctypes.byref(params), int(total_tokens), int(num_seqs), int(heads_per_pass)))
+
+
+def backward_varlen(q, k, v, o, lse, dO, sel, cu_seqlens, block_size, top_k, softmax_scale=0.0,
+                    ws=None, dq=None, dk=None, dv=None, stream=None):
+    """Gradients (dq, dk, dv) for packed sequences: q, o, dO [T, Hq, d], k, v
+    [T, Hkv, d], lse [Hq, T] and sel [Hq, T, top_k] as forward_varlen wrote them."""
+    torch = _torch()
+    _require_cuda_bf16(q, k, v, o, dO)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    nseq = cu_seqlens.numel() - 1
+    p = make_params(1, 0, Hq, Hkv, d, block_size, top_k, softmax_scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if ws is None:
+        hp = pick_heads_per_pass(lambda n: backward_workspace_size_varlen(p, T, nseq, n), Hkv)
+        ws = alloc_workspace(backward_workspace_size_varlen(p, T, nseq, hp), q.device)
+    _check(load_library().moba_backward_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(sel), _ptr(cu_seqlens),
+        nseq, T, _ptr(dq), _ptr(dk), _ptr(dv), ctypes.byref(p), _ptr(ws), ws.numel(),
+        _stream(stream)), "moba_backward_varlen")
+    return dq, dk, dv
 
 
 # ---------------------------------------------------------------- backward

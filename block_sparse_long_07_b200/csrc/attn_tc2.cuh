@@ -43,6 +43,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "aux_kernels.cuh"
 #include "common.cuh"
 #include "layout.cuh"
 
@@ -67,15 +68,19 @@ struct AttnArgs {
   float* own_lse;            // [nu][T][G]
   __nv_bfloat16* o;          // [T][Hq][D]
   float* lse;
-  uint32_t* status;
+  uint32_t* status;  // status[1]: largest |v| magnitude (vbound_kernel)
 };
 
-template <int D>
+// QB = Q buffers.  Long items (a block of 8 or more KV tiles, and the dense
+// kernel) take one Q buffer and a deep K/V ring: the ring runs a full KV step
+// ahead so that each TMA load has an MMA iteration to land in, and refilling
+// Q once per item costs little.  Short items (blocks of up to 1024 keys) take
+// two Q buffers, so the next item's rows are gathered (or loaded) while this
+// item computes; for d = 128 that leaves room for three ring slots.
+template <int D, int QB>
 struct Attn2Cfg {
-  // One Q buffer and a deep K/V ring: the ring must run a full KV step ahead
-  // so that each TMA load has an MMA iteration to land in.
-  static constexpr int kQBufs = 1;
-  static constexpr int kStages = (D == 128) ? 5 : 8;
+  static constexpr int kQBufs = QB;
+  static constexpr int kStages = (D == 64) ? 8 : (QB == 2 ? 3 : 5);
   static constexpr int kHalfBytes = kTileM * 128;          // 128 rows x 64 columns bf16
   static constexpr int kSubQBytes = kTileM * D * 2;        // one 128-row Q sub-tile
   static constexpr int kQBytes = 2 * kSubQBytes;           // one work item's Q
@@ -295,11 +300,11 @@ __device__ __forceinline__ float tile_exp_to_p(uint32_t tS, int r, float scale_l
   return ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
 }
 
-template <int D, int MODE>
+template <int D, int MODE, int QBUFS>
 __global__ void __launch_bounds__(352, 1)
     attn2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const AttnArgs a, int pair_own) {
-  using C = Attn2Cfg<D>;
+  using C = Attn2Cfg<D, QBUFS>;
   constexpr int ST = C::kStages;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -486,6 +491,17 @@ __global__ void __launch_bounds__(352, 1)
                        sdesc_mnmajor_sw128(vbase + kk * 2048, C::kHalfBytes, 1024), C::kIdescPV,
                        (acc || kk > 0) ? 1u : 0u);
     };
+    // K_{j+1}: its slot and ring position are assigned in order when step j
+    // starts; the wait happens only before the first S MMA that reads it, so
+    // PV_0(j) never waits on the next K tile's load (with a shallow ring
+    // that load starts only when PV(j-1) frees a slot).
+    uint32_t k_pos = 0;
+    bool k_pending = false;
+    auto ensure_k = [&]() -> bool {
+      if (!k_pending) return true;
+      k_pending = false;
+      return wait(&kv_full[k_pos % ST], (k_pos / ST) & 1);
+    };
     // one sub-tile's share of KV step j: PV_X(j), then S_X(j+1)
     auto kv_step = [&](int x, const Item& it, int j, uint32_t vs, uint32_t ks2, uint32_t qbase) {
       if (j >= it.nkv_x[x]) return true;
@@ -511,7 +527,11 @@ __global__ void __launch_bounds__(352, 1)
         tc_commit_warp(&o_full[x]);
         if (x == 0) ++no0; else ++no1;
       }
-      if (j + 1 < it.nkv_x[x]) issue_s(x, qbase, ks2);
+      if (j + 1 < it.nkv_x[x]) {
+        if (!ensure_k()) return false;
+        tc_fence_after();
+        issue_s(x, qbase, ks2);
+      }
       return true;
     };
     for (int64_t w = first; w < items && ok; w += step, ++lt) {
@@ -534,11 +554,14 @@ __global__ void __launch_bounds__(352, 1)
         uint32_t ks2 = 0;
         if (more) {
           ks2 = kv_it % ST;
-          if (!(ok = wait(&kv_full[ks2], (kv_it / ST) & 1))) break;
+          k_pos = kv_it;
+          k_pending = true;
           ++kv_it;
         }
         if (!(ok = kv_step(0, it, j, vs, ks2, qbase))) break;
         if (!(ok = kv_step(1, it, j, vs, ks2, qbase))) break;
+        // a slot is released only after its load has been waited for
+        if (!(ok = ensure_k())) break;
         tc_commit_warp(&kv_empty[vs]);
         if (more) tc_commit_warp(&kv_empty[ks2]);
       }
@@ -553,6 +576,8 @@ __global__ void __launch_bounds__(352, 1)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::col_s(x);
     const uint32_t tO = tmem + lane_off + C::col_o(x);
+    // routed partials are stored times 2^-S (see partial_scale_log2)
+    const float pscale = (MODE == kRouted) ? exp2f(-(float)partial_scale_log2(a.status[1])) : 1.f;
     uint32_t ns = 0, no = 0;
     bool ok = true;
     for (int64_t w = first; w < items && ok; w += step) {
@@ -662,16 +687,17 @@ __global__ void __launch_bounds__(352, 1)
         } else if (kind == 1) {
           // Routed partial O in fp16: a convex combination of V rows, so
           // |O| <= max |v|; 8x finer than bf16, for the second rounding
-          // the merge adds before the final bf16 output.  A value beyond
-          // the fp16 range is stored as inf, which the merge reports.
+          // the merge adds before the final bf16 output.  Scaled by 2^-S,
+          // which keeps it below the fp16 maximum whatever the bf16 input.
           uint4* d4 = reinterpret_cast<uint4*>(dsth + c4 * 32);
+          const float ps = inv * pscale;
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
             const float* f = reinterpret_cast<const float*>(&ov[q8 * 8]);
-            d4[q8] = make_uint4(pack_half2(f[0] * inv, f[1] * inv),
-                                pack_half2(f[2] * inv, f[3] * inv),
-                                pack_half2(f[4] * inv, f[5] * inv),
-                                pack_half2(f[6] * inv, f[7] * inv));
+            d4[q8] = make_uint4(pack_half2(f[0] * ps, f[1] * ps),
+                                pack_half2(f[2] * ps, f[3] * ps),
+                                pack_half2(f[4] * ps, f[5] * ps),
+                                pack_half2(f[6] * ps, f[7] * ps));
           }
         } else if (kind == 2) {
           float4* d4 = reinterpret_cast<float4*>(dst32 + c4 * 32);

@@ -30,6 +30,7 @@ __global__ void plan_kernel(SeqLayout L, int B, Plan P, int NBmax, int NQTmax,
   __shared__ int32_t sb[1024], sq[1024], sp[1024];
   const int tid = threadIdx.x, nt = blockDim.x;
   if (tid == 0) {
+    status[1] = 0u;  // the largest |v| seen by vbound_kernel (see there)
     carry_b = 0;
     carry_q = 0;
     carry_p = 0;
@@ -164,6 +165,72 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   }
 }
 
+// ------------------------------------------------------------------- |v| bound
+// The routed partial outputs are stored in fp16 (see the attention
+// epilogue).  A partial is a convex combination of its block's v rows, so
+// its magnitude is below the largest |v|.  This kernel takes the largest
+// |v| magnitude, as its bf16 bit pattern without the sign (integer order of
+// those patterns is the order of the magnitudes; NaN sorts above inf), over
+// every block of kv heads g0 .. g0 + gridDim.y - 1 into *vmag (atomic max;
+// the plan kernel zeroes it).  From it the attention and the merge derive
+// one power-of-two scale for the partials (partial_scale_log2), so that no
+// valid bf16 input overflows fp16.  Grid (NBmax, heads), 256 threads,
+// 16-byte loads.
+template <int D>
+__global__ void __launch_bounds__(256) vbound_kernel(const __nv_bfloat16* __restrict__ v,
+                                                     int Hkv, Plan P, uint32_t* __restrict__ vmag,
+                                                     int g0 = 0) {
+  constexpr int CH = D / 8;
+  constexpr int RPI = 256 / CH;
+  const int J = blockIdx.x, g = g0 + blockIdx.y;
+  if (J >= P.totals[0]) return;
+  const int64_t t0 = P.blk_tok[J];
+  const int len = P.blk_len[J];
+  const int c = threadIdx.x % CH, rs = threadIdx.x / CH;
+  const uint4* base = reinterpret_cast<const uint4*>(v + ((size_t)t0 * Hkv + g) * D) + c;
+  const size_t rstride = (size_t)Hkv * D / 8;
+  uint32_t mx = 0u;  // two 16-bit magnitudes, packed
+  int r = rs;
+  for (; r + 3 * RPI < len; r += 4 * RPI) {
+    uint4 x[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = __ldg(base + (size_t)(r + u * RPI) * rstride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      mx = __vmaxu2(__vmaxu2(mx, x[u].x & 0x7fff7fffu),
+                    __vmaxu2(__vmaxu2(x[u].y & 0x7fff7fffu, x[u].z & 0x7fff7fffu),
+                             x[u].w & 0x7fff7fffu));
+  }
+  for (; r < len; r += RPI) {
+    const uint4 x = __ldg(base + (size_t)r * rstride);
+    mx = __vmaxu2(__vmaxu2(mx, x.x & 0x7fff7fffu),
+                  __vmaxu2(__vmaxu2(x.y & 0x7fff7fffu, x.z & 0x7fff7fffu), x.w & 0x7fff7fffu));
+  }
+  uint32_t m = max(mx & 0xffffu, mx >> 16);
+  m = __reduce_max_sync(0xffffffffu, m);
+  __shared__ uint32_t wm[8];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = wm[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) b = max(b, wm[w]);
+    if (b) atomicMax(vmag, b);
+  }
+}
+
+// log2 of the factor the routed partials are multiplied by before their fp16
+// store (and divided by again in the merge): 0 while every |v| < 2^15, else
+// just enough that a partial, at most max|v| (1 + 2^-8) with the bf16
+// rounding of the weights, stays below 2^15 * 1.004 < 65504.  The magnitude
+// is a bf16 pattern: exponent field e means |v| < 2^(e - 126).  Inf or NaN
+// inputs give 0 (their rows come out non-finite and the merge reports them).
+__device__ __forceinline__ int partial_scale_log2(uint32_t vmag) {
+  if (vmag >= 0x7f80u) return 0;
+  const int e = (int)(vmag >> 7);
+  return e > 141 ? e - 141 : 0;
+}
+
 // ------------------------------------------------------------------- gate
 // One CTA per (query tile, query head), one thread per query row.
 // Scores s_j = <q, Kbar_j> for the past blocks j < i (fp32), top-(k-1) by
@@ -178,7 +245,8 @@ template <int D, int KM>
 __global__ void __launch_bounds__(128) gate_kernel(
     const __nv_bfloat16* __restrict__ q, int Hq, int G, int B, int topk, SeqLayout L, Plan P,
     int NBmax, const float* __restrict__ kbar, int32_t* __restrict__ sel, RowLayout R,
-    uint32_t* __restrict__ count_out, uint32_t* __restrict__ status, int h0 = 0) {
+    uint32_t* __restrict__ count_out, uint32_t* __restrict__ status, int h0 = 0,
+    int min_past = -1) {
   extern __shared__ __align__(16) unsigned char gate_smem[];
   float* kb = reinterpret_cast<float*>(gate_smem);                             // [chunk][D]
   uint32_t* cnt = reinterpret_cast<uint32_t*>(kb + kGateChunk * D);           // [blocks]
@@ -188,6 +256,9 @@ __global__ void __launch_bounds__(128) gate_kernel(
   const int64_t st = seq_start(L, s), len = seq_len(L, s);
   const int64_t p0 = (int64_t)(qt - P.qt_off[s]) * kTileM;
   const int i = (int)(p0 / B);  // own block of every row in the tile
+  // as the tensor-core gate's companion (min_past >= 0): only tiles with
+  // more than min_past past blocks are this kernel's (uniform over the CTA)
+  if (i <= min_past) return;
   const int r = threadIdx.x;
   const int64_t pos = p0 + r;
   const bool valid = pos < len;
@@ -462,16 +533,17 @@ __global__ void __launch_bounds__(128) bucket_scatter_kernel(
 // four slots are loaded before any is used.  Rows whose selection is the own
 // block alone were finished by the own-block kernel and are skipped.  The
 // own-block partial is combined first, then the routed slots in ascending
-// order.  A routed partial beyond the fp16 range (a value of 65520 or more,
-// possible only where the block's |v| exceeds it) was stored as inf; the
-// merged row is then not finite and the status word records
-// MOBA_DEV_CAPACITY.
+// order.  The routed partials were stored multiplied by 2^-S (S from
+// partial_scale_log2, 0 unless some |v| reaches 2^15); their weights carry
+// the 2^S back.  A merged row that is not finite (non-finite inputs) is
+// reported in the status word as MOBA_DEV_CAPACITY.
 template <int D>
 __global__ void __launch_bounds__(256) merge_kernel(
     const __half* __restrict__ part_O, const float* __restrict__ part_lse,
     const float* __restrict__ own_O, const float* __restrict__ own_lse, int topk, int B, int G,
     int Hq, int u0, int nu, SeqLayout L, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
     RowLayout R, uint32_t* __restrict__ status) {
+  const float unscale = exp2f((float)partial_scale_log2(status[1]));
   constexpr int LPR = D / 8;       // lanes per row
   constexpr int RPW = 32 / LPR;    // rows per warp
   const int lane = threadIdx.x & 31;
@@ -524,12 +596,13 @@ __global__ void __launch_bounds__(256) merge_kernel(
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       den += w[q];
+      const float wo = w[q] * unscale;
       const __half2* h2 = reinterpret_cast<const __half2*>(&v[q]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 f = __half22float2(h2[e]);
-        acc[2 * e] = fmaf(w[q], f.x, acc[2 * e]);
-        acc[2 * e + 1] = fmaf(w[q], f.y, acc[2 * e + 1]);
+        acc[2 * e] = fmaf(wo, f.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(wo, f.y, acc[2 * e + 1]);
       }
     }
   }
@@ -537,12 +610,13 @@ __global__ void __launch_bounds__(256) merge_kernel(
     const uint4 v = orow[sl * kStride];
     const float w = ex2_approx(lrow[sl] - m);
     den += w;
+    const float wo = w * unscale;
     const __half2* h2 = reinterpret_cast<const __half2*>(&v);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 f = __half22float2(h2[e]);
-      acc[2 * e] = fmaf(w, f.x, acc[2 * e]);
-      acc[2 * e + 1] = fmaf(w, f.y, acc[2 * e + 1]);
+      acc[2 * e] = fmaf(wo, f.x, acc[2 * e]);
+      acc[2 * e + 1] = fmaf(wo, f.y, acc[2 * e + 1]);
     }
   }
   bool finite = true;

@@ -50,8 +50,11 @@
 namespace moba {
 
 constexpr int kGateTcMaxPast = 256;  // past blocks one score tile holds (TMEM columns)
-constexpr int kGateTcCap = 24;       // candidate slots per row
-constexpr int kGateTcMaxKeep = 16;   // largest k-1 this kernel ranks
+constexpr int kGateTcMaxKeep = 32;   // largest k-1 this kernel ranks
+// k-1 <= 16: score tiles of up to 256 past blocks, 24 candidate slots per row;
+// 16 < k-1 <= 32: up to 128 past blocks (the block means of 256 would not fit
+// shared memory beside the longer candidate lists), 48 slots.
+constexpr int gate_tc_max_past(int KM) { return KM <= 16 ? 256 : 128; }
 
 struct GateTcArgs {
   const float* kbar;  // [Hkv][NBmax][D] fp32 block means
@@ -61,34 +64,40 @@ struct GateTcArgs {
   RowLayout R;
   int32_t* sel;
   uint32_t* status;
-  int g0, ng;  // kv heads g0 .. g0 + ng - 1 (their items are contiguous)
+  int g0, ng;     // kv heads g0 .. g0 + ng - 1 (their items are contiguous)
+  int companion;  // 1: query tiles with more past blocks than a score tile holds
+                  // are left to the SIMT gate, launched after this kernel
 };
 
-template <int D>
+template <int D, int KM>
 struct GateTcCfg {
+  static constexpr int kMaxPast = gate_tc_max_past(KM);
+  static constexpr int kCap = KM <= 16 ? 24 : 48;           // candidate slots per row
   static constexpr int kQHalf = kTileM * 128;               // 128 rows x 64 columns bf16
   static constexpr int kQBytes = kTileM * D * 2;
-  static constexpr int kKbHalf = kGateTcMaxPast * 128;      // 256 rows x 64 columns bf16
-  static constexpr int kKbBytes = kGateTcMaxPast * D * 2;   // one part (hi or lo)
+  static constexpr int kKbHalf = kMaxPast * 128;            // kMaxPast rows x 64 columns bf16
+  static constexpr int kKbBytes = kMaxPast * D * 2;         // one part (hi or lo)
   static constexpr int kOffQ = 0;
   static constexpr int kOffKb = kOffQ + 2 * kQBytes;
   static constexpr int kOffCv = kOffKb + 2 * kKbBytes;                  // float [2][cap][128]
-  static constexpr int kOffCi = kOffCv + 2 * kGateTcCap * kTileM * 4;   // uint8 [2][cap][128]
-  static constexpr int kOffBar = kOffCi + 2 * kGateTcCap * kTileM;
+  static constexpr int kOffCi = kOffCv + 2 * kCap * kTileM * 4;         // uint8 [2][cap][128]
+  static constexpr int kOffBar = kOffCi + 2 * kCap * kTileM;
   static constexpr int kNumBars = 2 * 6 + 1;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
   static constexpr int kThreads = 352;
   static constexpr uint32_t kTmemCols = 512;  // two 256-column score buffers
+  static_assert(kSmemBytes <= 232448, "gate shared memory beyond the per-CTA limit");
 };
 
 struct GateTcItem {
   int g, h, s, i, rows;
   int64_t st, p0;
   bool direct;  // no scoring: k = 1, or every past block is kept
-  bool bad;     // more past blocks than a score tile holds (refused on the host)
+  bool bad;     // more past blocks than a score tile holds (the SIMT gate's)
 };
 
-__device__ __forceinline__ GateTcItem gate_tc_item(const GateTcArgs& a, int64_t w) {
+__device__ __forceinline__ GateTcItem gate_tc_item(const GateTcArgs& a, int64_t w,
+                                                   int max_past) {
   GateTcItem it;
   const int NQT = a.P.totals[1];
   const int64_t per_g = (int64_t)NQT * a.G;
@@ -103,7 +112,7 @@ __device__ __forceinline__ GateTcItem gate_tc_item(const GateTcArgs& a, int64_t 
   it.rows = (int)min((int64_t)kTileM, seq_len(a.L, it.s) - it.p0);
   const int npast = a.topk - 1;
   it.direct = (npast == 0) || (it.i <= npast);
-  it.bad = !it.direct && it.i > kGateTcMaxPast;
+  it.bad = !it.direct && it.i > max_past;
   return it;
 }
 
@@ -152,7 +161,8 @@ __device__ __forceinline__ void load_scores(uint32_t taddr, int c, int ncol, flo
 template <int D, int KM>
 __global__ void __launch_bounds__(352, 1)
     gate_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const GateTcArgs a) {
-  using C = GateTcCfg<D>;
+  using C = GateTcCfg<D, KM>;
+  constexpr int kCap = C::kCap;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -205,7 +215,7 @@ __global__ void __launch_bounds__(352, 1)
       uint32_t n = 0;
       bool ok = true;
       for (int64_t w = first; w < items && ok; w += step) {
-        const GateTcItem it = gate_tc_item(a, w);
+        const GateTcItem it = gate_tc_item(a, w, C::kMaxPast);
         if (it.direct || it.bad) continue;
         const int b = n & 1;
         ok = mbar_wait(&q_empty[b], ((n >> 1) & 1) ^ 1, abort_flag, st);
@@ -235,7 +245,7 @@ __global__ void __launch_bounds__(352, 1)
     int cur_s = -1, cur_g = -1, loaded = 0;
     bool ok = true;
     for (int64_t w = first; w < items && ok; w += step) {
-      const GateTcItem it = gate_tc_item(a, w);
+      const GateTcItem it = gate_tc_item(a, w, C::kMaxPast);
       if (it.direct || it.bad) continue;
       const int b = n & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&kb_empty[b], ((n >> 1) & 1) ^ 1, abort_flag, st));
@@ -289,7 +299,7 @@ __global__ void __launch_bounds__(352, 1)
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, st));
     };
     for (int64_t w = first; w < items && ok; w += step) {
-      const GateTcItem it = gate_tc_item(a, w);
+      const GateTcItem it = gate_tc_item(a, w, C::kMaxPast);
       if (it.direct || it.bad) continue;
       const int b = n & 1;
       const uint32_t ph = (n >> 1) & 1;
@@ -324,19 +334,19 @@ __global__ void __launch_bounds__(352, 1)
     const int grp = warp >> 2, quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t tS = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)grp * 256;
-    float* cv = cv_all + grp * kGateTcCap * kTileM + r;    // slot q at cv[q * kTileM]
-    uint8_t* ci = ci_all + grp * kGateTcCap * kTileM + r;
+    float* cv = cv_all + grp * kCap * kTileM + r;    // slot q at cv[q * kTileM]
+    uint8_t* ci = ci_all + grp * kCap * kTileM + r;
     uint32_t n = 0, li = 0;
     bool ok = true;
     for (int64_t w = first; w < items && ok; w += step, ++li) {
-      const GateTcItem it = gate_tc_item(a, w);
+      const GateTcItem it = gate_tc_item(a, w, C::kMaxPast);
       const bool valid = r < it.rows;
       const int64_t pos = it.p0 + r;
       int32_t* out = a.sel + row_index(a.R, it.s, it.h, pos, it.st + pos) * a.topk;
       if (it.direct || it.bad) {
         if ((int)(li & 1) != grp) continue;
         if (it.bad) {
-          if (r == 0) atomicOr(st, MOBA_DEV_CAPACITY);
+          if (r == 0 && !a.companion) atomicOr(st, MOBA_DEV_CAPACITY);
           continue;
         }
         if (valid) {
@@ -380,7 +390,7 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const bool take = v[e] >= T0;
-          const int slot = min(nc, kGateTcCap - 1);
+          const int slot = min(nc, kCap - 1);
           if (take) {
             cv[slot * kTileM] = v[e];
             ci[slot * kTileM] = (uint8_t)(c + e);
@@ -389,7 +399,7 @@ __global__ void __launch_bounds__(352, 1)
         }
       }
       if (!valid) nc = 0;
-      const bool overflow = nc > kGateTcCap;
+      const bool overflow = nc > kCap;
       // ---- rare fallback: rank the whole row with an insertion list
       int32_t fb[KM];
       if (__any_sync(0xffffffffu, overflow)) {

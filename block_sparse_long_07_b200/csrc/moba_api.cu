@@ -39,13 +39,13 @@ namespace {
 enum KernelClass {
   kKPlan, kKPool, kKGate, kKGateCount, kKScan, kKScatter, kKRouted, kKOwn, kKMerge, kKDense,
   kKKbarCache, kKDecGate, kKDecAttn, kKDecMerge, kKMinmaxPool, kKGateMinmax, kKStaticSel,
-  kKBwPrep, kKBwKv, kKBwQ, kKBwFinish, kKNum
+  kKBwPrep, kKBwKv, kKBwQ, kKBwFinish, kKVbound, kKNum
 };
 const char* const kKernelNames[kKNum] = {
     "plan",        "pool",        "gate",         "gate_count",  "bucket_scan",
     "bucket_scatter", "attn_routed", "attn_own",  "merge",       "attn_dense",
     "kbar_cache",  "decode_gate", "decode_attn",  "decode_merge", "minmax_pool",
-    "gate_minmax", "static_select", "bw_prep", "bw_kv", "bw_q", "bw_finish"};
+    "gate_minmax", "static_select", "bw_prep", "bw_kv", "bw_q", "bw_finish", "vbound"};
 struct TimedLaunch {
   int cls;
   cudaEvent_t a, b;
@@ -286,11 +286,11 @@ int num_sms() {
   return n;
 }
 
-template <int D, int MODE>
-moba_status launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const AttnArgs& a, int pair_own, cudaStream_t stream) {
-  using C = Attn2Cfg<D>;
-  auto kern = attn2_kernel<D, MODE>;
+template <int D, int MODE, int QB>
+moba_status launch_attn_qb(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const AttnArgs& a, int pair_own, cudaStream_t stream) {
+  using C = Attn2Cfg<D, QB>;
+  auto kern = attn2_kernel<D, MODE, QB>;
   MOBA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmemBytes));
   const int grid = num_sms();
@@ -300,9 +300,23 @@ moba_status launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
   return cuda_status(cudaGetLastError());
 }
 
+// Routed and own-block items over blocks of up to kShortBlock keys are short
+// (at most 8 KV tiles): they take two Q buffers so the next item's rows load
+// during this one.  Longer blocks and the dense kernel take one.
+constexpr int kShortBlock = 1024;
+
+template <int D, int MODE>
+moba_status launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const AttnArgs& a, int pair_own, cudaStream_t stream) {
+  if (MODE != kDense && a.B <= kShortBlock)
+    return launch_attn_qb<D, MODE == kDense ? kOwn : MODE, 2>(tq, tk, tv, a, pair_own, stream);
+  return launch_attn_qb<D, MODE, 1>(tq, tk, tv, a, pair_own, stream);
+}
+
 template <int D, int KM>
 moba_status launch_gate_km(const Problem& pr, const void* q, const Ws& w, int32_t* sel,
-                           uint32_t* counts, cudaStream_t st, int g0, int ng) {
+                           uint32_t* counts, cudaStream_t st, int g0, int ng,
+                           int min_past = -1) {
   const size_t smem = sizeof(float) * kGateChunk * D + sizeof(uint32_t) * kMaxBlocksPerSeq;
   auto kern = gate_kernel<D, KM>;
   if (smem > 48 * 1024)
@@ -312,7 +326,7 @@ moba_status launch_gate_km(const Problem& pr, const void* q, const Ws& w, int32_
   Timed tm(kKGate, st);
   kern<<<grid, 128, smem, st>>>(reinterpret_cast<const __nv_bfloat16*>(q), pr.Hq, pr.G, pr.B,
                                 pr.topk, L, w.P, (int)pr.NBmax, w.kbar, sel, pr.R, counts,
-                                w.status, g0 * pr.G);
+                                w.status, g0 * pr.G, min_past);
   return cuda_status(cudaGetLastError());
 }
 
@@ -321,7 +335,7 @@ moba_status launch_gate_km(const Problem& pr, const void* q, const Ws& w, int32_
 template <int D, int KM>
 moba_status launch_gate_tc_km(const Problem& pr, const void* q, const Ws& w, int32_t* sel,
                               uint32_t* counts, cudaStream_t st, int g0, int ng) {
-  using C = GateTcCfg<D>;
+  using C = GateTcCfg<D, KM>;
   CUtensorMap tq;
   if (!make_tmap(&tq, q, pr.Hq, pr.T, D)) return MOBA_ERR_CUDA;
   auto kern = gate_tc_kernel<D, KM>;
@@ -344,11 +358,17 @@ moba_status launch_gate_tc_km(const Problem& pr, const void* q, const Ws& w, int
   a.status = w.status;
   a.g0 = g0;
   a.ng = ng;
+  // sequences longer than a score tile covers: their later query tiles go to
+  // the SIMT gate (only those tiles; the others return at once)
+  a.companion = pr.max_blocks_per_seq - 1 > C::kMaxPast ? 1 : 0;
   {
     Timed tm(kKGate, st);
     kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, a);
     MOBA_CUDA(cudaGetLastError());
   }
+  if (a.companion)
+    MOBA_TRY((launch_gate_km<D, (KM <= 16 ? 16 : KM)>(pr, q, w, sel, nullptr, st, g0, ng,
+                                                        C::kMaxPast)));
   if (counts) {
     const size_t smem = sizeof(uint32_t) * kMaxBlocksPerSeq;
     dim3 cgrid((unsigned)pr.NQTmax, (unsigned)ng);
@@ -360,11 +380,12 @@ moba_status launch_gate_tc_km(const Problem& pr, const void* q, const Ws& w, int
   return MOBA_OK;
 }
 
-// The tensor-core gate ranks up to 16 past blocks out of at most 256 per sequence.
+// The tensor-core gate ranks up to 32 past blocks; query tiles with more past
+// blocks than its score tile holds (256, or 128 when k-1 > 16) are handed to
+// the SIMT gate.
 bool gate_tc_fits(const Problem& pr) {
   const int64_t npast = pr.topk - 1;
-  return npast >= 1 && npast <= kGateTcMaxKeep && npast < pr.max_blocks_per_seq - 1 &&
-         pr.max_blocks_per_seq - 1 <= kGateTcMaxPast;
+  return npast >= 1 && npast <= kGateTcMaxKeep && npast < pr.max_blocks_per_seq - 1;
 }
 
 // The gate for the q heads of kv heads g0 .. g0 + ng - 1 (default: all).
@@ -379,9 +400,10 @@ moba_status launch_gate(const Problem& pr, const void* q, const Ws& w, int32_t* 
       case 2: return launch_gate_tc_km<D, 2>(pr, q, w, sel, counts, st, g0, ng);
       case 4: return launch_gate_tc_km<D, 4>(pr, q, w, sel, counts, st, g0, ng);
       case 8: return launch_gate_tc_km<D, 8>(pr, q, w, sel, counts, st, g0, ng);
-      default:
+      case 16:
         if (npast <= 12) return launch_gate_tc_km<D, 12>(pr, q, w, sel, counts, st, g0, ng);
         return launch_gate_tc_km<D, 16>(pr, q, w, sel, counts, st, g0, ng);
+      default: return launch_gate_tc_km<D, 32>(pr, q, w, sel, counts, st, g0, ng);
     }
   }
   const int64_t need = (npast >= pr.max_blocks_per_seq - 1) ? 1 : npast;
@@ -450,6 +472,22 @@ moba_status run_pool(const Problem& pr, const void* k, const Ws& w, cudaStream_t
   else
     pool_kernel<64><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(k), pr.Hkv,
                                           w.P, (int)pr.NBmax, w.kbar, g0);
+  return cuda_status(cudaGetLastError());
+}
+
+// Largest |v| of kv heads g0 .. g0 + ng - 1 into status[1] (the routed
+// partials' scale; see vbound_kernel).
+moba_status run_vbound(const Problem& pr, const void* v, const Ws& w, cudaStream_t st, int g0,
+                       int ng) {
+  if (pr.topk <= 1) return MOBA_OK;  // no routed partials
+  dim3 grid((unsigned)pr.NBmax, (unsigned)ng);
+  Timed tm(kKVbound, st);
+  if (pr.D == 128)
+    vbound_kernel<128><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(v), pr.Hkv,
+                                             w.P, w.status + 1, g0);
+  else
+    vbound_kernel<64><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(v), pr.Hkv,
+                                            w.P, w.status + 1, g0);
   return cuda_status(cudaGetLastError());
 }
 
@@ -747,6 +785,7 @@ moba_status forward_host_passes(const Problem& pr, const void* q_h, const void* 
     const int g0 = p * nu_max, ng = (pr.Hkv - g0) < nu_max ? (pr.Hkv - g0) : nu_max;
     if (cudaStreamWaitEvent(st, in_ready(p), 0) != cudaSuccess) return fail(MOBA_ERR_CUDA);
     if ((r = run_pool(pr, hb.k, w, st, g0, ng)) != MOBA_OK) return fail(r);
+    if ((r = run_vbound(pr, hb.v, w, st, g0, ng)) != MOBA_OK) return fail(r);
     if ((r = launch_gate<D>(pr, hb.q, w, hb.sel, w.counts, st, g0, ng)) != MOBA_OK) return fail(r);
     if ((r = forward_one_pass<D>(pr, c, w, hb.sel, hb.o, hb.lse, g0, ng, st)) != MOBA_OK)
       return fail(r);
@@ -798,6 +837,7 @@ moba_status forward_impl(const Problem& pr, const void* q, const void* k, const 
   } else {
     MOBA_TRY(run_plan(pr, w, st));
   }
+  MOBA_TRY(run_vbound(pr, v, w, st, 0, pr.Hkv));
   return pr.D == 128 ? forward_passes<128>(pr, q, k, v, o, lse, w, sel, nu, route, st)
                      : forward_passes<64>(pr, q, k, v, o, lse, w, sel, nu, route, st);
 }
@@ -1339,10 +1379,27 @@ int moba_profile_read(moba_kernel_time* out, int max_entries) {
 }
 
 // ---------------------------------------------------------------- routing variants
+moba_status gate_minmax_impl(const Problem& pr, const void* q, const void* k, int32_t* sel,
+                             void* ws, size_t ws_bytes, moba_stream_t stream);
+
 moba_status moba_gate_minmax(const void* q, const void* k, int32_t* sel, const moba_params* p,
                              void* ws, size_t ws_bytes, moba_stream_t stream) {
   Problem pr;
   MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  return gate_minmax_impl(pr, q, k, sel, ws, ws_bytes, stream);
+}
+
+moba_status moba_gate_minmax_varlen(const void* q, const void* k, const int32_t* cu_seqlens,
+                                    int num_seqs, int64_t total_tokens, int32_t* sel,
+                                    const moba_params* p, void* ws, size_t ws_bytes,
+                                    moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, true, cu_seqlens, num_seqs, total_tokens, true, &pr));
+  return gate_minmax_impl(pr, q, k, sel, ws, ws_bytes, stream);
+}
+
+moba_status gate_minmax_impl(const Problem& pr, const void* q, const void* k, int32_t* sel,
+                             void* ws, size_t ws_bytes, moba_stream_t stream) {
   if (!q || !k || !sel || !aligned16(q) || !aligned16(k) ||
       (reinterpret_cast<uintptr_t>(sel) & 3))
     return MOBA_ERR_INVALID_ARG;
@@ -1357,19 +1414,32 @@ moba_status moba_gate_minmax(const void* q, const void* k, int32_t* sel, const m
                      : launch_gate_minmax<64>(pr, q, w, sel, nullptr, st);
 }
 
+moba_status static_selection_impl(const Problem& pr, int32_t* sel, int mode,
+                                  cudaStream_t st) {
+  if (!sel || (reinterpret_cast<uintptr_t>(sel) & 3)) return MOBA_ERR_INVALID_ARG;
+  if (mode != MOBA_ROUTE_WINDOW && mode != MOBA_ROUTE_SINK) return MOBA_ERR_INVALID_ARG;
+  const int64_t rows = pr.T * pr.Hq;
+  if (rows == 0) return MOBA_OK;
+  SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
+  Timed tm(kKStaticSel, st);
+  static_select_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(
+      sel, rows, L, pr.Hq, pr.B, pr.topk, mode == MOBA_ROUTE_SINK ? kRouteSink : kRouteWindow);
+  return cuda_status(cudaGetLastError());
+}
+
 moba_status moba_static_selection(int32_t* sel, int mode, const moba_params* p,
                                   moba_stream_t stream) {
   Problem pr;
   MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
-  if (!sel || (reinterpret_cast<uintptr_t>(sel) & 3)) return MOBA_ERR_INVALID_ARG;
-  if (mode != MOBA_ROUTE_WINDOW && mode != MOBA_ROUTE_SINK) return MOBA_ERR_INVALID_ARG;
-  const int64_t rows = (int64_t)pr.nseq * pr.Hq * pr.N;
-  if (rows == 0) return MOBA_OK;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  Timed tm(kKStaticSel, st);
-  static_select_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(
-      sel, rows, pr.N, pr.Hq, pr.B, pr.topk, mode == MOBA_ROUTE_SINK ? kRouteSink : kRouteWindow);
-  return cuda_status(cudaGetLastError());
+  return static_selection_impl(pr, sel, mode, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moba_status moba_static_selection_varlen(int32_t* sel, int mode, const int32_t* cu_seqlens,
+                                         int num_seqs, int64_t total_tokens,
+                                         const moba_params* p, moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, true, cu_seqlens, num_seqs, total_tokens, true, &pr));
+  return static_selection_impl(pr, sel, mode, reinterpret_cast<cudaStream_t>(stream));
 }
 
 moba_status moba_forward_selected(const void* q, const void* k, const void* v, void* o,
@@ -1387,6 +1457,29 @@ moba_status moba_forward_minmax(const void* q, const void* k, const void* v, voi
                                 size_t ws_bytes, moba_stream_t stream) {
   Problem pr;
   MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  return forward_impl(pr, q, k, v, o, lse, sel_out, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), kRouteMinmaxGate);
+}
+
+moba_status moba_forward_selected_varlen(const void* q, const void* k, const void* v,
+                                         const int32_t* cu_seqlens, int num_seqs,
+                                         int64_t total_tokens, void* o, float* lse,
+                                         const int32_t* sel, const moba_params* p, void* ws,
+                                         size_t ws_bytes, moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, true, cu_seqlens, num_seqs, total_tokens, true, &pr));
+  if (!sel) return MOBA_ERR_INVALID_ARG;
+  return forward_impl(pr, q, k, v, o, lse, const_cast<int32_t*>(sel), ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), kRouteGiven);
+}
+
+moba_status moba_forward_minmax_varlen(const void* q, const void* k, const void* v,
+                                       const int32_t* cu_seqlens, int num_seqs,
+                                       int64_t total_tokens, void* o, float* lse,
+                                       int32_t* sel_out, const moba_params* p, void* ws,
+                                       size_t ws_bytes, moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, true, cu_seqlens, num_seqs, total_tokens, true, &pr));
   return forward_impl(pr, q, k, v, o, lse, sel_out, ws, ws_bytes,
                       reinterpret_cast<cudaStream_t>(stream), kRouteMinmaxGate);
 }
@@ -1439,6 +1532,26 @@ moba_status moba_backward(const void* q, const void* k, const void* v, const voi
                           moba_stream_t stream) {
   Problem pr;
   MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  return backward_impl(pr, q, k, v, o, lse, dO, sel, dq, dk, dv, ws, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moba_backward_workspace_size_varlen(const moba_params* p, int64_t total_tokens,
+                                           int num_seqs, int heads_per_pass) {
+  Problem pr;
+  static const int32_t dummy = 0;
+  if (make_problem(p, true, &dummy, num_seqs, total_tokens, true, &pr) != MOBA_OK) return 0;
+  int nu = (heads_per_pass <= 0 || heads_per_pass > pr.Hkv) ? pr.Hkv : heads_per_pass;
+  return carve_bw(pr, nu, nullptr).bytes;
+}
+
+moba_status moba_backward_varlen(const void* q, const void* k, const void* v, const void* o,
+                                 const float* lse, const void* dO, const int32_t* sel,
+                                 const int32_t* cu_seqlens, int num_seqs, int64_t total_tokens,
+                                 void* dq, void* dk, void* dv, const moba_params* p, void* ws,
+                                 size_t ws_bytes, moba_stream_t stream) {
+  Problem pr;
+  MOBA_TRY(make_problem(p, true, cu_seqlens, num_seqs, total_tokens, true, &pr));
   return backward_impl(pr, q, k, v, o, lse, dO, sel, dq, dk, dv, ws, ws_bytes,
                        reinterpret_cast<cudaStream_t>(stream));
 }

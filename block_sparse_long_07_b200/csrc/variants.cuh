@@ -247,15 +247,23 @@ __global__ void __launch_bounds__(128) gate_minmax_kernel(
   }
 }
 
-// Window / sink selections for a batch of b sequences of N tokens (batch
-// layout sel [b][Hq][N][k]): the own block i and min(k-1, i) past blocks,
+// Window / sink selections: the own block i and min(k-1, i) past blocks,
 // the most recent ones (window) or block 0 plus the most recent ones (sink).
-__global__ void static_select_kernel(int32_t* __restrict__ sel, int64_t rows, int N, int Hq,
-                                     int B, int topk, int mode) {
-  const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // (b, h, pos)
+// Batch layout sel [b][Hq][N][k] (row x = (b, h, pos)); packed sequences
+// (L.cu set) sel [Hq][T][k] (row x = (h, token)), positions counted from
+// each sequence's start.
+__global__ void static_select_kernel(int32_t* __restrict__ sel, int64_t rows, SeqLayout L,
+                                     int Hq, int B, int topk, int mode) {
+  const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (x >= rows) return;
-  const int pos = (int)(x % N);
-  const int i = pos / B;
+  int64_t pos;
+  if (L.cu) {
+    const int64_t t = x % L.T;
+    pos = t - seq_start(L, seq_of_token(L, t));
+  } else {
+    pos = x % L.N;
+  }
+  const int i = (int)(pos / B);
   const int npast = min(topk - 1, i);
   int32_t* out = sel + x * topk;
   int u = 0;

@@ -184,10 +184,21 @@ moba_status moba_backward(const void *q, const void *k, const void *v, const voi
                           const float *lse, const void *dO, const int32_t *sel, void *dq,
                           void *dk, void *dv, const moba_params *p, void *ws, size_t ws_bytes,
                           moba_stream_t stream);
+/* The backward for packed sequences (cu_seqlens [num_seqs + 1] int32 on the
+ * device, as moba_forward_varlen): q, o, dO, dq [T][Hq][d], k, v, dk, dv
+ * [T][Hkv][d], lse [Hq][T], sel [Hq][T][top_k] as moba_forward_varlen wrote
+ * them; p->batch and p->seqlen are not used.  Workspace:
+ * moba_backward_workspace_size_varlen.  Errors as moba_backward. */
+size_t moba_backward_workspace_size_varlen(const moba_params *p, int64_t total_tokens,
+                                           int num_seqs, int heads_per_pass);
+moba_status moba_backward_varlen(const void *q, const void *k, const void *v, const void *o,
+                                 const float *lse, const void *dO, const int32_t *sel,
+                                 const int32_t *cu_seqlens, int num_seqs, int64_t total_tokens,
+                                 void *dq, void *dk, void *dv, const moba_params *p, void *ws,
+                                 size_t ws_bytes, moba_stream_t stream);
 
 /* ------------------------------------------------------- routing variants
- * The pages present the gate as one member of a family (batch layout only
- * here): sliding-window attention is a gate that always selects the most
+ * The pages present the gate as one member of a family: sliding-window attention is a gate that always selects the most
  * recent blocks, sink attention one that always selects the initial and the
  * most recent blocks (wispaper.ai blog, "Why the Change Is Plausible"), and
  * Quest is MoBA with smaller blocks and min/max pooling (elamur summary
@@ -224,6 +235,31 @@ moba_status moba_forward_selected(const void *q, const void *k, const void *v, v
 moba_status moba_forward_minmax(const void *q, const void *k, const void *v, void *o,
                                 float *lse, int32_t *sel_out, const moba_params *p, void *ws,
                                 size_t ws_bytes, moba_stream_t stream);
+
+/* Packed-sequence forms of the four calls above (cu_seqlens [num_seqs + 1]
+ * int32 on the device; blocks and positions counted from each sequence's
+ * start, as moba_forward_varlen): q, o [T][Hq][d], k, v [T][Hkv][d], lse
+ * [Hq][T], sel [Hq][T][top_k].  Workspace: moba_workspace_size_varlen(p,
+ * total_tokens, num_seqs, 1) for the gate, any heads_per_pass for the
+ * forwards.  Errors as the batch forms; malformed cu_seqlens latch
+ * MOBA_ERR_DEVICE_CHECK. */
+moba_status moba_static_selection_varlen(int32_t *sel, int mode, const int32_t *cu_seqlens,
+                                         int num_seqs, int64_t total_tokens,
+                                         const moba_params *p, moba_stream_t stream);
+moba_status moba_gate_minmax_varlen(const void *q, const void *k, const int32_t *cu_seqlens,
+                                    int num_seqs, int64_t total_tokens, int32_t *sel,
+                                    const moba_params *p, void *ws, size_t ws_bytes,
+                                    moba_stream_t stream);
+moba_status moba_forward_selected_varlen(const void *q, const void *k, const void *v,
+                                         const int32_t *cu_seqlens, int num_seqs,
+                                         int64_t total_tokens, void *o, float *lse,
+                                         const int32_t *sel, const moba_params *p, void *ws,
+                                         size_t ws_bytes, moba_stream_t stream);
+moba_status moba_forward_minmax_varlen(const void *q, const void *k, const void *v,
+                                       const int32_t *cu_seqlens, int num_seqs,
+                                       int64_t total_tokens, void *o, float *lse,
+                                       int32_t *sel_out, const moba_params *p, void *ws,
+                                       size_t ws_bytes, moba_stream_t stream);
 
 /* Dense causal attention over every earlier token of each sequence: the
  * k = n limit of the method (wispaper.ai blog, "The Change": k = n
@@ -310,7 +346,7 @@ moba_status moba_last_device_status(void *ws, moba_stream_t stream);
  * (plan, pool, gate, gate_count, bucket_scan, bucket_scatter, attn_routed,
  * attn_own, merge, attn_dense, kbar_cache, decode_gate, decode_attn,
  * decode_merge, minmax_pool, gate_minmax, static_select, bw_prep, bw_kv,
- * bw_q, bw_finish), the launch count and summed device milliseconds since the
+ * bw_q, bw_finish, vbound), the launch count and summed device milliseconds since the
  * last reset.  Returns the number of classes written (<= max_entries).
  * Not thread safe; meant for one benchmarking thread. */
 typedef struct moba_kernel_time {

@@ -85,8 +85,13 @@ PREFILL_10M_SHARD = Workload("prefill_10m_shard", [10485760], 4, 1, 128, 40960, 
 LONG_128K_H8 = Workload("long_128k_h8", [131072], 8, 2, 128, 4096, 12, seed=2,
                         note="8 q / 2 kv heads, d=128, N=131072, B=4096 (32 blocks), k=12")
 
+# fine_32k's shape with a quarter of the heads (same N, B, k): the small
+# case for multi-pass captures of the short-block kernels.
+FINE_32K_H8 = Workload("fine_32k_h8", [32768], 8, 2, 128, 256, 32, seed=1,
+                       note="8 q / 2 kv heads, d=128, N=32768, B=256 (128 blocks), k=32")
+
 WORKLOADS = {w.name: w for w in (TINY, FINE_32K, LONG_128K, MILLION, VARLEN, PREFILL_10M_SHARD,
-                                 LONG_128K_H8)}
+                                 LONG_128K_H8, FINE_32K_H8)}
 
 
 def block_ids(lengths: List[int], B: int) -> np.ndarray:

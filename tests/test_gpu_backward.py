@@ -84,3 +84,35 @@ def test_backward_is_deterministic_up_to_atomic_order(moba):
     for x, y in zip(a, b):
         # fp32 atomic sums may add in a different order: equal to bf16 rounding
         assert torch.allclose(x.float(), y.float(), rtol=1e-2, atol=1e-3)
+
+
+@pytest.mark.parametrize("lengths,Hq,Hkv,d,B,k", [
+    ([700, 1, 1300, 0, 900], 4, 2, 128, 256, 3),
+    ([1500, 600], 4, 1, 64, 128, 4),
+])
+def test_backward_varlen_matches_oracle(moba, lengths, Hq, Hkv, d, B, k):
+    """The packed-sequence backward: every element of dq, dk, dv against the
+    oracle, over the selection forward_varlen wrote (blocks counted from each
+    sequence's start, no key or row crossing a sequence boundary)."""
+    w = S.Workload("bw_varlen", lengths, Hq, Hkv, d, B, k, seed=1212, batch_mode=False)
+    q, kk, v = S.make_qkv(w, "cuda")
+    cu = torch.tensor(w.cu, dtype=torch.int32, device="cuda")
+    sel = torch.empty(Hq, w.T, k, dtype=torch.int32, device="cuda")
+    o, lse = moba.forward_varlen(q, kk, v, cu, B, k, sel_out=sel)
+    g = torch.Generator(device="cuda").manual_seed(79)
+    dO = torch.randn(w.T, Hq, d, generator=g, device="cuda").to(torch.bfloat16)
+    p = moba.make_params(1, 0, Hq, Hkv, d, B, k)
+    ws = moba.alloc_workspace(moba.backward_workspace_size_varlen(p, w.T, len(lengths), 0))
+    dq, dk, dv = moba.backward_varlen(q, kk, v, o, lse, dO, sel, cu, B, k, ws=ws)
+    torch.cuda.synchronize()
+    assert moba.last_device_status(ws) == 0
+    orc = Oracle(bf16_bits(q), bf16_bits(kk), bf16_bits(v), w.cu, Hq, Hkv, d, B, k)
+    rows = np.arange(w.T, dtype=np.int64)
+    sel_rows = sel.permute(1, 0, 2).contiguous().cpu().numpy()
+    rq, rk, rv = orc.attend_backward(rows, sel_rows, bf16_bits(dO))
+    for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        got = got.float().cpu().numpy().astype(np.float64)
+        scale = np.abs(ref).max()
+        err = np.abs(got - ref)
+        assert err.max() <= MAX_REL * scale, (name, err.max(), scale)
+        assert err.mean() <= MEAN_REL * scale, (name, err.mean(), scale)

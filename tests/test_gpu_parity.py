@@ -87,7 +87,9 @@ SMALL = [
     ([4096], 8, 2, 128, 128, 5),      # many blocks, top-k ranking
     ([32896], 2, 1, 128, 128, 6),     # 257 blocks: 256 past, the tensor-core gate's limit
     ([40000], 2, 1, 64, 128, 8),      # 313 blocks: beyond it, the SIMT gate
-    ([4096], 4, 1, 128, 128, 17),     # k - 1 = 16, the longest list the tensor-core gate ranks
+    ([4096], 4, 1, 128, 128, 17),     # k - 1 = 16: the last of the 256-block score tiles
+    ([16384], 2, 1, 128, 128, 32),    # k - 1 = 31 of up to 127 past blocks (32-long lists)
+    ([20000], 2, 1, 64, 128, 20),     # k - 1 = 19 beyond 128 past blocks: the SIMT gate's rows
 ]
 
 
@@ -102,6 +104,9 @@ VARLEN_SMALL = [
     ([300, 1, 1024, 129, 640], 4, 2, 128, 128, 3),
     ([0, 513, 0, 1], 2, 1, 64, 256, 2),   # empty and one-token sequences
     ([2000, 700, 1500], 8, 2, 128, 256, 4),
+    # one sequence of 258 blocks: its last tiles go to the SIMT gate, the rest
+    # (and the other sequences) to the tensor-core gate, in one call
+    ([300, 33024, 1000], 2, 1, 64, 128, 4),
 ]
 
 
@@ -181,25 +186,40 @@ def test_first_rows_of_a_block_round_once(moba, d):
     assert np.all(err_d <= _half_ulp_bf16(ref_d) + 1e-4), err_d.max()
 
 
-def test_routed_partial_beyond_fp16_range_is_reported(moba):
-    # Routed partials are stored in fp16.  Every row of block 1 routes to
-    # block 0, its only past block.  With block 0's V at 65280 (the largest
-    # bf16 value below the fp16 maximum) nothing is reported; at 65536 the
-    # partial rounds to inf in fp16 and the forward reports a device check.
-    N, Hq, Hkv, d, B, k = 1024, 2, 1, 128, 256, 3
+@pytest.mark.parametrize("scale", [65536.0, 1.0e6])
+def test_routed_partials_beyond_fp16_range(moba, scale):
+    """Routed partials are stored in fp16, scaled by a power of two derived
+    from the largest |v| (1 below 2^15), so values past the fp16 maximum
+    still give the exact attention.  Block 0's v is a constant `scale` (every
+    row of block 1 routes there: its only past block), block 2's v is N(0,1)
+    times `scale`; the other blocks are ordinary.  Bound per element: the
+    prefill's 1e-2 plus 2^-7 of the largest |v| the row attends (the bf16
+    weights, the fp16 partial and the bf16 output each round relative to it)."""
+    N, Hq, Hkv, d, B, k = 2048, 2, 1, 128, 256, 3
     w = S.Workload("fp16_range", [N], Hq, Hkv, d, B, k, seed=111)
     q, kk, v = S.make_qkv(w, "cuda")
-    q4, k4 = (x.view(1, N, x.shape[1], d) for x in (q, kk))
+    v = v.clone()
+    v[:B] = scale
+    v[2 * B:3 * B] = (v[2 * B:3 * B].float() * scale).to(torch.bfloat16)
+    q4, k4, v4 = (x.view(1, N, x.shape[1], d) for x in (q, kk, v))
     p = moba.make_params(1, N, Hq, Hkv, d, B, k)
-    for val, want in ((65280.0, 0), (65536.0, 6)):  # 6 = MOBA_ERR_DEVICE_CHECK
-        v2 = v.clone()
-        v2[:B] = val
-        ws = moba.alloc_workspace(moba.workspace_size(p, 1))
-        o, _ = moba.forward(q4, k4, v2.view(1, N, Hkv, d), B, k, ws=ws)
-        torch.cuda.synchronize()
-        assert moba.last_device_status(ws) == want, val
-        if want == 0:
-            assert torch.isfinite(o.float()).all()
+    ws = moba.alloc_workspace(moba.workspace_size(p, 1))
+    sel = torch.empty(1, Hq, N, k, dtype=torch.int32, device="cuda")
+    o, lse = moba.forward(q4, k4, v4, B, k, ws=ws, sel_out=sel)
+    torch.cuda.synchronize()
+    assert moba.last_device_status(ws) == 0
+    assert torch.isfinite(o.float()).all()
+    orc = Oracle(bf16_bits(q), bf16_bits(kk), bf16_bits(v), w.cu, Hq, Hkv, d, B, k)
+    rows = np.arange(N, dtype=np.int64)
+    Og, Lg, Sg = gather_rows_packed(o, lse, sel, rows, Hq, False, N)
+    ref, lref, _ = orc.attend(rows, Sg)
+    vmax_blk = v.float().abs().view(N // B, B * Hkv * d).max(dim=1).values.cpu().numpy()
+    m_row = np.where(Sg >= 0, vmax_blk[np.maximum(Sg, 0)], 0.0).max(axis=2)  # [R, H]
+    err = np.abs(Og.astype(np.float64) - ref)
+    bound = 1e-2 + 2.0 ** -7 * m_row[..., None]
+    assert np.all(err <= bound), float((err / bound).max())
+    assert np.abs(Lg - lref).max() <= 1e-3
+    assert (Sg == 0).any()  # block 0 is routed to
 
 
 def test_k_equal_n_matches_full_causal_kernel(moba):

@@ -119,3 +119,73 @@ def test_forward_selected_flags_a_future_block(moba):
     moba.forward_selected(q, kk, v, sel, B, k, ws=ws)
     torch.cuda.synchronize()
     assert moba.last_device_status(ws) == 6  # MOBA_ERR_DEVICE_CHECK
+
+
+# ---------------------------------------------------------------- packed sequences
+VARLEN_CASES = [
+    # lengths, Hq, Hkv, d, B, k
+    ([1500, 1, 0, 3000, 700], 4, 2, 128, 256, 4),
+    ([300, 4100, 129], 4, 1, 64, 128, 3),
+]
+VIDS = ["v" + "_".join(map(str, c[0])) for c in VARLEN_CASES]
+
+
+def _setup_varlen(case, seed):
+    lengths, Hq, Hkv, d, B, k = case
+    w = S.Workload("variant_v", lengths, Hq, Hkv, d, B, k, seed=seed, batch_mode=False)
+    q, kk, v = S.make_qkv(w, "cuda")
+    orc = Oracle(bf16_bits(q), bf16_bits(kk), bf16_bits(v), w.cu, Hq, Hkv, d, B, k)
+    cu = torch.tensor(w.cu, dtype=torch.int32, device="cuda")
+    return w, q, kk, v, cu, orc
+
+
+def _gpu_rows_varlen(o, lse, sel):
+    """o [T,H,d], lse [H,T], sel [H,T,k] -> [T,H,d], [T,H], [T,H,k]."""
+    return (o.float().cpu().numpy(), lse.t().contiguous().cpu().numpy(),
+            None if sel is None else sel.permute(1, 0, 2).contiguous().cpu().numpy())
+
+
+@pytest.mark.parametrize("mode", ["window", "sink"])
+@pytest.mark.parametrize("case", VARLEN_CASES, ids=VIDS)
+def test_static_selection_and_forward_varlen(moba, case, mode):
+    lengths, Hq, Hkv, d, B, k = case
+    w, q, kk, v, cu, orc = _setup_varlen(case, seed=616)
+    m = moba.ROUTE_WINDOW if mode == "window" else moba.ROUTE_SINK
+    sel = moba.static_selection_varlen(cu, w.T, Hq, B, k, m)
+    o, lse = moba.forward_selected_varlen(q, kk, v, cu, sel, B, k)
+    torch.cuda.synchronize()
+    rows = np.arange(w.T, dtype=np.int64)
+    want = static_selection(w.cu, rows, B, k, mode)
+    O, L, Sg = _gpu_rows_varlen(o, lse, sel)
+    assert np.array_equal(Sg, np.broadcast_to(want[:, None, :], Sg.shape))
+    _check_attention(orc, rows, O, L, Sg)
+
+
+@pytest.mark.parametrize("case", VARLEN_CASES, ids=VIDS)
+def test_minmax_gate_and_forward_varlen(moba, case):
+    lengths, Hq, Hkv, d, B, k = case
+    w, q, kk, v, cu, orc = _setup_varlen(case, seed=717)
+    sel = torch.full((Hq, w.T, k), -7, dtype=torch.int32, device="cuda")
+    o, lse = moba.forward_minmax_varlen(q, kk, v, cu, B, k, sel_out=sel)
+    sel_g = moba.gate_minmax_varlen(q, kk, cu, B, k)
+    torch.cuda.synchronize()
+    assert torch.equal(sel, sel_g)
+    rows = np.arange(w.T, dtype=np.int64)
+    O, L, Sg = _gpu_rows_varlen(o, lse, sel)
+    _, _, own = local_block_info(w.cu, rows, B)
+    check_selection_invariants(Sg, own, k)
+    ref, margin, maxabs = orc.select_minmax(rows)
+    differ = np.any(Sg != ref, axis=2)
+    flagged = margin < FLAG_REL * maxabs
+    assert not np.any(differ & ~flagged), np.argwhere(differ & ~flagged)[:3]
+    _check_attention(orc, rows, O, L, Sg)
+
+
+def test_forward_selected_varlen_with_the_gate_selection_equals_forward_varlen(moba):
+    case = ([2000, 900, 2500], 8, 2, 128, 256, 5)
+    w, q, kk, v, cu, _ = _setup_varlen(case, seed=818)
+    sel = torch.empty(8, w.T, 5, dtype=torch.int32, device="cuda")
+    o1, l1 = moba.forward_varlen(q, kk, v, cu, 256, 5, sel_out=sel)
+    o2, l2 = moba.forward_selected_varlen(q, kk, v, cu, sel, 256, 5)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
