@@ -34,7 +34,8 @@ EXPORTS = ("moba_workspace_size", "moba_workspace_size_varlen", "moba_gate", "mo
            "moba_forward_host_buffer_size", "moba_forward_host",
            "moba_static_selection_varlen", "moba_gate_minmax_varlen",
            "moba_forward_selected_varlen", "moba_forward_minmax_varlen",
-           "moba_backward_workspace_size_varlen", "moba_backward_varlen")
+           "moba_backward_workspace_size_varlen", "moba_backward_varlen",
+           "moba_forward_host_buffer_size_varlen", "moba_forward_host_varlen")
 
 ROUTE_WINDOW, ROUTE_SINK = 0, 1
 
@@ -148,6 +149,11 @@ def load_library(path=None):
     lib.moba_backward_varlen.restype = i32
     lib.moba_backward_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp,
                                          pp, vp, sz, vp]
+    lib.moba_forward_host_buffer_size_varlen.restype = sz
+    lib.moba_forward_host_buffer_size_varlen.argtypes = [pp, i64, i32, i32]
+    lib.moba_forward_host_varlen.restype = i32
+    lib.moba_forward_host_varlen.argtypes = [vp, vp, vp, vp, i32, i64, vp, vp, vp, pp, vp, sz,
+                                             vp]
     dp = ctypes.POINTER(MobaDecodeParams)
     lib.moba_decode_workspace_size.restype = sz
     lib.moba_decode_workspace_size.argtypes = [dp]
@@ -651,4 +657,31 @@ def forward_host(q, k, v, block_size, top_k, out, lse, dev_buf=None, heads_per_p
                                             _ptr(sel_out), ctypes.byref(p), _ptr(dev_buf),
                                             dev_buf.numel(), _stream(stream)),
            "moba_forward_host")
+    return out, lse
+
+
+def forward_host_buffer_size_varlen(params, total_tokens, num_seqs, heads_per_pass=0):
+    return int(load_library().moba_forward_host_buffer_size_varlen(
+        ctypes.byref(params), int(total_tokens), int(num_seqs), int(heads_per_pass)))
+
+
+def forward_host_varlen(q, k, v, cu_seqlens, block_size, top_k, out, lse, dev_buf=None,
+                        heads_per_pass=0, softmax_scale=0.0, sel_out=None, stream=None):
+    """forward_host for packed sequences: host tensors q [T,Hq,d], k/v [T,Hkv,d],
+    cu_seqlens (int32, host), out [T,Hq,d], lse [Hq,T] (and sel_out [Hq,T,k])."""
+    torch = _torch()
+    for t in (q, k, v, out, cu_seqlens):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("expected contiguous host tensors")
+    if cu_seqlens.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    T, Hq, d = q.shape
+    nseq = cu_seqlens.numel() - 1
+    p = make_params(1, 0, Hq, k.shape[1], d, block_size, top_k, softmax_scale)
+    if dev_buf is None:
+        dev_buf = alloc_workspace(forward_host_buffer_size_varlen(p, T, nseq, heads_per_pass))
+    _check(load_library().moba_forward_host_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, _ptr(out), _ptr(lse),
+        _ptr(sel_out), ctypes.byref(p), _ptr(dev_buf), dev_buf.numel(), _stream(stream)),
+        "moba_forward_host_varlen")
     return out, lse

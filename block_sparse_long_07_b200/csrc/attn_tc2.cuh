@@ -492,9 +492,12 @@ __global__ void __launch_bounds__(352, 1)
                        (acc || kk > 0) ? 1u : 0u);
     };
     // K_{j+1}: its slot and ring position are assigned in order when step j
-    // starts; the wait happens only before the first S MMA that reads it, so
-    // PV_0(j) never waits on the next K tile's load (with a shallow ring
-    // that load starts only when PV(j-1) frees a slot).
+    // starts.  With two Q buffers (a three-slot ring) the wait happens only
+    // before the first S MMA that reads it, so PV_0(j) never waits on the
+    // next K tile's load (that load starts only when PV(j-1) frees a slot).
+    // With the deep ring the wait comes first, where it overlaps the wait
+    // for the softmax (measured: 4 % faster at 4096-key blocks).
+    constexpr bool kLateK = (QBUFS == 2);
     uint32_t k_pos = 0;
     bool k_pending = false;
     auto ensure_k = [&]() -> bool {
@@ -557,6 +560,7 @@ __global__ void __launch_bounds__(352, 1)
           k_pos = kv_it;
           k_pending = true;
           ++kv_it;
+          if (!kLateK && !(ok = ensure_k())) break;
         }
         if (!(ok = kv_step(0, it, j, vs, ks2, qbase))) break;
         if (!(ok = kv_step(1, it, j, vs, ks2, qbase))) break;

@@ -684,6 +684,7 @@ struct HostBufs {
   char *q, *k, *v, *o;
   float* lse;
   int32_t* sel;
+  int32_t* cu;    // packed sequences: the device copy of cu_seqlens
   size_t staged;  // staging bytes
 };
 
@@ -703,6 +704,7 @@ HostBufs carve_host(const Problem& pr, char* base, size_t ws_bytes) {
   h.o = take(qb);
   h.lse = reinterpret_cast<float*>(take(sizeof(float) * (size_t)pr.T * pr.Hq));
   h.sel = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)pr.T * pr.Hq * pr.topk));
+  if (pr.varlen) h.cu = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * (size_t)(pr.nseq + 1)));
   h.staged = off - align_up(ws_bytes);
   return h;
 }
@@ -736,7 +738,8 @@ cudaError_t copy_cols(void* dst, const void* src, int64_t rows, int64_t ncols, i
 template <int D>
 moba_status forward_host_passes(const Problem& pr, const void* q_h, const void* k_h,
                                 const void* v_h, void* o_h, float* lse_h, int32_t* sel_h,
-                                const HostBufs& hb, const Ws& w, int nu_max, cudaStream_t st) {
+                                const int32_t* cu_h, const HostBufs& hb, const Ws& w, int nu_max,
+                                cudaStream_t st) {
   cudaStream_t h2d = copy_stream(0), d2h = copy_stream(1);
   if (!h2d || !d2h) return MOBA_ERR_CUDA;
   const int npass = (pr.Hkv + nu_max - 1) / nu_max;
@@ -754,9 +757,14 @@ moba_status forward_host_passes(const Problem& pr, const void* q_h, const void* 
   };
   auto in_ready = [&](int p) { return ev[p]; };
   auto done = [&](int p) { return ev[npass + p]; };
-  const int64_t rows_b = pr.nseq;                      // batch rows of lse / sel
-  const int64_t per_head_lse = pr.N, per_head_sel = (int64_t)pr.N * pr.topk;
+  // lse / sel rows: batch [b][Hq][N](...), packed [Hq][T](...) (one row)
+  const int64_t rows_b = pr.varlen ? 1 : pr.nseq;
+  const int64_t per_head_lse = pr.varlen ? pr.T : pr.N;
+  const int64_t per_head_sel = per_head_lse * pr.topk;
   if (cudaEventRecord(start, st) != cudaSuccess || cudaStreamWaitEvent(h2d, start, 0) != cudaSuccess)
+    return fail(MOBA_ERR_CUDA);
+  if (pr.varlen && cudaMemcpyAsync(hb.cu, cu_h, sizeof(int32_t) * (size_t)(pr.nseq + 1),
+                                   cudaMemcpyHostToDevice, h2d) != cudaSuccess)
     return fail(MOBA_ERR_CUDA);
   // inputs of every pass, in pass order, on the copy stream
   for (int p = 0; p < npass; ++p) {
@@ -773,6 +781,8 @@ moba_status forward_host_passes(const Problem& pr, const void* q_h, const void* 
   FwdCtx c;
   moba_status r = forward_setup<D>(pr, hb.q, hb.k, hb.v, hb.o, hb.lse, w, &c);
   if (r != MOBA_OK) return fail(r);
+  if (pr.varlen && cudaStreamWaitEvent(st, in_ready(0), 0) != cudaSuccess)  // cu_seqlens in
+    return fail(MOBA_ERR_CUDA);
   {
     SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
     Timed tm(kKPlan, st);
@@ -1493,11 +1503,43 @@ size_t moba_forward_host_buffer_size(const moba_params* p, int heads_per_pass) {
   return align_up(ws) + carve_host(pr, nullptr, ws).staged;
 }
 
+moba_status forward_host_impl(Problem pr, const void* q, const void* k, const void* v, void* o,
+                              float* lse, int32_t* sel_out, const int32_t* cu_h, void* dev_buf,
+                              size_t dev_bytes, moba_stream_t stream);
+
 moba_status moba_forward_host(const void* q, const void* k, const void* v, void* o, float* lse,
                               int32_t* sel_out, const moba_params* p, void* dev_buf,
                               size_t dev_bytes, moba_stream_t stream) {
   Problem pr;
   MOBA_TRY(make_problem(p, false, nullptr, 0, 0, true, &pr));
+  return forward_host_impl(pr, q, k, v, o, lse, sel_out, nullptr, dev_buf, dev_bytes, stream);
+}
+
+size_t moba_forward_host_buffer_size_varlen(const moba_params* p, int64_t total_tokens,
+                                            int num_seqs, int heads_per_pass) {
+  Problem pr;
+  static const int32_t dummy = 0;
+  if (make_problem(p, true, &dummy, num_seqs, total_tokens, true, &pr) != MOBA_OK) return 0;
+  int nu = (heads_per_pass <= 0 || heads_per_pass > pr.Hkv) ? pr.Hkv : heads_per_pass;
+  const size_t ws = carve(pr, nu, nullptr).bytes;
+  return align_up(ws) + carve_host(pr, nullptr, ws).staged;
+}
+
+moba_status moba_forward_host_varlen(const void* q, const void* k, const void* v,
+                                     const int32_t* cu_seqlens, int num_seqs,
+                                     int64_t total_tokens, void* o, float* lse, int32_t* sel_out,
+                                     const moba_params* p, void* dev_buf, size_t dev_bytes,
+                                     moba_stream_t stream) {
+  Problem pr;
+  static const int32_t dummy = 0;  // replaced by the device copy below
+  if (!cu_seqlens) return MOBA_ERR_INVALID_ARG;
+  MOBA_TRY(make_problem(p, true, &dummy, num_seqs, total_tokens, true, &pr));
+  return forward_host_impl(pr, q, k, v, o, lse, sel_out, cu_seqlens, dev_buf, dev_bytes, stream);
+}
+
+moba_status forward_host_impl(Problem pr, const void* q, const void* k, const void* v, void* o,
+                              float* lse, int32_t* sel_out, const int32_t* cu_h, void* dev_buf,
+                              size_t dev_bytes, moba_stream_t stream) {
   if (!q || !k || !v || !o || !lse) return MOBA_ERR_INVALID_ARG;
   if (!topk_supported(pr)) return MOBA_ERR_UNSUPPORTED;
   if ((int64_t)pr.T * pr.G * (pr.topk > 1 ? pr.topk - 1 : 1) >= INT32_MAX)
@@ -1513,9 +1555,11 @@ moba_status moba_forward_host(const void* q, const void* k, const void* v, void*
     ++nu;
   const Ws w = carve(pr, nu, static_cast<char*>(dev_buf));
   const HostBufs hb = carve_host(pr, static_cast<char*>(dev_buf), w.bytes);
+  if (pr.varlen) pr.cu = hb.cu;  // the kernels read the staged copy
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return pr.D == 128 ? forward_host_passes<128>(pr, q, k, v, o, lse, sel_out, hb, w, nu, st)
-                     : forward_host_passes<64>(pr, q, k, v, o, lse, sel_out, hb, w, nu, st);
+  return pr.D == 128
+             ? forward_host_passes<128>(pr, q, k, v, o, lse, sel_out, cu_h, hb, w, nu, st)
+             : forward_host_passes<64>(pr, q, k, v, o, lse, sel_out, cu_h, hb, w, nu, st);
 }
 
 // ---------------------------------------------------------------- backward

@@ -158,6 +158,19 @@ size_t moba_forward_host_buffer_size(const moba_params *p, int heads_per_pass);
 moba_status moba_forward_host(const void *q, const void *k, const void *v, void *o, float *lse,
                               int32_t *sel_out, const moba_params *p, void *dev_buf,
                               size_t dev_bytes, moba_stream_t stream);
+/* moba_forward_host for packed sequences: q, o [T][Hq][d], k, v [T][Hkv][d],
+ * lse [Hq][T], sel_out [Hq][T][top_k] and cu_seqlens [num_seqs + 1] int32,
+ * all in HOST memory (cu_seqlens is copied into dev_buf, sized by
+ * moba_forward_host_buffer_size_varlen).  Results equal moba_forward_varlen's.
+ * Errors as moba_forward_host; malformed cu_seqlens latch
+ * MOBA_ERR_DEVICE_CHECK in dev_buf's status word. */
+size_t moba_forward_host_buffer_size_varlen(const moba_params *p, int64_t total_tokens,
+                                            int num_seqs, int heads_per_pass);
+moba_status moba_forward_host_varlen(const void *q, const void *k, const void *v,
+                                     const int32_t *cu_seqlens, int num_seqs,
+                                     int64_t total_tokens, void *o, float *lse, int32_t *sel_out,
+                                     const moba_params *p, void *dev_buf, size_t dev_bytes,
+                                     moba_stream_t stream);
 
 /* ----------------------------------------------------------------- backward
  * Gradients of the forward's attention for an output gradient dO, over the

@@ -355,3 +355,25 @@ def test_forward_host_matches_forward(moba):
     torch.cuda.synchronize()
     assert moba.last_device_status(buf) == 0
     assert torch.equal(oh, o.cpu()) and torch.equal(lh, lse.cpu()) and torch.equal(sh, sel.cpu())
+
+
+def test_forward_host_varlen_matches_forward_varlen(moba):
+    """The packed-sequence host-buffer call gives forward_varlen's o, lse and
+    selection bit for bit (one kv head per pass, so the copies pipeline)."""
+    lengths, Hq, Hkv, d, B, k = [3000, 1, 0, 2500, 700], 8, 2, 128, 256, 4
+    w = S.Workload("host_varlen", lengths, Hq, Hkv, d, B, k, seed=4343, batch_mode=False)
+    q, kk, v = S.make_qkv(w, "cuda")
+    cu = torch.tensor(w.cu, dtype=torch.int32, device="cuda")
+    sel = torch.empty(Hq, w.T, k, dtype=torch.int32, device="cuda")
+    o, lse = moba.forward_varlen(q, kk, v, cu, B, k, sel_out=sel)
+    pin = lambda x: x.cpu().pin_memory()
+    qh, kh, vh = pin(q), pin(kk), pin(v)
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    sh = torch.empty(sel.shape, dtype=sel.dtype, pin_memory=True)
+    p = moba.make_params(1, 0, Hq, Hkv, d, B, k)
+    buf = moba.alloc_workspace(moba.forward_host_buffer_size_varlen(p, w.T, len(lengths), 1))
+    moba.forward_host_varlen(qh, kh, vh, cu.cpu(), B, k, oh, lh, dev_buf=buf, sel_out=sh)
+    torch.cuda.synchronize()
+    assert moba.last_device_status(buf) == 0
+    assert torch.equal(oh, o.cpu()) and torch.equal(lh, lse.cpu()) and torch.equal(sh, sel.cpu())
