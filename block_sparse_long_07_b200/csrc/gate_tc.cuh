@@ -148,6 +148,19 @@ __device__ __forceinline__ void chunk_group_max(const float (&v)[32], float (&t)
   }
 }
 
+// Candidate store: score v at shared address av and its column id at ai,
+// when take != 0 (predicated stores, so the caller's loop has no branch).
+__device__ __forceinline__ void st_shared_pred(uint32_t av, uint32_t ai, float v, int id,
+                                               uint32_t take) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %4, 0;\n\t"
+      "@p st.shared.f32 [%0], %2;\n\t"
+      "@p st.shared.u8 [%1], %3;\n\t}" ::"r"(av),
+      "r"(ai), "f"(v), "r"(id), "r"(take)
+      : "memory");
+}
+
 // Scores of columns [c, c + 32) of this lane's TMEM row; columns >= ncol -> -inf.
 __device__ __forceinline__ void load_scores(uint32_t taddr, int c, int ncol, float (&v)[32]) {
   uint32_t u[32];
@@ -336,6 +349,7 @@ __global__ void __launch_bounds__(352, 1)
     const uint32_t tS = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)grp * 256;
     float* cv = cv_all + grp * kCap * kTileM + r;    // slot q at cv[q * kTileM]
     uint8_t* ci = ci_all + grp * kCap * kTileM + r;
+    const uint32_t cv_s = smem_u32(cv), ci_s = smem_u32(ci);
     uint32_t n = 0, li = 0;
     bool ok = true;
     for (int64_t w = first; w < items && ok; w += step, ++li) {
@@ -389,13 +403,11 @@ __global__ void __launch_bounds__(352, 1)
         load_scores(tS, c, ncol, v);
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const bool take = v[e] >= T0;
-          const int slot = min(nc, kCap - 1);
-          if (take) {
-            cv[slot * kTileM] = v[e];
-            ci[slot * kTileM] = (uint8_t)(c + e);
-          }
-          nc += take ? 1 : 0;
+          const uint32_t take = v[e] >= T0 ? 1u : 0u;
+          const uint32_t slot = (uint32_t)min(nc, kCap - 1);
+          // predicated stores, no branch: a row takes a candidate here or not
+          st_shared_pred(cv_s + slot * (kTileM * 4), ci_s + slot * kTileM, v[e], c + e, take);
+          nc += (int)take;
         }
       }
       if (!valid) nc = 0;
@@ -465,21 +477,48 @@ __global__ void __launch_bounds__(352, 1)
       // ---- pass 3: T1 = (k-1)-th largest candidate, then the kept set
 #pragma unroll
       for (int u = 0; u < KM; ++u) t[u] = __int_as_float(0xff800000);
-      for (int q = 0; q < nc; ++q) chain_insert<KM>(t, cv[q * kTileM]);
-      const float T1 = list_at<KM>(t, npast - 1);
-      int gt = 0;
-      for (int q = 0; q < nc; ++q) gt += cv[q * kTileM] > T1 ? 1 : 0;
-      int eq_left = npast - gt;  // candidates equal to T1 still to keep, lowest blocks first
       int kept = 0;
-      for (int q = 0; q < nc; ++q) {
-        const float v = cv[q * kTileM];
-        bool take = v > T1;
-        if (v == T1 && eq_left > 0) {
-          take = true;
-          --eq_left;
+      if (kCap <= 24) {
+        // short lists: every slot into registers (independent loads), slots
+        // past nc as -inf, then fixed-length loops with no divergence
+        float cvr[kCap];
+#pragma unroll
+        for (int q = 0; q < kCap; ++q) {
+          const float x = cv[q * kTileM];
+          cvr[q] = q < nc ? x : __int_as_float(0xff800000);
         }
-        if (take && kept < npast) out[kept] = (int32_t)ci[q * kTileM];
-        kept += take ? 1 : 0;
+#pragma unroll
+        for (int q = 0; q < kCap; ++q) chain_insert<KM>(t, cvr[q]);
+        const float T1 = list_at<KM>(t, npast - 1);
+        int gt = 0;
+#pragma unroll
+        for (int q = 0; q < kCap; ++q) gt += cvr[q] > T1 ? 1 : 0;
+        int eq_left = npast - gt;  // candidates equal to T1 still to keep, lowest blocks first
+#pragma unroll
+        for (int q = 0; q < kCap; ++q) {
+          const bool eq = q < nc && cvr[q] == T1;
+          const bool take = cvr[q] > T1 || (eq && eq_left > 0);
+          eq_left -= (eq && take) ? 1 : 0;
+          const int32_t id = (int32_t)ci[q * kTileM];
+          if (take && kept < npast) out[kept] = id;
+          kept += take ? 1 : 0;
+        }
+      } else {
+        for (int q = 0; q < nc; ++q) chain_insert<KM>(t, cv[q * kTileM]);
+        const float T1 = list_at<KM>(t, npast - 1);
+        int gt = 0;
+        for (int q = 0; q < nc; ++q) gt += cv[q * kTileM] > T1 ? 1 : 0;
+        int eq_left = npast - gt;  // candidates equal to T1 still to keep, lowest blocks first
+        for (int q = 0; q < nc; ++q) {
+          const float v = cv[q * kTileM];
+          bool take = v > T1;
+          if (v == T1 && eq_left > 0) {
+            take = true;
+            --eq_left;
+          }
+          if (take && kept < npast) out[kept] = (int32_t)ci[q * kTileM];
+          kept += take ? 1 : 0;
+        }
       }
       for (int u = kept; u < npast; ++u) out[u] = -1;  // only with non-finite scores
       out[npast] = it.i;

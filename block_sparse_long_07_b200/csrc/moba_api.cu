@@ -127,6 +127,7 @@ struct Ws {
   int32_t* entry_off;
   int32_t* tile_off;
   uint32_t* cursor;
+  int4* items;     // routed work items (routed_items_kernel)
   uint2* entries;
   __half* part_O;  // routed partial O, fp16
   float* part_lse;
@@ -163,6 +164,9 @@ Ws carve(const Problem& pr, int nu, char* base) {
   w.tile_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * ((size_t)nu * NB + 1)));
   w.cursor = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * (size_t)nu * NB));
   const size_t prow = (size_t)nu * pr.T * pr.G;  // partial rows per pass
+  // at most one partly filled 256-row item per bucket beyond the full ones
+  w.items = reinterpret_cast<int4*>(
+      take(sizeof(int4) * (prow * np / (2 * kTileM) + (size_t)nu * NB + 1)));
   w.entries = reinterpret_cast<uint2*>(take(sizeof(uint2) * prow * np));
   w.part_O = reinterpret_cast<__half*>(take(2 * prow * np * pr.D));
   w.part_lse = reinterpret_cast<float*>(take(sizeof(float) * prow * np));
@@ -611,6 +615,7 @@ moba_status forward_setup(const Problem& pr, const void* q, const void* k, const
   a.R = pr.R;
   a.tile_off = w.tile_off;
   a.entry_off = w.entry_off;
+  a.items = w.items;
   a.entries = w.entries;
   a.part_O = w.part_O;
   a.part_lse = w.part_lse;
@@ -635,6 +640,12 @@ moba_status forward_one_pass(const Problem& pr, FwdCtx& c, const Ws& w, const in
       Timed tm(kKScan, st);
       bucket_scan_kernel<<<1, 1024, 0, st>>>(w.counts, u0, nu, 2 * kTileM, w.P, (int)pr.NBmax,
                                              w.entry_off, w.tile_off, w.cursor);
+    }
+    MOBA_CUDA(cudaGetLastError());
+    {
+      Timed tm(kKScan, st);
+      routed_items_kernel<<<(unsigned)(nu * pr.NBmax), 128, 0, st>>>(
+          w.entry_off, w.tile_off, w.P, nu, 2 * kTileM, w.items);
     }
     MOBA_CUDA(cudaGetLastError());
     MOBA_TRY(launch_scatter(pr, w, sel, u0, nu, st));
