@@ -61,7 +61,6 @@ struct AttnArgs {
   int u0, nu;              // pass: kv heads u0 .. u0+nu-1
   const int32_t* tile_off;   // routed: [nu*NB + 1] work items per bucket, prefix
   const int32_t* entry_off;  // routed: [nu*NB + 1] bucket entries, prefix
-  const int4* items;         // routed: per work item {first entry, first key, unit, rows}
   const uint2* entries;
   __half* part_O;            // [nu][T][G][topk-1][D], fp16 (see the epilogue)
   float* part_lse;           // [nu][T][G][topk-1]
@@ -126,46 +125,31 @@ __device__ __forceinline__ int64_t num_items2(const AttnArgs& a, int pair_own) {
 
 // Work item w of the launch.  For own/dense modes the items of one head are
 // query-tile pairs numbered through P.totals[2] / P.pair_off (see plan).
-// A routed item from its descriptor (routed_items_kernel): up to 256 rows
-// of one bucket against the B keys of its block.
-__device__ __forceinline__ Item routed_item(const AttnArgs& a, int4 d) {
-  Item it;
-  it.u = d.z;
-  it.g = a.u0 + d.z;
-  it.h = -1;
-  it.kstart = d.y;
-  it.nkv = a.B / kTileN;
-  it.rows_x[0] = min(kTileM, d.w);
-  it.rows_x[1] = max(0, min(kTileM, d.w - kTileM));
-  it.nkv_x[0] = it.nkv;
-  it.nkv_x[1] = it.rows_x[1] > 0 ? it.nkv : 0;
-  it.qstart = 0;
-  it.seq = 0;
-  it.seq_start = 0;
-  it.own_block = 0;
-  it.e0 = d.x;
-  return it;
-}
-
-// Walks a role's items w = first, first + step, ...  Routed descriptors are
-// loaded one item ahead: the load for the next item is issued when the
-// current one is taken, so its latency hides behind the current item's work.
-template <int MODE>
-struct ItemWalk {
-  int4 raw;
-  __device__ __forceinline__ ItemWalk(const AttnArgs& a, int64_t first, int64_t items) {
-    raw = make_int4(0, 0, 0, 0);
-    if (MODE == kRouted && first < items) raw = a.items[first];
-  }
-  __device__ __forceinline__ Item take(const AttnArgs& a, int64_t w, int64_t step,
-                                       int64_t items, int pair_own);
-};
-
 template <int MODE>
 __device__ __forceinline__ Item item_info(const AttnArgs& a, int64_t w, int pair_own) {
   Item it;
   if (MODE == kRouted) {
-    it = routed_item(a, a.items[w]);
+    const int NB = a.P.totals[0];
+    const int M = a.nu * NB;
+    const int f = upper_index(a.tile_off, M + 1, w);
+    const int u = f / NB, J = f % NB;
+    const int64_t row0 = (w - a.tile_off[f]) * (int64_t)(2 * kTileM);
+    const int64_t cnt = (int64_t)a.entry_off[f + 1] - a.entry_off[f];
+    const int64_t left = cnt - row0;
+    it.u = u;
+    it.g = a.u0 + u;
+    it.h = -1;
+    it.kstart = a.P.blk_tok[J];
+    it.nkv = a.B / kTileN;
+    it.rows_x[0] = (int)min((int64_t)kTileM, left);
+    it.rows_x[1] = (int)max((int64_t)0, min((int64_t)kTileM, left - kTileM));
+    it.nkv_x[0] = it.nkv;
+    it.nkv_x[1] = it.rows_x[1] > 0 ? it.nkv : 0;
+    it.qstart = 0;
+    it.seq = 0;
+    it.seq_start = 0;
+    it.own_block = 0;
+    it.e0 = a.entry_off[f] + row0;
   } else {
     const int HP = (MODE == kOwn) ? a.nu * a.G : a.Hq;
     const bool paired = (MODE == kDense) || pair_own;
@@ -199,15 +183,6 @@ __device__ __forceinline__ Item item_info(const AttnArgs& a, int64_t w, int pair
     it.nkv = max(it.nkv_x[0], it.nkv_x[1]);
     it.e0 = 0;
   }
-  return it;
-}
-
-template <int MODE>
-__device__ __forceinline__ Item ItemWalk<MODE>::take(const AttnArgs& a, int64_t w, int64_t step,
-                                                     int64_t items, int pair_own) {
-  if (MODE != kRouted) return item_info<MODE>(a, w, pair_own);
-  const Item it = routed_item(a, raw);
-  if (w + step < items) raw = a.items[w + step];
   return it;
 }
 
@@ -394,9 +369,8 @@ __global__ void __launch_bounds__(352, 1)
     if (lane == 0) {
       uint32_t kv_it = 0, lt = 0;
       bool ok = true;
-      ItemWalk<MODE> walk(a, first, items);
       for (int64_t w = first; w < items && ok; w += step, ++lt) {
-        const Item it = walk.take(a, w, step, items, pair_own);
+        const Item it = item_info<MODE>(a, w, pair_own);
         if (MODE != kRouted) {
           const int qb = lt % QB;
           ok = mbar_wait(&q_empty[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
@@ -446,9 +420,8 @@ __global__ void __launch_bounds__(352, 1)
       bool ok = true;
       constexpr int CPR = D / 8;     // 16-B chunks per row
       constexpr int RPI = 32 / CPR;  // rows per warp instruction
-      ItemWalk<MODE> walk(a, first, items);
       for (int64_t w = first; w < items && ok; w += step, ++lt) {
-        const Item it = walk.take(a, w, step, items, pair_own);
+        const Item it = item_info<MODE>(a, w, pair_own);
         const int qb = lt % QB;
         ok = mbar_wait(&q_empty[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
         ok = __all_sync(0xffffffffu, ok);
@@ -564,9 +537,8 @@ __global__ void __launch_bounds__(352, 1)
       }
       return true;
     };
-    ItemWalk<MODE> walk(a, first, items);
     for (int64_t w = first; w < items && ok; w += step, ++lt) {
-      const Item it = walk.take(a, w, step, items, pair_own);
+      const Item it = item_info<MODE>(a, w, pair_own);
       const int qb = lt % QB;
       const uint32_t qbase = sQa + qb * C::kQBytes;
       if (!(ok = wait(&q_full[qb], (lt / QB) & 1))) break;
@@ -612,21 +584,8 @@ __global__ void __launch_bounds__(352, 1)
     const float pscale = (MODE == kRouted) ? exp2f(-(float)partial_scale_log2(a.status[1])) : 1.f;
     uint32_t ns = 0, no = 0;
     bool ok = true;
-    ItemWalk<MODE> walk(a, first, items);
     for (int64_t w = first; w < items && ok; w += step) {
-      // only a few of the item's fields stay live through the softmax loop
-      // (registers are what that loop is short of); own / dense items are
-      // decoded again for the epilogue
-      int nkv, rows_x, unit = 0;
-      uint2 ent = make_uint2(0xFFFFFFFFu, 0u);
-      {
-        const Item it0 = walk.take(a, w, step, items, pair_own);
-        nkv = it0.nkv_x[x];
-        rows_x = it0.rows_x[x];
-        unit = it0.u;
-        // routed: this row's entry, needed only by the epilogue, loaded now
-        if (MODE == kRouted && nkv > 0 && r < rows_x) ent = a.entries[it0.e0 + x * kTileM + r];
-      }
+      const int nkv = item_info<MODE>(a, w, pair_own).nkv_x[x];
       if (nkv == 0) continue;
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < nkv; ++j) {
@@ -674,8 +633,8 @@ __global__ void __launch_bounds__(352, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const Item it = (MODE == kRouted) ? Item{} : item_info<MODE>(a, w, pair_own);
-      const bool valid = r < rows_x;
+      const Item it = item_info<MODE>(a, w, pair_own);
+      const bool valid = r < it.rows_x[x];
       const float inv = 1.f / l_run;
       const float lse2 = m_run + lg2_approx(l_run);
       // destination of this row
@@ -687,11 +646,11 @@ __global__ void __launch_bounds__(352, 1)
       float lse_val = lse2;
       if (valid) {
         if (MODE == kRouted) {
-          const uint2 e = ent;
+          const uint2 e = a.entries[it.e0 + x * kTileM + r];
           const int hh = (int)(e.y & 0xFFFFu), sl = (int)(e.y >> 16);
           if (e.x < (uint32_t)a.L.T && hh < a.G && sl < a.topk - 1) {
             const int64_t prow =
-                (((int64_t)unit * a.L.T + e.x) * a.G + hh) * (a.topk - 1) + sl;
+                (((int64_t)it.u * a.L.T + e.x) * a.G + hh) * (a.topk - 1) + sl;
             kind = 1;
             dsth = a.part_O + prow * D;
             lse_dst = a.part_lse + prow;

@@ -455,27 +455,6 @@ __global__ void bucket_scan_kernel(const uint32_t* __restrict__ counts, int u0, 
   }
 }
 
-// Work items of the routed attention, one per 256 gathered rows of a bucket
-// (u, J): items[w] = {first entry, first key of block J, u, rows}, so a
-// kernel role finds its item with one 16-byte load instead of a search over
-// tile_off.  One CTA per bucket of the pass.
-__global__ void __launch_bounds__(128) routed_items_kernel(const int32_t* __restrict__ entry_off,
-                                                           const int32_t* __restrict__ tile_off,
-                                                           const Plan P, int nu, int item_rows,
-                                                           int4* __restrict__ items) {
-  const int NB = P.totals[0];
-  const int f = blockIdx.x;
-  if (f >= nu * NB) return;
-  const int u = f / NB, J = f % NB;
-  const int32_t t0 = tile_off[f], t1 = tile_off[f + 1];
-  const int32_t e0 = entry_off[f], cnt = entry_off[f + 1] - e0;
-  const int32_t k0 = P.blk_tok[J];
-  for (int32_t t = t0 + (int32_t)threadIdx.x; t < t1; t += blockDim.x) {
-    const int32_t row0 = (t - t0) * item_rows;
-    items[t] = make_int4(e0 + row0, k0, u, min(item_rows, cnt - row0));
-  }
-}
-
 // ---------------------------------------------------------------- scatter
 // One CTA per (query tile, query head of the pass).  Every routed
 // (row, head, slot) -- a past block in the row's selection -- is written to

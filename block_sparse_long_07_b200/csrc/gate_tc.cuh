@@ -127,6 +127,17 @@ __device__ __forceinline__ void chain_insert(float (&t)[KM], float v) {
   }
 }
 
+// Insert v into the ascending list t[0..L) of the L smallest values.
+template <int L>
+__device__ __forceinline__ void chain_insert_min(float (&t)[L], float v) {
+#pragma unroll
+  for (int u = 0; u < L; ++u) {
+    const float lo = fminf(t[u], v);
+    v = fmaxf(t[u], v);
+    t[u] = lo;
+  }
+}
+
 template <int KM>
 __device__ __forceinline__ float list_at(const float (&t)[KM], int idx) {
   float r = t[0];
@@ -487,9 +498,25 @@ __global__ void __launch_bounds__(352, 1)
           const float x = cv[q * kTileM];
           cvr[q] = q < nc ? x : __int_as_float(0xff800000);
         }
+        // T1 = the (k-1)-th largest candidate = the (nc - (k-1) + 1)-th
+        // smallest.  A row has a few candidates more than k-1 (about two
+        // for i.i.d. scores), so a list of the 4 smallest usually settles it.
+        const int drop = max(nc - npast, 0);
+        float T1;
+        // the lanes here are this warp's valid rows without an overflow
+        if (__all_sync(__activemask(), drop < 4)) {
+          float sm[4];
 #pragma unroll
-        for (int q = 0; q < kCap; ++q) chain_insert<KM>(t, cvr[q]);
-        const float T1 = list_at<KM>(t, npast - 1);
+          for (int u = 0; u < 4; ++u) sm[u] = __int_as_float(0x7f800000);
+#pragma unroll
+          for (int q = 0; q < kCap; ++q)
+            chain_insert_min<4>(sm, q < nc ? cvr[q] : __int_as_float(0x7f800000));
+          T1 = list_at<4>(sm, drop);
+        } else {
+#pragma unroll
+          for (int q = 0; q < kCap; ++q) chain_insert<KM>(t, cvr[q]);
+          T1 = list_at<KM>(t, npast - 1);
+        }
         int gt = 0;
 #pragma unroll
         for (int q = 0; q < kCap; ++q) gt += cvr[q] > T1 ? 1 : 0;

@@ -127,7 +127,6 @@ struct Ws {
   int32_t* entry_off;
   int32_t* tile_off;
   uint32_t* cursor;
-  int4* items;     // routed work items (routed_items_kernel)
   uint2* entries;
   __half* part_O;  // routed partial O, fp16
   float* part_lse;
@@ -164,9 +163,6 @@ Ws carve(const Problem& pr, int nu, char* base) {
   w.tile_off = reinterpret_cast<int32_t*>(take(sizeof(int32_t) * ((size_t)nu * NB + 1)));
   w.cursor = reinterpret_cast<uint32_t*>(take(sizeof(uint32_t) * (size_t)nu * NB));
   const size_t prow = (size_t)nu * pr.T * pr.G;  // partial rows per pass
-  // at most one partly filled 256-row item per bucket beyond the full ones
-  w.items = reinterpret_cast<int4*>(
-      take(sizeof(int4) * (prow * np / (2 * kTileM) + (size_t)nu * NB + 1)));
   w.entries = reinterpret_cast<uint2*>(take(sizeof(uint2) * prow * np));
   w.part_O = reinterpret_cast<__half*>(take(2 * prow * np * pr.D));
   w.part_lse = reinterpret_cast<float*>(take(sizeof(float) * prow * np));
@@ -615,7 +611,6 @@ moba_status forward_setup(const Problem& pr, const void* q, const void* k, const
   a.R = pr.R;
   a.tile_off = w.tile_off;
   a.entry_off = w.entry_off;
-  a.items = w.items;
   a.entries = w.entries;
   a.part_O = w.part_O;
   a.part_lse = w.part_lse;
@@ -640,12 +635,6 @@ moba_status forward_one_pass(const Problem& pr, FwdCtx& c, const Ws& w, const in
       Timed tm(kKScan, st);
       bucket_scan_kernel<<<1, 1024, 0, st>>>(w.counts, u0, nu, 2 * kTileM, w.P, (int)pr.NBmax,
                                              w.entry_off, w.tile_off, w.cursor);
-    }
-    MOBA_CUDA(cudaGetLastError());
-    {
-      Timed tm(kKScan, st);
-      routed_items_kernel<<<(unsigned)(nu * pr.NBmax), 128, 0, st>>>(
-          w.entry_off, w.tile_off, w.P, nu, 2 * kTileM, w.items);
     }
     MOBA_CUDA(cudaGetLastError());
     MOBA_TRY(launch_scatter(pr, w, sel, u0, nu, st));
@@ -1009,10 +998,11 @@ moba_status backward_passes(const Problem& pr, const void* q, const void* k, con
   CUtensorMap tk, tv;
   if (!make_tmap(&tk, k, pr.Hkv, pr.T, D) || !make_tmap(&tv, v, pr.Hkv, pr.T, D))
     return MOBA_ERR_CUDA;
-  MOBA_CUDA(cudaFuncSetAttribute(bw_kv_kernel<D, kBwRouted>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
-  MOBA_CUDA(cudaFuncSetAttribute(bw_kv_kernel<D, kBwOwn>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
+  using C2 = BwKv2Cfg<D>;
+  MOBA_CUDA(cudaFuncSetAttribute(bw_kv2_kernel<D, kBwRouted>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C2::kSmemBytes));
+  MOBA_CUDA(cudaFuncSetAttribute(bw_kv2_kernel<D, kBwOwn>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C2::kSmemBytes));
   MOBA_CUDA(cudaFuncSetAttribute(bw_q_kernel<D, kBwRouted>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytesQ));
   MOBA_CUDA(cudaFuncSetAttribute(bw_q_kernel<D, kBwOwn>,
@@ -1054,8 +1044,8 @@ moba_status backward_passes(const Problem& pr, const void* q, const void* k, con
       MOBA_TRY(launch_scatter(pr, w, sel, u0, nu, st));
       {
         Timed tm(kKBwKv, st);
-        bw_kv_kernel<D, kBwRouted><<<(unsigned)(nu * pr.NBmax * KT), 256, C::kSmemBytes, st>>>(
-            tk, tv, a);
+        bw_kv2_kernel<D, kBwRouted>
+            <<<(unsigned)(nu * pr.NBmax * KT), C2::kThreads, C2::kSmemBytes, st>>>(tk, tv, a);
         MOBA_CUDA(cudaGetLastError());
       }
       {
@@ -1067,8 +1057,8 @@ moba_status backward_passes(const Problem& pr, const void* q, const void* k, con
     }
     {
       Timed tm(kKBwKv, st);
-      bw_kv_kernel<D, kBwOwn><<<(unsigned)(nu * pr.NBmax * KT), 256, C::kSmemBytes, st>>>(tk, tv,
-                                                                                       a);
+      bw_kv2_kernel<D, kBwOwn>
+          <<<(unsigned)(nu * pr.NBmax * KT), C2::kThreads, C2::kSmemBytes, st>>>(tk, tv, a);
       MOBA_CUDA(cudaGetLastError());
     }
     {
