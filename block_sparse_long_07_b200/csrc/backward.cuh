@@ -490,6 +490,323 @@ __global__ void __launch_bounds__(256, 1)
   }
 }
 
+// ---------------------------------------------------------------- dK / dV, warp-specialised
+// One CTA per (bucket or own block, 128-key tile), as bw_kv_kernel, with the
+// rows in 64-row tiles so that TMEM holds two tiles' S^T / dP^T next to the
+// dV / dK accumulators: the elementwise pass of tile n runs while the tensor
+// core computes dV / dK of tile n - 1 and S^T / dP^T of tile n + 1.
+//   warps 0-7  elementwise: warp w takes keys 32 (w % 4) .. + 31 (its TMEM lane
+//              quarter) and rows 32 (w / 4) .. + 31 of the tile; forms P^T and
+//              dS^T = P^T (dP^T - D) and packs them as bf16 over the columns it
+//              read (rows 2j, 2j + 1 -> column j of its half)
+//   warp  8    TMEM allocation, the K / V load and the MMA issue
+//   warps 9-10 row gather (q, dO and (D, lse2) of 32 rows each) into a
+//              three-stage ring, two tiles in flight
+// MMA order: S^T(n), dP^T(n) [buffer n % 2], then dV / dK(n - 1) once its P^T /
+// dS^T are packed.  S^T(n + 2) reuses buffer n % 2; it is issued after dV /
+// dK(n), the last reader of the packed values there, and tensor-core
+// operations from one thread complete in issue order.
+template <int D>
+struct BwKv2Cfg {
+  static constexpr int kRows = 64;                   // rows per tile
+  static constexpr int kStages = 3;                  // row-tile ring
+  static constexpr int kKVTile = kTileN * D * 2;     // one 128-key K or V tile
+  static constexpr int kKVHalf = kTileN * 128;       // 128 rows x 64 columns bf16
+  static constexpr int kRowTile = kRows * D * 2;     // one 64-row q or dO tile
+  static constexpr int kRowHalf = kRows * 128;       // 64 rows x 64 columns bf16
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kKVTile;
+  static constexpr int kOffQ = kOffV + kKVTile;               // [stage]
+  static constexpr int kOffDO = kOffQ + kStages * kRowTile;   // [stage]
+  static constexpr int kOffDL = kOffDO + kStages * kRowTile;  // [stage][64] (D, lse2)
+  static constexpr int kOffBar = kOffDL + kStages * kRows * 8;
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 1;
+  static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
+  static constexpr int kThreads = 352;
+  static constexpr uint32_t kColS = 0;         // [2] x 64 columns: S^T, then packed P^T
+  static constexpr uint32_t kColDP = 128;      // [2] x 64 columns: dP^T, then packed dS^T
+  static constexpr uint32_t kColV = 256;       // dV accumulator
+  static constexpr uint32_t kColK = 256 + D;   // dK accumulator
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kSmemBytes <= 232448, "bw_kv2 shared memory beyond the per-CTA limit");
+};
+
+// Packed column of the A operand for rows 16 kk .. 16 kk + 15 of a tile:
+// rows 0..31 pack into columns 0..15, rows 32..63 into 32..47.
+__host__ __device__ constexpr uint32_t bw2_packed_col(int kk) {
+  return kk < 2 ? 8u * kk : 16u + 8u * kk;
+}
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(352, 1)
+    bw_kv2_kernel(const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const BwArgs a) {
+  using C = BwKv2Cfg<D>;
+  constexpr int ST = C::kStages;
+  constexpr int RT = C::kRows;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* kv_bar = bars;               // K / V landed
+  uint64_t* rows_full = bars + 1;        // [ST] a row tile gathered
+  uint64_t* rows_empty = rows_full + ST; // [ST] its dV / dK MMAs done
+  uint64_t* s_full = rows_empty + ST;    // [2] S^T / dP^T of a tile in TMEM
+  uint64_t* p_full = s_full + 2;         // [2] P^T / dS^T packed
+  uint64_t* done_bar = p_full + 2;       // every MMA done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int NB = a.P.totals[0];
+  const int KT = a.B / kTileN;
+  const int64_t f = blockIdx.x / KT;
+  const int kt = (int)(blockIdx.x % KT);
+  if (f >= (int64_t)a.nu * NB) return;
+  const int u = (int)(f / NB), J = (int)(f % NB);
+  const int g = a.u0 + u;
+  const int blen = a.P.blk_len[J];
+  const int nkeys = min(kTileN, blen - kt * kTileN);
+  if (nkeys <= 0) return;
+  const int64_t kstart = (int64_t)a.P.blk_tok[J] + (int64_t)kt * kTileN;
+  const int64_t bend = (int64_t)a.P.blk_tok[J] + blen;
+  int64_t e0 = 0, e1 = 0;
+  int ntiles, own_tiles = 0;
+  if (MODE == kBwRouted) {
+    e0 = a.entry_off[f];
+    e1 = a.entry_off[f + 1];
+    ntiles = (int)((e1 - e0 + RT - 1) / RT);
+  } else {
+    own_tiles = (int)((bend - kstart + RT - 1) / RT);  // row tiles from the key tile on
+    ntiles = own_tiles * a.G;
+  }
+  if (ntiles == 0) return;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_bar, 1);
+    for (int q = 0; q < ST; ++q) {
+      mbar_init(&rows_full[q], 2);
+      mbar_init(&rows_empty[q], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 8);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  uint32_t* st = a.status;
+  unsigned char* sK = smem + C::kOffK;
+  unsigned char* sV = smem + C::kOffV;
+  float2* sdl = reinterpret_cast<float2*>(smem + C::kOffDL);
+
+  if (warp >= 9) {
+    // ------------------------------------------------------------ row gather
+    const int r = (warp - 9) * 32 + lane;  // row of the tile
+    bool ok = true;
+    int n = 0;
+    for (; n < ntiles && ok; ++n) {
+      const int sg = n % ST;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&rows_empty[sg], ((n / ST) & 1) ^ 1, abort_flag, st));
+      if (!ok) break;
+      BwRow x{-1, 0};
+      if (MODE == kBwRouted) {
+        x = bw_row_routed(a, g, e0 + (int64_t)n * RT, e1, r);
+      } else {
+        const int hh = n / own_tiles;
+        const int64_t t = kstart + (int64_t)(n % own_tiles) * RT + r;
+        if (t < bend) {
+          x.t = t;
+          x.h = g * a.G + hh;
+        }
+      }
+      const int64_t t = x.t < 0 ? 0 : x.t;  // a missing row reads token 0 (finite); P = 0
+      const __nv_bfloat16* qs = a.q + ((size_t)t * a.Hq + (x.t < 0 ? 0 : x.h)) * D;
+      const __nv_bfloat16* gs = a.dO + ((size_t)t * a.Hq + (x.t < 0 ? 0 : x.h)) * D;
+      unsigned char* dq_ = smem + C::kOffQ + sg * C::kRowTile;
+      unsigned char* ddo = smem + C::kOffDO + sg * C::kRowTile;
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint32_t off = (uint32_t)(c >> 3) * C::kRowHalf + sw128_offset(r, c & 7);
+        cp_async_16(dq_ + off, qs + c * 8);
+        cp_async_16(ddo + off, gs + c * 8);
+      }
+      float2* d = sdl + sg * RT + r;
+      if (x.t >= 0)
+        cp_async_8(d, a.dl + (size_t)x.t * a.Hq + x.h);
+      else
+        *d = make_float2(0.f, __int_as_float(0x7f800000));
+      cp_async_commit();
+      if (n > 0) {  // tile n - 1 landed: publish it (two tiles in flight)
+        cp_async_wait_group<1>();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rows_full[(n - 1) % ST]);
+      }
+    }
+    cp_async_wait_all();
+    if (ok && n > 0) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rows_full[(n - 1) % ST]);
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ K / V load, MMA issue
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_bar, 2 * C::kKVTile);
+#pragma unroll
+      for (int hx = 0; hx < D / 64; ++hx) {
+        tma_load_3d(sK + hx * C::kKVHalf, &tm_k, kv_bar, hx * 64, g, (int)kstart);
+        tma_load_3d(sV + hx * C::kKVHalf, &tm_v, kv_bar, hx * 64, g, (int)kstart);
+      }
+    }
+    __syncwarp();
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, st));
+    };
+    constexpr uint32_t idS = idesc_bf16_f32(kTileN, RT, false, false);  // M = keys, N = rows
+    constexpr uint32_t idG = idesc_bf16_f32(kTileN, D, false, true);    // A in TMEM, B MN-major
+    const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
+    const uint32_t sQa = smem_u32(smem + C::kOffQ), sDOa = smem_u32(smem + C::kOffDO);
+    bool ok = wait(kv_bar, 0);
+    // dV / dK of tile m (its P^T / dS^T packed in buffer m % 2)
+    auto grad_mmas = [&](int m) -> bool {
+      const int b = m & 1, sg = m % ST;
+      if (!wait(&p_full[b], (m >> 1) & 1)) return false;
+      tc_fence_after();
+      const uint32_t qb = sQa + sg * C::kRowTile, ob = sDOa + sg * C::kRowTile;
+#pragma unroll
+      for (int kk = 0; kk < RT / 16; ++kk) {  // K = rows, 16 per step
+        const uint32_t acc = (m > 0 || kk > 0) ? 1u : 0u;
+        tc_mma_ts_warp(tmem + C::kColV, tmem + C::kColS + 64u * b + bw2_packed_col(kk),
+                       sdesc_mnmajor_sw128(ob + kk * 2048, C::kRowHalf, 1024), idG, acc);
+        tc_mma_ts_warp(tmem + C::kColK, tmem + C::kColDP + 64u * b + bw2_packed_col(kk),
+                       sdesc_mnmajor_sw128(qb + kk * 2048, C::kRowHalf, 1024), idG, acc);
+      }
+      tc_commit_warp(&rows_empty[sg]);
+      return true;
+    };
+    int n = 0;
+    for (; n < ntiles && ok; ++n) {
+      const int b = n & 1, sg = n % ST;
+      if (!(ok = wait(&rows_full[sg], (n / ST) & 1))) break;
+      tc_fence_after();
+      const uint32_t qb = sQa + sg * C::kRowTile, ob = sDOa + sg * C::kRowTile;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t koff = (kk >> 2) * C::kKVHalf + (kk & 3) * 32;
+        const uint32_t roff = (kk >> 2) * C::kRowHalf + (kk & 3) * 32;
+        tc_mma_ss_warp(tmem + C::kColS + 64u * b, sdesc_kmajor_sw128(sKa + koff),
+                       sdesc_kmajor_sw128(qb + roff), idS, kk > 0 ? 1u : 0u);
+        tc_mma_ss_warp(tmem + C::kColDP + 64u * b, sdesc_kmajor_sw128(sVa + koff),
+                       sdesc_kmajor_sw128(ob + roff), idS, kk > 0 ? 1u : 0u);
+      }
+      tc_commit_warp(&s_full[b]);
+      if (n > 0 && !(ok = grad_mmas(n - 1))) break;
+    }
+    if (ok && n > 0) ok = grad_mmas(n - 1);
+    tc_commit_warp(done_bar);  // every MMA of this CTA (also after an abort)
+  } else {
+    // ------------------------------------------------------------ elementwise (warps 0-7)
+    const int quad = warp & 3, hc = warp >> 2;
+    const int key = quad * 32 + lane;  // TMEM lane
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const bool key_ok = key < nkeys;
+    const int64_t key_tok = kstart + key;
+    bool ok = true;
+    for (int n = 0; n < ntiles && ok; ++n) {
+      const int b = n & 1, sg = n % ST;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (n >> 1) & 1, abort_flag, st));
+      if (!ok) break;
+      // the tile's (D, lse2) were published with its rows
+      ok = __all_sync(0xffffffffu, mbar_wait(&rows_full[sg], (n / ST) & 1, abort_flag, st));
+      if (!ok) break;
+      tc_fence_after();
+      const int c0 = 32 * hc;
+      const uint32_t tS = tmem + lane_off + C::kColS + 64u * b;
+      const uint32_t tDP = tmem + lane_off + C::kColDP + 64u * b;
+      uint32_t sv[32], dv[32];
+      tmem_ld32(tS + c0, sv);
+      tmem_ld32(tDP + c0, dv);
+      tc_wait_ld();
+      int64_t row_tok0 = 0;
+      if (MODE == kBwOwn) row_tok0 = kstart + (int64_t)(n % own_tiles) * RT + c0;
+      const float2* dl = sdl + sg * RT + c0;
+      uint32_t pp[16], dd[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float4 l = *reinterpret_cast<const float4*>(dl + 2 * e);  // (D, lse2) of 2 rows
+        float p2[2], d2[2];
+#pragma unroll
+        for (int xx = 0; xx < 2; ++xx) {
+          bool keep = key_ok;
+          if (MODE == kBwOwn) keep = keep && (key_tok <= row_tok0 + 2 * e + xx);
+          const float Dc = xx ? l.z : l.x, lc = xx ? l.w : l.y;
+          const float p =
+              keep ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + xx]), a.scale_log2, -lc)) : 0.f;
+          p2[xx] = p;
+          d2[xx] = p * (__uint_as_float(dv[2 * e + xx]) - Dc);
+        }
+        pp[e] = pack_bf16x2(p2[0], p2[1]);
+        dd[e] = pack_bf16x2(d2[0], d2[1]);
+      }
+      // rows c0 .. c0 + 31 pack into columns c0 / 2 * ... see bw2_packed_col
+      const uint32_t pc = hc ? 32u : 0u;
+      tmem_st16(tS + pc, pp);
+      tmem_st16(tDP + pc, dd);
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[b]);
+    }
+    // every MMA done: add the accumulators (row = key, columns of half hc)
+    const bool done = __all_sync(0xffffffffu, mbar_wait(done_bar, 0, abort_flag, st));
+    if (ok && done) {
+      tc_fence_after();
+      float* dvp = a.dv32 + ((size_t)key_tok * a.Hkv + g) * D;
+      float* dkp = a.dk32 + ((size_t)key_tok * a.Hkv + g) * D;
+#pragma unroll 1
+      for (int cc = hc * (D / 2); cc < (hc + 1) * (D / 2); cc += 32) {
+        uint32_t va[32], vb[32];
+        tmem_ld32(tmem + lane_off + C::kColV + cc, va);
+        tmem_ld32(tmem + lane_off + C::kColK + cc, vb);
+        tc_wait_ld();
+        if (key_ok) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            atomicAdd(dvp + cc + e, __uint_as_float(va[e]));
+            atomicAdd(dkp + cc + e, __uint_as_float(vb[e]) * a.scale);
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  // after an abort: every MMA was committed to done_bar by the MMA warp, and
+  // the K / V load may still be in flight; wait for both (bounded)
+  if (threadIdx.x == 0) {
+    mbar_wait_teardown(done_bar, 0, 500000000ull);
+    mbar_wait_teardown(kv_bar, 0, 200000000ull);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
 // dQ of one 128-row tile.
 //   routed: blockIdx.x = item over the pass's 128-row items (tile_off);
 //           keys = all of the bucket's block
