@@ -300,6 +300,20 @@ __device__ __forceinline__ float tile_exp_to_p(uint32_t tS, int r, float scale_l
   return ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
 }
 
+// 32-byte global store (one instruction for eight 32-bit words; the address
+// must be 32-byte aligned).  Used for the partials, whose workspace rows are
+// 32-byte aligned: each lane writes its own row, so the store width halves
+// the requests of a scattered epilogue (measured 10 % faster at 256-key
+// blocks).  The caller's o is only required to be 16-byte aligned and keeps
+// 16-byte stores.
+__device__ __forceinline__ void st_global_v8(void* p, uint32_t a0, uint32_t a1, uint32_t a2,
+                                             uint32_t a3, uint32_t a4, uint32_t a5,
+                                             uint32_t a6, uint32_t a7) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a0),
+               "r"(a1), "r"(a2), "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+               : "memory");
+}
+
 template <int D, int MODE, int QBUFS>
 __global__ void __launch_bounds__(352, 1)
     attn2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -693,24 +707,30 @@ __global__ void __launch_bounds__(352, 1)
           // |O| <= max |v|; 8x finer than bf16, for the second rounding
           // the merge adds before the final bf16 output.  Scaled by 2^-S,
           // which keeps it below the fp16 maximum whatever the bf16 input.
-          uint4* d4 = reinterpret_cast<uint4*>(dsth + c4 * 32);
           const float ps = inv * pscale;
 #pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            const float* f = reinterpret_cast<const float*>(&ov[q8 * 8]);
-            d4[q8] = make_uint4(pack_half2(f[0] * ps, f[1] * ps),
-                                pack_half2(f[2] * ps, f[3] * ps),
-                                pack_half2(f[4] * ps, f[5] * ps),
-                                pack_half2(f[6] * ps, f[7] * ps));
+          for (int q16 = 0; q16 < 2; ++q16) {
+            const float* f = reinterpret_cast<const float*>(&ov[q16 * 16]);
+            st_global_v8(dsth + c4 * 32 + q16 * 16, pack_half2(f[0] * ps, f[1] * ps),
+                         pack_half2(f[2] * ps, f[3] * ps), pack_half2(f[4] * ps, f[5] * ps),
+                         pack_half2(f[6] * ps, f[7] * ps), pack_half2(f[8] * ps, f[9] * ps),
+                         pack_half2(f[10] * ps, f[11] * ps), pack_half2(f[12] * ps, f[13] * ps),
+                         pack_half2(f[14] * ps, f[15] * ps));
           }
         } else if (kind == 2) {
-          float4* d4 = reinterpret_cast<float4*>(dst32 + c4 * 32);
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4)
-            d4[q4] = make_float4(__uint_as_float(ov[4 * q4]) * inv,
-                                 __uint_as_float(ov[4 * q4 + 1]) * inv,
-                                 __uint_as_float(ov[4 * q4 + 2]) * inv,
-                                 __uint_as_float(ov[4 * q4 + 3]) * inv);
+          for (int q8 = 0; q8 < 4; ++q8) {
+            const uint32_t* u = &ov[8 * q8];
+            st_global_v8(dst32 + c4 * 32 + q8 * 8,
+                         __float_as_uint(__uint_as_float(u[0]) * inv),
+                         __float_as_uint(__uint_as_float(u[1]) * inv),
+                         __float_as_uint(__uint_as_float(u[2]) * inv),
+                         __float_as_uint(__uint_as_float(u[3]) * inv),
+                         __float_as_uint(__uint_as_float(u[4]) * inv),
+                         __float_as_uint(__uint_as_float(u[5]) * inv),
+                         __float_as_uint(__uint_as_float(u[6]) * inv),
+                         __float_as_uint(__uint_as_float(u[7]) * inv));
+          }
         }
       }
       if (kind != 0) *lse_dst = lse_val;

@@ -611,15 +611,18 @@ __global__ void __launch_bounds__(352, 1)
 
   if (warp >= 9) {
     // ------------------------------------------------------------ row gather
-    const int r = (warp - 9) * 32 + lane;  // row of the tile
-    bool ok = true;
-    int n = 0;
-    for (; n < ntiles && ok; ++n) {
-      const int sg = n % ST;
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(&rows_empty[sg], ((n / ST) & 1) ^ 1, abort_flag, st));
-      if (!ok) break;
+    // Warp gw gathers rows 32 gw .. 32 gw + 31 of each tile.  Lane l reads the
+    // entry of row 32 gw + l (one tile ahead); the copies then take RPI rows
+    // per instruction, CPR consecutive 16-byte chunks of a row per group of
+    // lanes, so one instruction reads a few contiguous rows instead of 32
+    // scattered pieces.
+    constexpr int CPR = D / 8;     // 16-byte chunks per row
+    constexpr int RPI = 32 / CPR;  // rows per instruction
+    const int rbase = (warp - 9) * 32;
+    auto row_of = [&](int n) -> BwRow {
       BwRow x{-1, 0};
+      if (n >= ntiles) return x;
+      const int r = rbase + lane;
       if (MODE == kBwRouted) {
         x = bw_row_routed(a, g, e0 + (int64_t)n * RT, e1, r);
       } else {
@@ -630,18 +633,35 @@ __global__ void __launch_bounds__(352, 1)
           x.h = g * a.G + hh;
         }
       }
-      const int64_t t = x.t < 0 ? 0 : x.t;  // a missing row reads token 0 (finite); P = 0
-      const __nv_bfloat16* qs = a.q + ((size_t)t * a.Hq + (x.t < 0 ? 0 : x.h)) * D;
-      const __nv_bfloat16* gs = a.dO + ((size_t)t * a.Hq + (x.t < 0 ? 0 : x.h)) * D;
+      return x;
+    };
+    bool ok = true;
+    int n = 0;
+    BwRow xn = row_of(0);
+    for (; n < ntiles && ok; ++n) {
+      const int sg = n % ST;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&rows_empty[sg], ((n / ST) & 1) ^ 1, abort_flag, st));
+      if (!ok) break;
+      const BwRow x = xn;
+      xn = row_of(n + 1);  // next tile's entry, in flight while this one copies
+      // a missing row reads token 0, head 0 (finite); its P is forced to 0
+      const int64_t my_t = x.t < 0 ? 0 : x.t;
+      const int my_h = x.t < 0 ? 0 : x.h;
       unsigned char* dq_ = smem + C::kOffQ + sg * C::kRowTile;
       unsigned char* ddo = smem + C::kOffDO + sg * C::kRowTile;
+      const int c = lane % CPR;
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
-        const uint32_t off = (uint32_t)(c >> 3) * C::kRowHalf + sw128_offset(r, c & 7);
-        cp_async_16(dq_ + off, qs + c * 8);
-        cp_async_16(ddo + off, gs + c * 8);
+      for (int i = 0; i < 32 / RPI; ++i) {
+        const int rl = i * RPI + lane / CPR;  // row within this warp's 32
+        const int64_t t = __shfl_sync(0xffffffffu, my_t, rl);
+        const int h = __shfl_sync(0xffffffffu, my_h, rl);
+        const size_t src = ((size_t)t * a.Hq + h) * D + c * 8;
+        const uint32_t off = (uint32_t)(c >> 3) * C::kRowHalf + sw128_offset(rbase + rl, c & 7);
+        cp_async_16(dq_ + off, a.q + src);
+        cp_async_16(ddo + off, a.dO + src);
       }
-      float2* d = sdl + sg * RT + r;
+      float2* d = sdl + sg * RT + rbase + lane;
       if (x.t >= 0)
         cp_async_8(d, a.dl + (size_t)x.t * a.Hq + x.h);
       else
