@@ -11,11 +11,13 @@
 // chose past block J (the forward's bucket of (kv head, J), gathered rows)
 // meet J's keys; for the own part, each block's rows meet the same block's
 // keys, causally.  Two kernels per part, each recomputing S and P:
-//   bw_kv_kernel  one CTA per (bucket or own block, 128-key tile): loops over
-//                 the rows in tiles of 128; S^T = K Q^T and dP^T = V dO^T
-//                 (keys on the TMEM lanes), P^T and dS^T packed as bf16 over
-//                 them, which are the TMEM A operands of dV += P^T dO and
-//                 dK += dS^T Q, accumulated in TMEM
+//   bw_kv2_kernel one CTA per (bucket or own block, 128-key tile), warp
+//                 roles: it loops over the rows in tiles of 64; S^T = K Q^T and
+//                 dP^T = V dO^T (keys on the TMEM lanes, two tiles' worth of
+//                 TMEM), P^T and dS^T packed as bf16 over them, which are the
+//                 TMEM A operands of dV += P^T dO and dK += dS^T Q, accumulated
+//                 in TMEM; the elementwise pass of a tile overlaps the MMAs
+//                 of its neighbours
 //   bw_q_kernel   one CTA per tile of 128 rows (gathered or own): loops over
 //                 the block's key tiles; dS packed as bf16 into TMEM is the A
 //                 operand of dQ += dS K
@@ -24,9 +26,7 @@
 // K / V tiles likewise.
 // Gradients are summed in fp32 buffers with atomic adds (each key gets one
 // routed and one own contribution per kv head; each row one per chosen
-// block) and converted to bf16 at the end.  Within a CTA, a tile's MMAs and
-// elementwise work run in turn; the next tile's operands (bw_kv: gathered
-// Q / dO rows, bw_q: K / V) load into a second buffer meanwhile.
+// block) and converted to bf16 at the end.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -60,19 +60,15 @@ template <int D>
 struct BwCfg {
   static constexpr int kHalf = kTileM * 128;   // 128 rows x 64 columns bf16
   static constexpr int kTile = kTileM * D * 2; // one [128][D] bf16 tile
-  // Six tile slots.  bw_kv: K, V, then two (Q, dO) buffers.  bw_q: K, V,
-  // Q, dO, a second (K, V) buffer and a third K buffer (kOffK3).
+  // bw_q: K, V, Q, dO, a second (K, V) buffer (slots 4, 5) and a third K
+  // buffer (kOffK3).
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kTile;
   static constexpr int kOffQ = kOffV + kTile;
   static constexpr int kOffDO = kOffQ + kTile;
   static constexpr int kOffX = kOffDO + kTile;   // slot 4
   static constexpr int kOffY = kOffX + kTile;    // slot 5
-  static constexpr int kOffDL = kOffY + kTile;   // bw_kv: float2 (D, lse2) [2][128 rows]
-  static constexpr int kOffBar = kOffDL + 2 * kTileM * 8;
-  static constexpr int kSmemBytes = kOffBar + 64 + 1024;
-  // bw_q: a seventh slot (a third K buffer) from kOffDL on, then its barriers
-  static constexpr int kOffK3 = kOffDL;
+  static constexpr int kOffK3 = kOffY + kTile;   // a seventh slot, then the barriers
   static constexpr int kOffBarQ = kOffK3 + kTile;
   static constexpr int kSmemBytesQ = kOffBarQ + 64 + 1024;
   static_assert(kSmemBytesQ <= 232448, "bw_q shared memory beyond the per-CTA limit");
@@ -196,298 +192,10 @@ __device__ __forceinline__ void bw_p_ds(const BwArgs& a, uint32_t tS, uint32_t t
   }
 }
 
-// P^T and dS^T of a key lane for half hc of one 128-row tile (dK / dV
-// kernel, keys on TMEM lanes): reads S^T and dP^T over the half's row
-// columns, with each row's (D, lse2) from shared memory (a row past the
-// tile's end has lse2 = +inf, so its P is 0).  Masks the lane when its key
-// is past the block end (key_ok false) and, when causal, rows before the
-// key's token.  Packs P^T as bf16 pairs from column kColS and dS^T from
-// kColDP (see bw_packed_col).
-__device__ __forceinline__ void bw_pt_dst(const BwArgs& a, uint32_t tS, uint32_t tDP,
-                                          const float2* __restrict__ dl, bool key_ok,
-                                          bool causal, int64_t key_tok, int64_t row_tok0,
-                                          int hc) {
-#pragma unroll 1
-  for (int i = 0; i < 2; ++i) {
-    const int c0 = hc ? 96 - 32 * i : 32 * i;
-    uint32_t sv[32], dv[32];
-    tmem_ld32(tS + c0, sv);
-    tmem_ld32(tDP + c0, dv);
-    tc_wait_ld();
-    uint32_t pp[16], dd[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float4 l = *reinterpret_cast<const float4*>(dl + c0 + 2 * e);  // D, lse2 of 2 rows
-      float p2[2], d2[2];
-#pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        const int c = c0 + 2 * e + x;
-        bool keep = key_ok;
-        if (causal) keep = keep && (key_tok <= row_tok0 + c);
-        const float Dc = x ? l.z : l.x, lc = x ? l.w : l.y;
-        const float p =
-            keep ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + x]), a.scale_log2, -lc)) : 0.f;
-        p2[x] = p;
-        d2[x] = p * (__uint_as_float(dv[2 * e + x]) - Dc);
-      }
-      pp[e] = pack_bf16x2(p2[0], p2[1]);
-      dd[e] = pack_bf16x2(d2[0], d2[1]);
-    }
-    const uint32_t pc = (hc ? 64 : 0) + (c0 >> 1);
-    tmem_st16(tS + pc, pp);
-    tmem_st16(tDP + pc, dd);
-  }
-}
-
 // Bounded wait of the whole CTA on an mbarrier phase.
 __device__ __forceinline__ bool bw_wait(uint64_t* bar, uint32_t parity,
                                         volatile uint32_t* abort_flag, uint32_t* st) {
   return __syncthreads_and(mbar_wait(bar, parity, abort_flag, st) ? 1 : 0) != 0;
-}
-
-// dK / dV of one 128-key tile, with the keys on the TMEM lanes.
-//   routed: blockIdx.x = f * KT + kt over the pass's buckets f = u * NB + J;
-//           rows = the bucket's entries
-//   own:    blockIdx.x = f * KT + kt over (unit, block); rows = the block's
-//           tokens at or after the key tile, for every q head of the unit
-// Per 128-row tile n: S^T = K Q^T and dP^T = V dO^T (M = keys, N = rows) go
-// to TMEM; the four warps (thread = key) form P^T and dS^T = P^T (dP^T - D)
-// and pack them as bf16 over the columns they came from; dV += P^T dO and
-// dK += dS^T Q take them as TMEM A operands (K = rows), with dO and Q as
-// MN-major B operands.  The rows are gathered into two (Q, dO) buffers: tile
-// n + 1 is gathered while tile n computes, once the dV / dK MMAs of tile
-// n - 1, the last readers of its buffer, are done.  The tensor pipe runs the
-// S^T MMA of tile n + 1 after the dV / dK MMAs of tile n that read the
-// columns it overwrites.  Eight warps: two per TMEM lane quarter, each taking
-// half of the row columns (see bw_packed_col); two threads gather each row.
-template <int D, int MODE>
-__global__ void __launch_bounds__(256, 1)
-    bw_kv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                 const BwArgs a) {
-  using C = BwCfg<D>;
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* kv_bar = bars + 0;   // K / V tile landed
-  uint64_t* s_bar = bars + 1;    // S^T / dP^T MMAs of a row tile done
-  uint64_t* mma_bar = bars + 2;  // dV / dK MMAs of a row tile (and every earlier MMA) done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
-  volatile uint32_t* abort_flag = tmem_slot + 1;
-  const int warp = threadIdx.x >> 5;
-  const int r = threadIdx.x & 127;  // TMEM lane (key) and gathered row of this thread
-  const int hc = warp >> 2;         // column half (elementwise) / row half (gather)
-
-  const int NB = a.P.totals[0];
-  const int KT = a.B / kTileN;
-  const int64_t f = blockIdx.x / KT;
-  const int kt = (int)(blockIdx.x % KT);
-  if (f >= (int64_t)a.nu * NB) return;
-  const int u = (int)(f / NB), J = (int)(f % NB);
-  const int g = a.u0 + u;
-  const int blen = a.P.blk_len[J];
-  const int nkeys = min(kTileN, blen - kt * kTileN);
-  if (nkeys <= 0) return;
-  const int64_t kstart = (int64_t)a.P.blk_tok[J] + (int64_t)kt * kTileN;
-  int64_t e0 = 0, e1 = 0;
-  int ntiles;
-  int own_tiles = 0;  // own: row tiles per q head
-  if (MODE == kBwRouted) {
-    e0 = a.entry_off[f];
-    e1 = a.entry_off[f + 1];
-    ntiles = (int)((e1 - e0 + kTileM - 1) / kTileM);
-  } else {
-    own_tiles = (blen - kt * kTileN + kTileM - 1) / kTileM;  // tiles from the key tile on
-    ntiles = own_tiles * a.G;
-  }
-  if (ntiles == 0) return;
-
-  if (threadIdx.x == 0) {
-    mbar_init(kv_bar, 1);
-    mbar_init(s_bar, 1);
-    mbar_init(mma_bar, 1);
-    *abort_flag = 0u;
-    fence_barrier_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  unsigned char* sK = smem + C::kOffK;
-  unsigned char* sV = smem + C::kOffV;
-  auto sQb = [&](int b) { return smem + (b ? C::kOffX : C::kOffQ); };
-  auto sDOb = [&](int b) { return smem + (b ? C::kOffY : C::kOffDO); };
-  float2* sdl = reinterpret_cast<float2*>(smem + C::kOffDL);  // [2][128] (D, lse2)
-  uint32_t* st = a.status;
-
-  // row r of row tile n: routed -> the bucket's entry, read one tile ahead
-  // (entry_of) so that no gather waits on it; own -> a token of the block at
-  // or after the key tile, for q head n / own_tiles
-  auto entry_of = [&](int n) -> uint2 {
-    uint2 en = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);  // no entry
-    if (MODE == kBwRouted) {
-      const int64_t e = e0 + (int64_t)n * kTileM + r;
-      if (e < e1) en = a.entries[e];
-    }
-    return en;
-  };
-  auto row_of = [&](int n, uint2 en) -> BwRow {
-    BwRow x{-1, 0};
-    if (MODE == kBwRouted) {
-      if (en.y != 0xFFFFFFFFu) {
-        const int hh = (int)(en.y & 0xFFFFu);
-        if (en.x < (uint32_t)a.L.T && hh < a.G) {
-          x.t = en.x;
-          x.h = g * a.G + hh;
-        } else {
-          atomicOr(a.status, MOBA_DEV_BAD_INDEX);
-        }
-      }
-    } else {
-      const int hh = n / own_tiles, qt = n % own_tiles;
-      const int64_t t = kstart + (int64_t)qt * kTileM + r;
-      if (t < (int64_t)a.P.blk_tok[J] + blen) {
-        x.t = t;
-        x.h = g * a.G + hh;
-      }
-    }
-    return x;
-  };
-  // gather row tile n into buffer n & 1, all by cp.async in one group: the
-  // q / dO rows and (D, lse2); a missing row gets (0, +inf), so its P is 0
-  uint2 ent = entry_of(0);
-  auto gather = [&](int n) {
-    const BwRow x = row_of(n, ent);
-    if (n + 1 < ntiles) ent = entry_of(n + 1);
-    if (hc == 0) {
-      float2* d = sdl + (n & 1) * kTileM + r;
-      if (x.t >= 0)
-        cp_async_8(d, a.dl + (size_t)x.t * a.Hq + x.h);
-      else
-        *d = make_float2(0.f, __int_as_float(0x7f800000));
-    }
-    bw_load_row<D>(a, x, r, hc, sQb(n & 1), sDOb(n & 1));
-    cp_async_commit();
-  };
-
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(kv_bar, 2 * C::kTile);
-#pragma unroll
-    for (int hx = 0; hx < D / 64; ++hx) {
-      tma_load_3d(sK + hx * C::kHalf, &tm_k, kv_bar, hx * 64, g, (int)kstart);
-      tma_load_3d(sV + hx * C::kHalf, &tm_v, kv_bar, hx * 64, g, (int)kstart);
-    }
-  }
-  gather(0);
-  bool ok = bw_wait(kv_bar, 0, abort_flag, st);
-
-  const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
-  constexpr uint32_t idS = idesc_bf16_f32(kTileN, kTileM, false, false);  // M = keys, N = rows
-  constexpr uint32_t idG = idesc_bf16_f32(kTileN, D, false, true);        // A in TMEM, B MN-major
-  const bool key_ok = r < nkeys;
-  const int64_t key_tok = kstart + r;
-  uint32_t ns = 0, nm = 0;  // s_bar and mma_bar phases
-  for (int n = 0; n < ntiles && ok; ++n) {
-    const int b = n & 1;
-    const uint32_t sQa = smem_u32(sQb(b)), sDOa = smem_u32(sDOb(b));
-    cp_async_wait_group<0>();  // this thread's rows of tile n (the only group pending)
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (warp == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * C::kHalf + (kk & 3) * 32;
-        tc_mma_ss_warp(tmem + C::kColS, sdesc_kmajor_sw128(sKa + off),
-                       sdesc_kmajor_sw128(sQa + off), idS, kk > 0 ? 1u : 0u);
-        tc_mma_ss_warp(tmem + C::kColDP, sdesc_kmajor_sw128(sVa + off),
-                       sdesc_kmajor_sw128(sDOa + off), idS, kk > 0 ? 1u : 0u);
-      }
-      tc_commit_warp(s_bar);
-    }
-    ++ns;
-    if (n + 1 < ntiles) {
-      // buffer (n + 1) & 1 was last read by the dV / dK MMAs of tile n - 1
-      if (n > 0) {
-        ok = bw_wait(mma_bar, (nm - 1) & 1, abort_flag, st);
-        if (!ok) break;
-      }
-      gather(n + 1);
-    }
-    ok = bw_wait(s_bar, (ns - 1) & 1, abort_flag, st);
-    if (!ok) break;
-    tc_fence_after();
-    int64_t row_tok0 = 0;
-    if (MODE == kBwOwn) row_tok0 = kstart + (int64_t)(n % own_tiles) * kTileM;
-    bw_pt_dst(a, tmem + lane_off + C::kColS, tmem + lane_off + C::kColDP, sdl + b * kTileM,
-              key_ok, MODE == kBwOwn, key_tok, row_tok0, hc);
-    tc_wait_st();
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kTileM / 16; ++kk) {  // K = rows, 16 per step
-        const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-        tc_mma_ts_warp(tmem + C::kColA, tmem + C::kColS + bw_packed_col(kk),
-                       sdesc_mnmajor_sw128(sDOa + kk * 2048, C::kHalf, 1024), idG, acc);
-        tc_mma_ts_warp(tmem + C::kColB, tmem + C::kColDP + bw_packed_col(kk),
-                       sdesc_mnmajor_sw128(sQa + kk * 2048, C::kHalf, 1024), idG, acc);
-      }
-      tc_commit_warp(mma_bar);
-    }
-    ++nm;
-  }
-  if (ok) {  // every dV / dK MMA done
-    if (warp == 0) tc_commit_warp(mma_bar);
-    ok = bw_wait(mma_bar, nm & 1, abort_flag, st);
-    ++nm;
-  }
-  if (ok) {
-    tc_fence_after();
-    // row r of the accumulators = key kstart + r, columns of half hc; every
-    // lane takes part in the (warp-collective) TMEM loads, only lanes of real
-    // keys store
-    float* dv = a.dv32 + ((size_t)(kstart + r) * a.Hkv + g) * D;
-    float* dk = a.dk32 + ((size_t)(kstart + r) * a.Hkv + g) * D;
-#pragma unroll 1
-    for (int c0 = hc * (D / 2); c0 < (hc + 1) * (D / 2); c0 += 32) {
-      uint32_t va[32], vb[32];
-      tmem_ld32(tmem + lane_off + C::kColA + c0, va);
-      tmem_ld32(tmem + lane_off + C::kColB + c0, vb);
-      tc_wait_ld();
-      if (key_ok) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          atomicAdd(dv + c0 + e, __uint_as_float(va[e]));
-          atomicAdd(dk + c0 + e, __uint_as_float(vb[e]) * a.scale);
-        }
-      }
-    }
-  }
-  // teardown: after an abort, row gathers, the K / V load and MMAs may still
-  // be in flight; wait for them (bounded) before TMEM and shared memory go
-  cp_async_wait_all();
-  if (!ok && threadIdx.x == 0) mbar_wait_teardown(kv_bar, 0, 200000000ull);
-  if (warp == 0) {
-    tc_commit_warp(mma_bar);  // arrives once every MMA of this CTA has completed
-    if (threadIdx.x == 0) {
-      mbar_wait_teardown(mma_bar, nm & 1, 500000000ull);
-      if (ns > 0) mbar_wait_teardown(s_bar, (ns - 1) & 1, 500000000ull);
-    }
-    __syncwarp();
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
-  }
 }
 
 // ---------------------------------------------------------------- dK / dV, warp-specialised
