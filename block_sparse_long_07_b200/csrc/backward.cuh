@@ -58,23 +58,8 @@ struct BwArgs {
 
 template <int D>
 struct BwCfg {
-  static constexpr int kHalf = kTileM * 128;   // 128 rows x 64 columns bf16
-  static constexpr int kTile = kTileM * D * 2; // one [128][D] bf16 tile
-  // bw_q: K, V, Q, dO, a second (K, V) buffer (slots 4, 5) and a third K
-  // buffer (kOffK3).
-  static constexpr int kOffK = 0;
-  static constexpr int kOffV = kOffK + kTile;
-  static constexpr int kOffQ = kOffV + kTile;
-  static constexpr int kOffDO = kOffQ + kTile;
-  static constexpr int kOffX = kOffDO + kTile;   // slot 4
-  static constexpr int kOffY = kOffX + kTile;    // slot 5
-  static constexpr int kOffK3 = kOffY + kTile;   // a seventh slot, then the barriers
-  static constexpr int kOffBarQ = kOffK3 + kTile;
-  static constexpr int kSmemBytesQ = kOffBarQ + 64 + 1024;
-  static_assert(kSmemBytesQ <= 232448, "bw_q shared memory beyond the per-CTA limit");
-  static constexpr uint32_t kTmemCols = 512;
-  // TMEM columns
-  static constexpr uint32_t kColS = 0, kColDP = 128, kColA = 256, kColB = 256 + D;
+  static constexpr int kHalf = kTileM * 128;    // 128 rows x 64 columns bf16
+  static constexpr int kTile = kTileM * D * 2;  // one [128][D] bf16 tile
 };
 
 // (D = dO . O, lse * log2 e) per (token, q head), one warp per row.
@@ -146,56 +131,6 @@ __device__ __forceinline__ void bw_load_row(const BwArgs& a, BwRow x, int r, int
     cp_async_16(sQ + off, qs + c * 8);
     cp_async_16(sDO + off, gs + c * 8);
   }
-}
-
-// Eight warps share the elementwise work of a 128 x 128 score tile: warp w
-// takes TMEM lanes 32 * (w % 4) .. + 31 and columns 64 * (w / 4) .. + 63.
-// Its 32-column chunks are packed as bf16 pairs over columns it has already
-// read: column c of the tile lands in packed column c / 2 (c < 64) or
-// 64 + c / 2 (c >= 64; that half walks its chunks from the top down).  The
-// MMA over tile columns 16 kk .. 16 kk + 15 reads its A operand there.
-__host__ __device__ constexpr uint32_t bw_packed_col(int kk) {
-  return kk < 4 ? 8u * kk : 64u + 8u * kk;
-}
-
-// dS of a row for its half hc of key tile [kbase, kbase + 128) (dQ kernel,
-// rows on TMEM lanes): reads S and dP from TMEM (this thread's lane), masks
-// keys >= nkeys and, when causal, keys after the row's token, and packs dS
-// as bf16 pairs into tOut: key column c at tOut + c / 2.
-template <int D>
-__device__ __forceinline__ void bw_p_ds(const BwArgs& a, uint32_t tS, uint32_t tDP,
-                                        uint32_t tOut, float lse2, float Dr, int nkeys,
-                                        bool causal, int64_t trow, int64_t kbase, int hc) {
-#pragma unroll 1
-  for (int i = 0; i < 2; ++i) {
-    const int c0 = 64 * hc + 32 * i;
-    uint32_t sv[32], dv[32];
-    tmem_ld32(tS + c0, sv);
-    tmem_ld32(tDP + c0, dv);
-    tc_wait_ld();
-    uint32_t dd[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      float d2[2];
-#pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        const int j = c0 + 2 * e + x;
-        bool keep = j < nkeys;
-        if (causal) keep = keep && (kbase + j <= trow);
-        const float p =
-            keep ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + x]), a.scale_log2, -lse2)) : 0.f;
-        d2[x] = p * (__uint_as_float(dv[2 * e + x]) - Dr);
-      }
-      dd[e] = pack_bf16x2(d2[0], d2[1]);
-    }
-    tmem_st16(tOut + (c0 >> 1), dd);
-  }
-}
-
-// Bounded wait of the whole CTA on an mbarrier phase.
-__device__ __forceinline__ bool bw_wait(uint64_t* bar, uint32_t parity,
-                                        volatile uint32_t* abort_flag, uint32_t* st) {
-  return __syncthreads_and(mbar_wait(bar, parity, abort_flag, st) ? 1 : 0) != 0;
 }
 
 // ---------------------------------------------------------------- dK / dV, warp-specialised
@@ -535,44 +470,61 @@ __global__ void __launch_bounds__(352, 1)
   }
 }
 
-// dQ of one 128-row tile.
-//   routed: blockIdx.x = item over the pass's 128-row items (tile_off);
-//           keys = all of the bucket's block
-//   own:    blockIdx.x = (unit head, query tile); keys = the tile's block up
-//           to and including the tile's own 128 keys (causal)
-// K tiles have three buffers and V tiles two; dS is packed into two TMEM
-// regions from kColB on, which S, dP and the dQ accumulator leave free.  The
-// MMAs of tile kt go S / dP(kt), then dQ(kt - 1), so the elementwise pass of
-// tile kt overlaps the dQ MMA of tile kt - 1.  Tile kt + 1 loads at the start
-// of iteration kt: its K slot was last read by dQ(kt - 2), which ran during
-// the previous elementwise pass, and its V slot by dP(kt - 1).  The commit
-// after S / dP(kt) covers dQ(kt - 2), the last reader of the dS region that
-// tile kt writes.  Eight warps: two per
-// TMEM lane quarter (row), each taking half of the key columns (see
-// bw_packed_col); two threads gather each row.
+// ---------------------------------------------------------------- dQ, warp-specialised
+// One CTA per 128-row tile, as bw_q_kernel, with each 128-key K / V tile taken
+// in two halves of 64 keys so that TMEM holds two halves' S / dP next to the
+// dQ accumulator: the elementwise pass of half m runs while the tensor core
+// computes dQ of half m - 1 and S / dP of half m + 1.
+//   warps 0-7  gather the tile's q / dO rows (two threads a row), then the
+//              elementwise pass: warp w takes rows 32 (w % 4) .. + 31 (its TMEM
+//              lane quarter) and keys 32 (w / 4) .. + 31 of the half; dS is
+//              packed as bf16 over the S columns it read (see bw2_packed_col)
+//   warp  8    TMEM allocation and the MMA issue
+//   warp  9    K / V tiles by TMA into a two-stage ring
+template <int D>
+struct BwQ2Cfg {
+  static constexpr int kStages = 2;
+  static constexpr int kTile = kTileM * D * 2;          // one [128][D] bf16 tile
+  static constexpr int kHalf = kTileM * 128;            // 128 rows x 64 columns bf16
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffDO = kOffQ + kTile;
+  static constexpr int kOffK = kOffDO + kTile;          // [stage]
+  static constexpr int kOffV = kOffK + kStages * kTile; // [stage]
+  static constexpr int kOffBar = kOffV + kStages * kTile;
+  static constexpr int kNumBars = 2 * kStages + 2 + 2 + 1;
+  static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
+  static constexpr int kThreads = 320;
+  static constexpr uint32_t kColS = 0;       // [2] x 64 columns: S, then packed dS
+  static constexpr uint32_t kColDP = 128;    // [2] x 64 columns: dP
+  static constexpr uint32_t kColQ = 256;     // dQ accumulator
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kSmemBytes <= 232448, "bw_q2 shared memory beyond the per-CTA limit");
+};
+
 template <int D, int MODE>
-__global__ void __launch_bounds__(256, 1)
-    bw_q_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                const BwArgs a) {
-  using C = BwCfg<D>;
+__global__ void __launch_bounds__(320, 1)
+    bw_q2_kernel(const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const BwArgs a) {
+  using C = BwQ2Cfg<D>;
+  constexpr int ST = C::kStages;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBarQ);
-  uint64_t* kv_full = bars + 0;  // [3] K / V of tile t landed (K slot t % 3)
-  uint64_t* mma_bar = bars + 3;  // S / dP MMAs of a tile (and all earlier MMAs) done
-  uint64_t* dq_bar = bars + 4;   // dQ MMA of a tile done: its K slot is free
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* kv_full = bars;            // [ST] K / V tile landed
+  uint64_t* kv_empty = kv_full + ST;   // [ST] its last dQ MMA done
+  uint64_t* s_full = kv_empty + ST;    // [2] S / dP of a half in TMEM
+  uint64_t* p_full = s_full + 2;       // [2] dS of a half packed
+  uint64_t* done_bar = p_full + 2;     // every MMA done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  const int warp = threadIdx.x >> 5;
-  const int r = threadIdx.x & 127;  // TMEM lane and row of this thread
-  const int hc = warp >> 2;         // column half (elementwise) / row half (gather)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = threadIdx.x & 127;  // row of this thread (warps 0-7)
+  const int hc = (warp >> 2) & 1;   // key half within a 64-key half (elementwise) / row half (gather)
   const int NB = a.P.totals[0];
 
-  int g, J;
-  int nkt;             // key tiles to visit
-  int64_t kblock;      // first token of the block
-  int blen;
+  int g, J, nkt, blen;
+  int64_t kblock;
   BwRow x{-1, 0};
   if (MODE == kBwRouted) {
     const int64_t nitems = a.tile_off[a.nu * NB];
@@ -582,12 +534,11 @@ __global__ void __launch_bounds__(256, 1)
     J = f % NB;
     g = a.u0 + u;
     const int64_t e0 = a.entry_off[f] + (int64_t)(blockIdx.x - a.tile_off[f]) * kTileM;
-    x = bw_row_routed(a, g, e0, a.entry_off[f + 1], r);
+    if (warp < 8) x = bw_row_routed(a, g, e0, a.entry_off[f + 1], r);
     blen = a.P.blk_len[J];
     kblock = a.P.blk_tok[J];
     nkt = (blen + kTileN - 1) / kTileN;
   } else {
-    // (head of the unit, query tile)
     const int NQT = a.P.totals[1];
     const int64_t idx = blockIdx.x;
     const int hl = (int)(idx / NQT);
@@ -602,161 +553,180 @@ __global__ void __launch_bounds__(256, 1)
     blen = a.P.blk_len[J];
     kblock = a.P.blk_tok[J];
     nkt = (int)((p0 - (int64_t)i * a.B) / kTileN) + 1;  // up to the diagonal tile
-    if (p0 + r < len) {
+    if (warp < 8 && p0 + r < len) {
       x.t = st0 + p0 + r;
       x.h = g * a.G + hl % a.G;
     }
   }
+  const int nh = 2 * nkt;  // 64-key halves
 
   if (threadIdx.x == 0) {
-    mbar_init(&kv_full[0], 1);
-    mbar_init(&kv_full[1], 1);
-    mbar_init(&kv_full[2], 1);
-    mbar_init(mma_bar, 1);
-    mbar_init(dq_bar, 1);
+    for (int q = 0; q < ST; ++q) {
+      mbar_init(&kv_full[q], 1);
+      mbar_init(&kv_empty[q], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 8);
+    }
+    mbar_init(done_bar, 1);
     *abort_flag = 0u;
     fence_barrier_init();
   }
-  if (warp == 0) {
+  if (warp == 8) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
+  }
+  unsigned char* sQ = smem + C::kOffQ;
+  unsigned char* sDO = smem + C::kOffDO;
+  float lse2 = __int_as_float(0x7f800000), Dr = 0.f;
+  if (warp < 8) {
+    if (x.t >= 0) {
+      const float2 v = a.dl[(size_t)x.t * a.Hq + x.h];
+      Dr = v.x;
+      lse2 = v.y;
+    }
+    bw_load_row<D>(a, x, r, hc, sQ, sDO);
+    cp_async_wait_all();
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  auto sKb = [&](int t) {  // K slot of tile t
-    const int m = t % 3;
-    return smem + (m == 0 ? C::kOffK : (m == 1 ? C::kOffX : C::kOffK3));
-  };
-  auto sVb = [&](int t) { return smem + ((t & 1) ? C::kOffY : C::kOffV); };  // V slot
-  unsigned char* sQ = smem + C::kOffQ;
-  unsigned char* sDO = smem + C::kOffDO;
   uint32_t* st = a.status;
-  int nloaded = 0, nused = 0;  // K / V tiles loaded (thread 0) and consumed
 
-  auto load_kv = [&](int kt) {  // thread 0
-    uint64_t* bar = &kv_full[kt % 3];
-    const int64_t kb = kblock + (int64_t)kt * kTileN;
-    mbar_arrive_expect_tx(bar, 2 * C::kTile);
+  if (warp == 9) {
+    // ------------------------------------------------------------ K / V producer
+    if (lane == 0) {
+      int t = 0;
+      bool ok = true;
+      for (; t < nkt && ok; ++t) {
+        const int sg = t % ST;
+        ok = mbar_wait(&kv_empty[sg], ((t / ST) & 1) ^ 1, abort_flag, st);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&kv_full[sg], 2 * C::kTile);
+        const int64_t kb = kblock + (int64_t)t * kTileN;
 #pragma unroll
-    for (int hx = 0; hx < D / 64; ++hx) {
-      tma_load_3d(sKb(kt) + hx * C::kHalf, &tm_k, bar, hx * 64, g, (int)kb);
-      tma_load_3d(sVb(kt) + hx * C::kHalf, &tm_v, bar, hx * 64, g, (int)kb);
+        for (int hx = 0; hx < D / 64; ++hx) {
+          tma_load_3d(smem + C::kOffK + sg * C::kTile + hx * C::kHalf, &tm_k, &kv_full[sg],
+                      hx * 64, g, (int)kb);
+          tma_load_3d(smem + C::kOffV + sg * C::kTile + hx * C::kHalf, &tm_v, &kv_full[sg],
+                      hx * 64, g, (int)kb);
+        }
+      }
+      if (!ok) {  // loads still in flight: the last ST issued
+        for (int b = 0; b < ST && b < t; ++b) {
+          const int l = t - 1 - b;
+          mbar_wait_teardown(&kv_full[l % ST], (l / ST) & 1, 200000000ull);
+        }
+      }
     }
-    ++nloaded;
-  };
-  if (threadIdx.x == 0) load_kv(0);  // overlaps the row gather below
-
-  float lse2 = __int_as_float(0x7f800000), Dr = 0.f;
-  if (x.t >= 0) {
-    const float2 v = a.dl[(size_t)x.t * a.Hq + x.h];
-    Dr = v.x;
-    lse2 = v.y;
-  }
-  bw_load_row<D>(a, x, r, hc, sQ, sDO);
-  cp_async_wait_all();
-  fence_proxy_async_smem();
-  __syncthreads();
-
-  const uint32_t sQa = smem_u32(sQ), sDOa = smem_u32(sDO);
-  constexpr uint32_t idS = idesc_bf16_f32(kTileM, kTileN, false, false);
-  constexpr uint32_t idQ = idesc_bf16_f32(kTileM, D, false, true);
-  bool ok = true;
-  uint32_t nm = 0, ndq = 0;  // mma_bar and dq_bar phases
-  // dQ(t) += dS(t) K(t): A = dS(t) packed in region t & 1, B = K(t)
-  auto issue_dq = [&](int t) {  // warp 0
-    const uint32_t kb = smem_u32(sKb(t));
-    const uint32_t ds = tmem + C::kColB + 64u * (uint32_t)(t & 1);
-#pragma unroll
-    for (int kk = 0; kk < kTileN / 16; ++kk)  // K = keys, 16 per step
-      tc_mma_ts_warp(tmem + C::kColA, ds + kk * 8,
-                     sdesc_mnmajor_sw128(kb + kk * 2048, C::kHalf, 1024), idQ,
-                     (t > 0 || kk > 0) ? 1u : 0u);
-    tc_commit_warp(dq_bar);
-  };
-  for (int kt = 0; kt < nkt && ok; ++kt) {
-    const int64_t kbase = kblock + (int64_t)kt * kTileN;
-    const int nkeys = min(kTileN, blen - kt * kTileN);
-    const uint32_t sKa = smem_u32(sKb(kt)), sVa = smem_u32(sVb(kt));
-    if (threadIdx.x == 0 && kt + 1 < nkt) {
-      // K slot of tile kt + 1 was last read by dQ(kt - 2); its V slot by dP(kt - 1)
-      const bool free_ok = kt < 2 || mbar_wait(dq_bar, (uint32_t)(kt - 2) & 1u, abort_flag, st);
-      if (free_ok) load_kv(kt + 1);
-    }
-    __syncwarp();  // warp 0 reconverges before the block-wide wait
-    ok = bw_wait(&kv_full[kt % 3], (uint32_t)(kt / 3) & 1u, abort_flag, st);
-    if (!ok) break;
-    ++nused;
-    if (warp == 0) {
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issue
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, st));
+    };
+    constexpr uint32_t idS = idesc_bf16_f32(kTileM, 64, false, false);  // M = rows, N = keys
+    constexpr uint32_t idQ = idesc_bf16_f32(kTileM, D, false, true);    // A in TMEM, B MN-major
+    const uint32_t sQa = smem_u32(sQ), sDOa = smem_u32(sDO);
+    const uint32_t sKa = smem_u32(smem + C::kOffK), sVa = smem_u32(smem + C::kOffV);
+    // dQ += dS(m) K(m): A = dS packed in buffer m % 2, B = the half's 64 keys x D
+    auto dq_mmas = [&](int m) -> bool {
+      const int b = m & 1, t = m >> 1, hf = m & 1, sg = t % ST;
+      if (!wait(&p_full[b], (m >> 1) & 1)) return false;
       tc_fence_after();
+      const uint32_t kb = sKa + sg * C::kTile + hf * 8192;  // keys 64 hf .. : 64 rows of 128 B
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)  // K = keys, 16 per step
+        tc_mma_ts_warp(tmem + C::kColQ, tmem + C::kColS + 64u * b + bw2_packed_col(kk),
+                       sdesc_mnmajor_sw128(kb + kk * 2048, C::kHalf, 1024), idQ,
+                       (m > 0 || kk > 0) ? 1u : 0u);
+      if (hf == 1) tc_commit_warp(&kv_empty[sg]);  // the tile's last reader
+      return true;
+    };
+    bool ok = true;
+    int m = 0;
+    for (; m < nh && ok; ++m) {
+      const int b = m & 1, t = m >> 1, hf = m & 1, sg = t % ST;
+      if (hf == 0 && !(ok = wait(&kv_full[sg], (t / ST) & 1))) break;
+      tc_fence_after();
+      const uint32_t kb = sKa + sg * C::kTile + hf * 8192;
+      const uint32_t vb = sVa + sg * C::kTile + hf * 8192;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * C::kHalf + (kk & 3) * 32;
-        tc_mma_ss_warp(tmem + C::kColS, sdesc_kmajor_sw128(sQa + off),
-                       sdesc_kmajor_sw128(sKa + off), idS, kk > 0 ? 1u : 0u);
-        tc_mma_ss_warp(tmem + C::kColDP, sdesc_kmajor_sw128(sDOa + off),
-                       sdesc_kmajor_sw128(sVa + off), idS, kk > 0 ? 1u : 0u);
+        tc_mma_ss_warp(tmem + C::kColS + 64u * b, sdesc_kmajor_sw128(sQa + off),
+                       sdesc_kmajor_sw128(kb + off), idS, kk > 0 ? 1u : 0u);
+        tc_mma_ss_warp(tmem + C::kColDP + 64u * b, sdesc_kmajor_sw128(sDOa + off),
+                       sdesc_kmajor_sw128(vb + off), idS, kk > 0 ? 1u : 0u);
       }
-      tc_commit_warp(mma_bar);
-      if (kt > 0) issue_dq(kt - 1);
+      tc_commit_warp(&s_full[b]);
+      if (m > 0 && !(ok = dq_mmas(m - 1))) break;
     }
-    if (kt > 0) ++ndq;
-    ok = bw_wait(mma_bar, nm & 1, abort_flag, st);
-    ++nm;
-    if (!ok) break;
-    tc_fence_after();
-    bw_p_ds<D>(a, tmem + lane_off + C::kColS, tmem + lane_off + C::kColDP,
-               tmem + lane_off + C::kColB + 64u * (uint32_t)(kt & 1), lse2, Dr, nkeys,
-               MODE == kBwOwn, x.t, kbase, hc);
-    tc_wait_st();
-    tc_fence_before();
-    __syncthreads();
-  }
-  if (ok) {  // the last tile's dQ MMA
-    if (warp == 0) {
+    if (ok && m > 0) ok = dq_mmas(m - 1);
+    tc_commit_warp(done_bar);  // every MMA of this CTA (also after an abort)
+  } else {
+    // ------------------------------------------------------------ elementwise (warps 0-7)
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    bool ok = true;
+    for (int m = 0; m < nh && ok; ++m) {
+      const int b = m & 1, t = m >> 1, hf = m & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (m >> 1) & 1, abort_flag, st));
+      if (!ok) break;
       tc_fence_after();
-      issue_dq(nkt - 1);
-    }
-    ++ndq;
-  }
-  if (ok) {  // every dQ MMA done
-    if (warp == 0) tc_commit_warp(mma_bar);
-    ok = bw_wait(mma_bar, nm & 1, abort_flag, st);
-    ++nm;
-  }
-  if (ok) {
-    tc_fence_after();
-#pragma unroll 1
-    for (int c0 = hc * (D / 2); c0 < (hc + 1) * (D / 2); c0 += 32) {
-      uint32_t va[32];
-      tmem_ld32(tmem + lane_off + C::kColA + c0, va);
+      const int c0 = 32 * hc;  // this warp's keys within the half
+      const uint32_t tS = tmem + lane_off + C::kColS + 64u * b;
+      const uint32_t tDP = tmem + lane_off + C::kColDP + 64u * b;
+      uint32_t sv[32], dv[32];
+      tmem_ld32(tS + c0, sv);
+      tmem_ld32(tDP + c0, dv);
       tc_wait_ld();
-      if (x.t >= 0) {
-        float* dq = a.dq32 + ((size_t)x.t * a.Hq + x.h) * D + c0;
+      const int key0 = t * kTileN + hf * 64 + c0;  // key of column 0 within the block
+      const int64_t ktok0 = kblock + key0;
+      uint32_t dd[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) atomicAdd(dq + e, __uint_as_float(va[e]) * a.scale);
+      for (int e = 0; e < 16; ++e) {
+        float d2[2];
+#pragma unroll
+        for (int xx = 0; xx < 2; ++xx) {
+          const int j = 2 * e + xx;
+          bool keep = key0 + j < blen;
+          if (MODE == kBwOwn) keep = keep && (ktok0 + j <= x.t);
+          const float p =
+              keep ? ex2_approx(fmaf(__uint_as_float(sv[j]), a.scale_log2, -lse2)) : 0.f;
+          d2[xx] = p * (__uint_as_float(dv[j]) - Dr);
+        }
+        dd[e] = pack_bf16x2(d2[0], d2[1]);
+      }
+      tmem_st16(tS + (hc ? 32u : 0u), dd);
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[b]);
+    }
+    const bool done = __all_sync(0xffffffffu, mbar_wait(done_bar, 0, abort_flag, st));
+    if (ok && done) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = hc * (D / 2); cc < (hc + 1) * (D / 2); cc += 32) {
+        uint32_t va[32];
+        tmem_ld32(tmem + lane_off + C::kColQ + cc, va);
+        tc_wait_ld();
+        if (x.t >= 0) {
+          float* dq = a.dq32 + ((size_t)x.t * a.Hq + x.h) * D + cc;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) atomicAdd(dq + e, __uint_as_float(va[e]) * a.scale);
+        }
       }
     }
   }
-  // teardown: after an abort, loads and MMAs may still be in flight
-  if (!ok && threadIdx.x == 0) {
-    // at most two loads are unconsumed (tiles nused and nused + 1)
-    for (int t = nused; t < nloaded; ++t)
-      mbar_wait_teardown(&kv_full[t % 3], (uint32_t)(t / 3) & 1u, 200000000ull);
-  }
-  if (warp == 0) {
-    tc_commit_warp(mma_bar);  // arrives once every MMA of this CTA has completed
-    if (threadIdx.x == 0) {
-      mbar_wait_teardown(mma_bar, nm & 1, 500000000ull);
-      if (ndq > 0) mbar_wait_teardown(dq_bar, (ndq - 1u) & 1u, 500000000ull);
-    }
-    __syncwarp();
-  }
+
+  // ------------------------------------------------------------ teardown
+  if (threadIdx.x == 0) mbar_wait_teardown(done_bar, 0, 500000000ull);
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }

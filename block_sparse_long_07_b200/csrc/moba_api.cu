@@ -976,7 +976,6 @@ moba_status backward_passes(const Problem& pr, const void* q, const void* k, con
                             const void* o, const float* lse, const void* dO, const int32_t* sel,
                             void* dq, void* dk, void* dv, const BwWs& b, int nu_max,
                             cudaStream_t st) {
-  using C = BwCfg<D>;
   const Ws& w = b.w;
   SeqLayout L{pr.cu, pr.nseq, pr.N, pr.T};
   MOBA_TRY(run_plan(pr, w, st));
@@ -1003,10 +1002,11 @@ moba_status backward_passes(const Problem& pr, const void* q, const void* k, con
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C2::kSmemBytes));
   MOBA_CUDA(cudaFuncSetAttribute(bw_kv2_kernel<D, kBwOwn>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C2::kSmemBytes));
-  MOBA_CUDA(cudaFuncSetAttribute(bw_q_kernel<D, kBwRouted>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytesQ));
-  MOBA_CUDA(cudaFuncSetAttribute(bw_q_kernel<D, kBwOwn>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytesQ));
+  using C3 = BwQ2Cfg<D>;
+  MOBA_CUDA(cudaFuncSetAttribute(bw_q2_kernel<D, kBwRouted>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C3::kSmemBytes));
+  MOBA_CUDA(cudaFuncSetAttribute(bw_q2_kernel<D, kBwOwn>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C3::kSmemBytes));
   BwArgs a;
   memset(&a, 0, sizeof a);
   a.q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -1051,7 +1051,7 @@ moba_status backward_passes(const Problem& pr, const void* q, const void* k, con
       {
         const int64_t items = (int64_t)nu * pr.T * pr.G * np / kTileM + (int64_t)nu * pr.NBmax;
         Timed tm(kKBwQ, st);
-        bw_q_kernel<D, kBwRouted><<<(unsigned)items, 256, C::kSmemBytesQ, st>>>(tk, tv, a);
+        bw_q2_kernel<D, kBwRouted><<<(unsigned)items, C3::kThreads, C3::kSmemBytes, st>>>(tk, tv, a);
         MOBA_CUDA(cudaGetLastError());
       }
     }
@@ -1063,8 +1063,8 @@ moba_status backward_passes(const Problem& pr, const void* q, const void* k, con
     }
     {
       Timed tm(kKBwQ, st);
-      bw_q_kernel<D, kBwOwn><<<(unsigned)(nu * pr.G * pr.NQTmax), 256, C::kSmemBytesQ, st>>>(
-          tk, tv, a);
+      bw_q2_kernel<D, kBwOwn>
+          <<<(unsigned)(nu * pr.G * pr.NQTmax), C3::kThreads, C3::kSmemBytes, st>>>(tk, tv, a);
       MOBA_CUDA(cudaGetLastError());
     }
   }
