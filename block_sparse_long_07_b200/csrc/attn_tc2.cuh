@@ -88,8 +88,11 @@ struct Attn2Cfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = kOffQ + kQBufs * kQBytes;
   static constexpr int kOffBar = kOffKV + kStages * kKVBytes;
-  static constexpr int kNumBars = 2 * kQBufs + 2 * kStages + 2 + 2 + 2 + 2 + 1 + 2;
-  static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
+  static constexpr int kNumBars = 3 * kQBufs + 2 * kStages + 2 + 2 + 2 + 2 + 1 + 2;
+  static constexpr int kOffItem = kOffBar + kNumBars * 8 + 16;  // [QB] item descriptors
+  static constexpr int kItemBytes = 96;
+  static constexpr int kSmemBytes = kOffItem + kQBufs * kItemBytes + 1024;
+  static_assert(kSmemBytes <= 232448, "attention shared memory beyond the per-CTA limit");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, false, true);
@@ -319,6 +322,7 @@ __global__ void __launch_bounds__(352, 1)
     attn2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const AttnArgs a, int pair_own) {
   using C = Attn2Cfg<D, QBUFS>;
+  static_assert(sizeof(Item) <= C::kItemBytes, "item descriptor slot too small");
   constexpr int ST = C::kStages;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -337,7 +341,9 @@ __global__ void __launch_bounds__(352, 1)
   uint64_t* o_free = o_full + 2;        // [2] epilogue has read O_X
   uint64_t* td_bar = o_free + 2;
   uint64_t* p_half = td_bar + 1;        // [2] first 64 keys of P_X in TMEM
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(p_half + 2);
+  uint64_t* desc_free = p_half + 2;     // [QB] every softmax warp has read the item descriptor
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(desc_free + QB);
+  Item* sItem = reinterpret_cast<Item*>(smem + C::kOffItem);  // [QB], with the Q buffers
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -345,6 +351,7 @@ __global__ void __launch_bounds__(352, 1)
     for (int b = 0; b < QB; ++b) {
       mbar_init(&q_full[b], 1);
       mbar_init(&q_empty[b], 1);
+      mbar_init(&desc_free[b], 8);  // one elected arrival per softmax warp
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -388,7 +395,9 @@ __global__ void __launch_bounds__(352, 1)
         if (MODE != kRouted) {
           const int qb = lt % QB;
           ok = mbar_wait(&q_empty[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
+          if (ok) ok = mbar_wait(&desc_free[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
           if (!ok) break;
+          sItem[qb] = it;  // published by the arrive below, with the Q tile
           mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
 #pragma unroll
           for (int x = 0; x < 2; ++x)
@@ -438,8 +447,10 @@ __global__ void __launch_bounds__(352, 1)
         const Item it = item_info<MODE>(a, w, pair_own);
         const int qb = lt % QB;
         ok = mbar_wait(&q_empty[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
+        if (ok) ok = mbar_wait(&desc_free[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
+        if (lane == 0) sItem[qb] = it;  // published by q_full, with the rows
         const int nrows = it.rows_x[0] + it.rows_x[1];
         const int c = lane % CPR;
 #pragma unroll
@@ -552,10 +563,10 @@ __global__ void __launch_bounds__(352, 1)
       return true;
     };
     for (int64_t w = first; w < items && ok; w += step, ++lt) {
-      const Item it = item_info<MODE>(a, w, pair_own);
       const int qb = lt % QB;
       const uint32_t qbase = sQa + qb * C::kQBytes;
       if (!(ok = wait(&q_full[qb], (lt / QB) & 1))) break;
+      const Item it = sItem[qb];  // written by the Q buffer's filler
       const uint32_t ks = kv_it % ST;
       if (!(ok = wait(&kv_full[ks], (kv_it / ST) & 1))) break;
       ++kv_it;
@@ -598,8 +609,25 @@ __global__ void __launch_bounds__(352, 1)
     const float pscale = (MODE == kRouted) ? exp2f(-(float)partial_scale_log2(a.status[1])) : 1.f;
     uint32_t ns = 0, no = 0;
     bool ok = true;
-    for (int64_t w = first; w < items && ok; w += step) {
-      const int nkv = item_info<MODE>(a, w, pair_own).nkv_x[x];
+    // The item comes from its descriptor in shared memory, published with
+    // the Q buffer (a clock trace put the global-memory decode at 3-5 k
+    // cycles per item here, twice per item); the fields the epilogue needs
+    // are kept in registers, since the descriptor's slot is refilled once
+    // every softmax warp has read it.
+    uint32_t lt = 0;
+    for (int64_t w = first; w < items && ok; w += step, ++lt) {
+      const int qb = lt % QB;
+      ok = mbar_wait(&q_full[qb], (lt / QB) & 1, abort_flag, st);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const int nkv = sItem[qb].nkv_x[x];
+      const int rows_x = sItem[qb].rows_x[x];
+      const int it_u = sItem[qb].u, it_h = sItem[qb].h, it_seq = sItem[qb].seq;
+      const int it_own = sItem[qb].own_block;
+      const int64_t it_e0 = sItem[qb].e0, it_q0 = sItem[qb].qstart;
+      const int64_t it_s0 = sItem[qb].seq_start;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&desc_free[qb]);
       if (nkv == 0) continue;
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < nkv; ++j) {
@@ -647,8 +675,7 @@ __global__ void __launch_bounds__(352, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const Item it = item_info<MODE>(a, w, pair_own);
-      const bool valid = r < it.rows_x[x];
+      const bool valid = r < rows_x;
       const float inv = 1.f / l_run;
       const float lse2 = m_run + lg2_approx(l_run);
       // destination of this row
@@ -660,11 +687,11 @@ __global__ void __launch_bounds__(352, 1)
       float lse_val = lse2;
       if (valid) {
         if (MODE == kRouted) {
-          const uint2 e = a.entries[it.e0 + x * kTileM + r];
+          const uint2 e = a.entries[it_e0 + x * kTileM + r];
           const int hh = (int)(e.y & 0xFFFFu), sl = (int)(e.y >> 16);
           if (e.x < (uint32_t)a.L.T && hh < a.G && sl < a.topk - 1) {
             const int64_t prow =
-                (((int64_t)it.u * a.L.T + e.x) * a.G + hh) * (a.topk - 1) + sl;
+                (((int64_t)it_u * a.L.T + e.x) * a.G + hh) * (a.topk - 1) + sl;
             kind = 1;
             dsth = a.part_O + prow * D;
             lse_dst = a.part_lse + prow;
@@ -672,15 +699,15 @@ __global__ void __launch_bounds__(352, 1)
             atomicOr(a.status, MOBA_DEV_BAD_INDEX);
           }
         } else {
-          const int64_t t = it.qstart + (int64_t)x * kTileM + r;
-          const bool final_row = (MODE == kDense) || a.topk == 1 || it.own_block == 0;
+          const int64_t t = it_q0 + (int64_t)x * kTileM + r;
+          const bool final_row = (MODE == kDense) || a.topk == 1 || it_own == 0;
           if (final_row) {
             kind = 3;
-            dst16 = a.o + ((size_t)t * a.Hq + it.h) * D;
-            lse_dst = a.lse + row_index(a.R, it.seq, it.h, t - it.seq_start, t);
+            dst16 = a.o + ((size_t)t * a.Hq + it_h) * D;
+            lse_dst = a.lse + row_index(a.R, it_seq, it_h, t - it_s0, t);
             lse_val = lse2 * 0.6931471805599453f;
           } else {
-            const int64_t prow = ((int64_t)it.u * a.L.T + t) * a.G + (it.h % a.G);
+            const int64_t prow = ((int64_t)it_u * a.L.T + t) * a.G + (it_h % a.G);
             kind = 2;
             dst32 = a.own_O + prow * D;
             lse_dst = a.own_lse + prow;
