@@ -21,7 +21,7 @@
 //   warps 4-7   softmax + epilogue of sub-tile 1
 //   warp  8     TMA producer: Q tiles (own/dense) and the K/V ring
 //   warp  9     TMEM allocation and MMA issue (one elected lane per MMA)
-//   warp 10     Q row gather for routed items (cp.async into swizzled smem)
+//   warp 10     Q row gather for routed items (TMA four-row gathers)
 // TMEM (512 columns): S_X at 128*X (fp32 scores; after the softmax the first
 // 64 columns hold P_X as packed bf16, and on the first tile of an own/dense
 // block columns 64..95 hold the residual weights of rows 0..63), O_X at
@@ -375,7 +375,7 @@ __global__ void __launch_bounds__(352, 1)
   if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
-    if (MODE != kRouted) tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_q);
   }
   tc_fence_before();
   __syncthreads();
@@ -438,11 +438,15 @@ __global__ void __launch_bounds__(352, 1)
     }
   } else if (warp == 10) {
     // ------------------------------------------------------------ Q gather
+    // Routed items: the rows the bucket entries name, four rows per TMA
+    // gather from q viewed as [T*Hq][D] (one-row boxes of 64 columns,
+    // 128-B swizzle), so that the TMA engine, not this warp, carries the
+    // latency of 256 scattered rows.  Lane l brings rows 4l..4l+3 of each
+    // sub-tile; rows past the item's end repeat its first row (their
+    // results are never stored).
     if (MODE == kRouted) {
       uint32_t lt = 0;
       bool ok = true;
-      constexpr int CPR = D / 8;     // 16-B chunks per row
-      constexpr int RPI = 32 / CPR;  // rows per warp instruction
       for (int64_t w = first; w < items && ok; w += step, ++lt) {
         const Item it = item_info<MODE>(a, w, pair_own);
         const int qb = lt % QB;
@@ -450,38 +454,38 @@ __global__ void __launch_bounds__(352, 1)
         if (ok) ok = mbar_wait(&desc_free[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        if (lane == 0) sItem[qb] = it;  // published by q_full, with the rows
         const int nrows = it.rows_x[0] + it.rows_x[1];
-        const int c = lane % CPR;
+        int ys[2][4];
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          uint2 ent[4];
+        for (int x = 0; x < 2; ++x)
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            int r = x * kTileM + lane + 32 * m;
+          for (int i = 0; i < 4; ++i) {
+            int r = x * kTileM + 4 * lane + i;
             if (r >= nrows) r = 0;
-            ent[m] = a.entries[it.e0 + r];
-          }
-          unsigned char* qdst = sQ + qb * C::kQBytes + x * C::kSubQBytes + (c >> 3) * C::kHalfBytes;
-#pragma unroll
-          for (int i = 0; i < kTileM / RPI; ++i) {
-            const int r = i * RPI + lane / CPR;
-            const int m = (i * RPI) / 32;
-            const uint2 e = make_uint2(__shfl_sync(0xffffffffu, ent[m].x, r & 31),
-                                       __shfl_sync(0xffffffffu, ent[m].y, r & 31));
+            const uint2 e = a.entries[it.e0 + r];
             const bool good = e.x < (uint32_t)a.L.T && (e.y & 0xFFFFu) < (uint32_t)a.G;
             const int hq = it.g * a.G + (good ? (int)(e.y & 0xFFFFu) : 0);
-            const __nv_bfloat16* src =
-                a.q + ((size_t)(good ? e.x : 0u) * a.Hq + hq) * D + c * 8;
-            cp_async_16(qdst + sw128_offset(r, c & 7), src);
+            ys[x][i] = (int)((int64_t)(good ? e.x : 0u) * a.Hq + hq);
           }
+        if (lane == 0) {
+          sItem[qb] = it;  // published by q_full, with the rows
+          mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
         }
-        cp_async_wait_all();
-        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&q_full[qb]);
+#pragma unroll
+        for (int x = 0; x < 2; ++x)
+#pragma unroll
+          for (int hx = 0; hx < D / 64; ++hx)
+            tma_gather4(sQ + qb * C::kQBytes + x * C::kSubQBytes + hx * C::kHalfBytes +
+                            lane * 4 * 128,
+                        &tm_q, &q_full[qb], hx * 64, ys[x][0], ys[x][1], ys[x][2], ys[x][3]);
       }
-      cp_async_wait_all();
+      if (!ok && lane == 0) {  // let the gathers in flight land before the CTA exits
+        for (uint32_t b = 0; b < (lt < (uint32_t)QB ? lt : (uint32_t)QB); ++b) {
+          const uint32_t l = lt - 1 - b;
+          mbar_wait_teardown(&q_full[l % QB], (l / QB) & 1, 200000000ull);
+        }
+      }
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
@@ -629,6 +633,10 @@ __global__ void __launch_bounds__(352, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&desc_free[qb]);
       if (nkv == 0) continue;
+      // routed: this row's bucket entry, loaded now so that its latency
+      // hides behind the softmax instead of opening the epilogue
+      uint2 ent = make_uint2(0xFFFFFFFFu, 0u);
+      if (MODE == kRouted && r < rows_x) ent = a.entries[it_e0 + x * kTileM + r];
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < nkv; ++j) {
         ok = mbar_wait(&s_full[x], ns & 1, abort_flag, st);
@@ -687,7 +695,7 @@ __global__ void __launch_bounds__(352, 1)
       float lse_val = lse2;
       if (valid) {
         if (MODE == kRouted) {
-          const uint2 e = a.entries[it_e0 + x * kTileM + r];
+          const uint2 e = ent;
           const int hh = (int)(e.y & 0xFFFFu), sl = (int)(e.y >> 16);
           if (e.x < (uint32_t)a.L.T && hh < a.G && sl < a.topk - 1) {
             const int64_t prow =

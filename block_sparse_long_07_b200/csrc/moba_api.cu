@@ -279,6 +279,22 @@ bool make_tmap(CUtensorMap* m, const void* ptr, int H, int64_t T, int D) {
   return r == CUDA_SUCCESS;
 }
 
+// [T][H][D] bf16 viewed as rows (x = D, y = T*H), box 64 x 1, 128-B swizzle:
+// the routed kernel's four-row gathers of (token, head) rows.  Row indices
+// are int32, so T*H must stay below 2^31 (forward_setup checks).
+bool make_tmap_rows(CUtensorMap* m, const void* ptr, int64_t rows, int D) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -588,14 +604,16 @@ moba_status gate_impl(const Problem& pr, const void* q, const void* k, int32_t* 
 // Attention arguments and tensor maps of one forward call.
 struct FwdCtx {
   CUtensorMap tq, tk, tv;
+  CUtensorMap tq_rows;  // q as [T*Hq][D] rows (routed gathers)
   AttnArgs a;
 };
 
 template <int D>
 moba_status forward_setup(const Problem& pr, const void* q, const void* k, const void* v,
                           void* o, float* lse, const Ws& w, FwdCtx* c) {
+  if (pr.T * pr.Hq >= (int64_t)INT32_MAX) return MOBA_ERR_UNSUPPORTED;  // int32 q row index
   if (!make_tmap(&c->tq, q, pr.Hq, pr.T, D) || !make_tmap(&c->tk, k, pr.Hkv, pr.T, D) ||
-      !make_tmap(&c->tv, v, pr.Hkv, pr.T, D))
+      !make_tmap(&c->tv, v, pr.Hkv, pr.T, D) || !make_tmap_rows(&c->tq_rows, q, pr.T * pr.Hq, D))
     return MOBA_ERR_CUDA;
   AttnArgs& a = c->a;
   memset(&a, 0, sizeof a);
@@ -638,7 +656,7 @@ moba_status forward_one_pass(const Problem& pr, FwdCtx& c, const Ws& w, const in
     }
     MOBA_CUDA(cudaGetLastError());
     MOBA_TRY(launch_scatter(pr, w, sel, u0, nu, st));
-    MOBA_TRY((launch_attn<D, kRouted>(c.tq, c.tk, c.tv, a, 1, st)));
+    MOBA_TRY((launch_attn<D, kRouted>(c.tq_rows, c.tk, c.tv, a, 1, st)));
   }
   MOBA_TRY((launch_attn<D, kOwn>(c.tq, c.tk, c.tv, a, pr.B % (2 * kTileM) == 0 ? 1 : 0, st)));
   if (pr.topk > 1) {
