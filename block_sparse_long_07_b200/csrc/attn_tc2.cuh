@@ -126,15 +126,11 @@ __device__ __forceinline__ int64_t num_items2(const AttnArgs& a, int pair_own) {
   return per_head * HP;
 }
 
-// Work item w of the launch.  For own/dense modes the items of one head are
-// query-tile pairs numbered through P.totals[2] / P.pair_off (see plan).
-template <int MODE>
-__device__ __forceinline__ Item item_info(const AttnArgs& a, int64_t w, int pair_own) {
+// Routed item w of bucket f (tile_off[f] <= w < tile_off[f + 1]).
+__device__ __forceinline__ Item routed_item(const AttnArgs& a, int64_t w, int f) {
   Item it;
-  if (MODE == kRouted) {
+  {
     const int NB = a.P.totals[0];
-    const int M = a.nu * NB;
-    const int f = upper_index(a.tile_off, M + 1, w);
     const int u = f / NB, J = f % NB;
     const int64_t row0 = (w - a.tile_off[f]) * (int64_t)(2 * kTileM);
     const int64_t cnt = (int64_t)a.entry_off[f + 1] - a.entry_off[f];
@@ -153,6 +149,34 @@ __device__ __forceinline__ Item item_info(const AttnArgs& a, int64_t w, int pair
     it.seq_start = 0;
     it.own_block = 0;
     it.e0 = a.entry_off[f] + row0;
+  }
+  return it;
+}
+
+// Bucket of routed item w, searched forward by a whole warp from the bucket
+// f of an earlier item (a CTA visits its items in increasing order): lane l
+// tests bound f + 1 + l, 32 bounds per load.  Falls back to a binary search
+// after two rounds.
+__device__ __forceinline__ int routed_bucket_after(const AttnArgs& a, int64_t w, int f, int lane) {
+  const int M = a.nu * a.P.totals[0];
+#pragma unroll 1
+  for (int round = 0; round < 2; ++round, f += 32) {
+    const int i = f + 1 + lane;
+    const bool past = (i >= M) || ((int64_t)a.tile_off[i] > w);
+    const unsigned b = __ballot_sync(0xffffffffu, past);
+    if (b) return f + __ffs(b) - 1;
+  }
+  return f + upper_index(a.tile_off + f, M + 1 - f, w);
+}
+
+// Work item w of the launch.  For own/dense modes the items of one head are
+// query-tile pairs numbered through P.totals[2] / P.pair_off (see plan).
+template <int MODE>
+__device__ __forceinline__ Item item_info(const AttnArgs& a, int64_t w, int pair_own) {
+  Item it;
+  if (MODE == kRouted) {
+    const int M = a.nu * a.P.totals[0];
+    it = routed_item(a, w, upper_index(a.tile_off, M + 1, w));
   } else {
     const int HP = (MODE == kOwn) ? a.nu * a.G : a.Hq;
     const bool paired = (MODE == kDense) || pair_own;
@@ -447,8 +471,11 @@ __global__ void __launch_bounds__(352, 1)
     if (MODE == kRouted) {
       uint32_t lt = 0;
       bool ok = true;
+      int f = -1;  // bucket of the previous item
       for (int64_t w = first; w < items && ok; w += step, ++lt) {
-        const Item it = item_info<MODE>(a, w, pair_own);
+        f = (f < 0) ? upper_index(a.tile_off, a.nu * a.P.totals[0] + 1, w)
+                    : routed_bucket_after(a, w, f, lane);
+        const Item it = routed_item(a, w, f);
         const int qb = lt % QB;
         ok = mbar_wait(&q_empty[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
         if (ok) ok = mbar_wait(&desc_free[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
