@@ -126,47 +126,67 @@ __device__ __forceinline__ int64_t num_items2(const AttnArgs& a, int pair_own) {
   return per_head * HP;
 }
 
-// Routed item w of bucket f (tile_off[f] <= w < tile_off[f + 1]).
-__device__ __forceinline__ Item routed_item(const AttnArgs& a, int64_t w, int f) {
+// Routed item w of bucket f, from the bucket's first item tile_lo, its
+// entry range [e_lo, e_hi) and its block's first token.
+__device__ __forceinline__ Item routed_fill(const AttnArgs& a, int64_t w, int f, int tile_lo,
+                                            int e_lo, int e_hi, int blk_tok) {
   Item it;
-  {
-    const int NB = a.P.totals[0];
-    const int u = f / NB, J = f % NB;
-    const int64_t row0 = (w - a.tile_off[f]) * (int64_t)(2 * kTileM);
-    const int64_t cnt = (int64_t)a.entry_off[f + 1] - a.entry_off[f];
-    const int64_t left = cnt - row0;
-    it.u = u;
-    it.g = a.u0 + u;
-    it.h = -1;
-    it.kstart = a.P.blk_tok[J];
-    it.nkv = a.B / kTileN;
-    it.rows_x[0] = (int)min((int64_t)kTileM, left);
-    it.rows_x[1] = (int)max((int64_t)0, min((int64_t)kTileM, left - kTileM));
-    it.nkv_x[0] = it.nkv;
-    it.nkv_x[1] = it.rows_x[1] > 0 ? it.nkv : 0;
-    it.qstart = 0;
-    it.seq = 0;
-    it.seq_start = 0;
-    it.own_block = 0;
-    it.e0 = a.entry_off[f] + row0;
-  }
+  const int NB = a.P.totals[0];
+  const int64_t row0 = (w - tile_lo) * (int64_t)(2 * kTileM);
+  const int64_t left = (int64_t)(e_hi - e_lo) - row0;
+  it.u = f / NB;
+  it.g = a.u0 + it.u;
+  it.h = -1;
+  it.kstart = blk_tok;
+  it.nkv = a.B / kTileN;
+  it.rows_x[0] = (int)min((int64_t)kTileM, left);
+  it.rows_x[1] = (int)max((int64_t)0, min((int64_t)kTileM, left - kTileM));
+  it.nkv_x[0] = it.nkv;
+  it.nkv_x[1] = it.rows_x[1] > 0 ? it.nkv : 0;
+  it.qstart = 0;
+  it.seq = 0;
+  it.seq_start = 0;
+  it.own_block = 0;
+  it.e0 = e_lo + row0;
   return it;
 }
 
-// Bucket of routed item w, searched forward by a whole warp from the bucket
-// f of an earlier item (a CTA visits its items in increasing order): lane l
-// tests bound f + 1 + l, 32 bounds per load.  Falls back to a binary search
-// after two rounds.
-__device__ __forceinline__ int routed_bucket_after(const AttnArgs& a, int64_t w, int f, int lane) {
-  const int M = a.nu * a.P.totals[0];
+// Routed item w of bucket f (tile_off[f] <= w < tile_off[f + 1]).
+__device__ __forceinline__ Item routed_item(const AttnArgs& a, int64_t w, int f) {
+  return routed_fill(a, w, f, a.tile_off[f], a.entry_off[f], a.entry_off[f + 1],
+                     a.P.blk_tok[f % a.P.totals[0]]);
+}
+
+// Routed item w for a whole warp, searched forward from the bucket f of an
+// earlier item (a CTA visits its items in increasing order): lane l reads
+// bucket f + l's bounds, entry range and block start in one round of loads,
+// and the first bucket whose end lies past w is the item's.  Falls back to
+// a binary search after two rounds.  Returns the bucket.
+__device__ __forceinline__ int routed_next(const AttnArgs& a, int64_t w, int f, int lane,
+                                           Item& it) {
+  const int NB = a.P.totals[0];
+  const int M = a.nu * NB;
 #pragma unroll 1
   for (int round = 0; round < 2; ++round, f += 32) {
-    const int i = f + 1 + lane;
-    const bool past = (i >= M) || ((int64_t)a.tile_off[i] > w);
-    const unsigned b = __ballot_sync(0xffffffffu, past);
-    if (b) return f + __ffs(b) - 1;
+    const int i = f + lane;
+    const bool in = i < M;
+    const int64_t end = in ? (int64_t)a.tile_off[i + 1] : INT64_MAX;
+    const int lo = in ? a.tile_off[i] : 0;
+    const int e_lo = in ? a.entry_off[i] : 0;
+    const int e_hi = in ? a.entry_off[i + 1] : 0;
+    const int bt = in ? a.P.blk_tok[i % NB] : 0;
+    const unsigned b = __ballot_sync(0xffffffffu, end > w);
+    if (b) {
+      const int L = __ffs(b) - 1;
+      it = routed_fill(a, w, f + L, __shfl_sync(0xffffffffu, lo, L),
+                       __shfl_sync(0xffffffffu, e_lo, L), __shfl_sync(0xffffffffu, e_hi, L),
+                       __shfl_sync(0xffffffffu, bt, L));
+      return f + L;
+    }
   }
-  return f + upper_index(a.tile_off + f, M + 1 - f, w);
+  f += upper_index(a.tile_off + f, M + 1 - f, w);
+  it = routed_item(a, w, f);
+  return f;
 }
 
 // Work item w of the launch.  For own/dense modes the items of one head are
@@ -471,29 +491,49 @@ __global__ void __launch_bounds__(352, 1)
     if (MODE == kRouted) {
       uint32_t lt = 0;
       bool ok = true;
-      int f = -1;  // bucket of the previous item
-      for (int64_t w = first; w < items && ok; w += step, ++lt) {
-        f = (f < 0) ? upper_index(a.tile_off, a.nu * a.P.totals[0] + 1, w)
-                    : routed_bucket_after(a, w, f, lane);
-        const Item it = routed_item(a, w, f);
-        const int qb = lt % QB;
-        ok = mbar_wait(&q_empty[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
-        if (ok) ok = mbar_wait(&desc_free[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        const int nrows = it.rows_x[0] + it.rows_x[1];
-        int ys[2][4];
+      // The next item and its entries are looked up before this item's
+      // gathers are issued, so that the entry loads land while the TMA
+      // requests queue (a clock trace put the lookup and the entry loads at
+      // 3 k cycles, the gather issue at 8-9 k, for a 256-row item).
+      int f = -1;  // bucket of the item looked up last
+      Item nxt;
+      uint2 nent[2][4];
+      auto lookup = [&](int64_t w2) {
+        if (f < 0) {
+          f = upper_index(a.tile_off, a.nu * a.P.totals[0] + 1, w2);
+          nxt = routed_item(a, w2, f);
+        } else {
+          f = routed_next(a, w2, f, lane, nxt);
+        }
+        const int nrows = nxt.rows_x[0] + nxt.rows_x[1];
 #pragma unroll
         for (int x = 0; x < 2; ++x)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             int r = x * kTileM + 4 * lane + i;
             if (r >= nrows) r = 0;
-            const uint2 e = a.entries[it.e0 + r];
+            nent[x][i] = a.entries[nxt.e0 + r];
+          }
+      };
+      if (first < items) lookup(first);
+      for (int64_t w = first; w < items && ok; w += step, ++lt) {
+        const Item it = nxt;
+        int ys[2][4];
+#pragma unroll
+        for (int x = 0; x < 2; ++x)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint2 e = nent[x][i];
             const bool good = e.x < (uint32_t)a.L.T && (e.y & 0xFFFFu) < (uint32_t)a.G;
             const int hq = it.g * a.G + (good ? (int)(e.y & 0xFFFFu) : 0);
             ys[x][i] = (int)((int64_t)(good ? e.x : 0u) * a.Hq + hq);
           }
+        if (w + step < items) lookup(w + step);
+        const int qb = lt % QB;
+        ok = mbar_wait(&q_empty[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
+        if (ok) ok = mbar_wait(&desc_free[qb], ((lt / QB) & 1) ^ 1, abort_flag, st);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
         if (lane == 0) {
           sItem[qb] = it;  // published by q_full, with the rows
           mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
