@@ -546,6 +546,24 @@ __global__ void __launch_bounds__(352, 1)
             tma_gather4(sQ + qb * C::kQBytes + x * C::kSubQBytes + hx * C::kHalfBytes +
                             lane * 4 * 128,
                         &tm_q, &q_full[qb], hx * 64, ys[x][0], ys[x][1], ys[x][2], ys[x][3]);
+        if (QB == 1 && w + step < items) {
+          // one Q buffer (long items): the next item's rows can only be
+          // gathered once this item's MMAs are done, so bring them into L2 now
+#pragma unroll
+          for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint2 e = nent[x][i];
+              const bool good = e.x < (uint32_t)a.L.T && (e.y & 0xFFFFu) < (uint32_t)a.G;
+              const int hq = nxt.g * a.G + (good ? (int)(e.y & 0xFFFFu) : 0);
+              ys[x][i] = (int)((int64_t)(good ? e.x : 0u) * a.Hq + hq);
+            }
+#pragma unroll
+          for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int hx = 0; hx < D / 64; ++hx)
+              tma_prefetch_gather4(&tm_q, hx * 64, ys[x][0], ys[x][1], ys[x][2], ys[x][3]);
+        }
       }
       if (!ok && lane == 0) {  // let the gathers in flight land before the CTA exits
         for (uint32_t b = 0; b < (lt < (uint32_t)QB ? lt : (uint32_t)QB); ++b) {
@@ -645,6 +663,10 @@ __global__ void __launch_bounds__(352, 1)
       if (it.nkv_x[0] > 0) issue_s(0, qbase, ks);
       if (it.nkv_x[1] > 0) issue_s(1, qbase, ks);
       tc_commit_warp(&kv_empty[ks]);
+      // The Q buffer is free once the item's last S MMAs complete, before
+      // its last PV MMAs: the next item's rows start loading that much
+      // earlier (the commit covers every MMA issued so far).
+      if (it.nkv == 1) tc_commit_warp(&q_empty[qb]);
       for (int j = 0; j < it.nkv && ok; ++j) {
         const uint32_t vs = kv_it % ST;
         if (!(ok = wait(&kv_full[vs], (kv_it / ST) & 1))) break;
@@ -660,12 +682,12 @@ __global__ void __launch_bounds__(352, 1)
         }
         if (!(ok = kv_step(0, it, j, vs, ks2, qbase))) break;
         if (!(ok = kv_step(1, it, j, vs, ks2, qbase))) break;
+        if (j == it.nkv - 2) tc_commit_warp(&q_empty[qb]);  // every S of the item issued
         // a slot is released only after its load has been waited for
         if (!(ok = ensure_k())) break;
         tc_commit_warp(&kv_empty[vs]);
         if (more) tc_commit_warp(&kv_empty[ks2]);
       }
-      if (ok) tc_commit_warp(&q_empty[qb]);
     }
     tc_commit_warp(td_bar);
     mbar_wait_teardown(td_bar, 0, 500000000ull);

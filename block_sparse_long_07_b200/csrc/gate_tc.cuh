@@ -530,6 +530,11 @@ __global__ void __launch_bounds__(352, 1)
           if (take && kept < npast) out[kept] = id;
           kept += take ? 1 : 0;
         }
+      } else if (nc <= npast) {
+        // no more candidates than kept blocks (pass 1's bound was exact, as
+        // it is whenever every score is its own group): keep them all
+        for (int q = 0; q < nc; ++q) out[q] = (int32_t)ci[q * kTileM];
+        kept = nc;
       } else {
         for (int q = 0; q < nc; ++q) chain_insert<KM>(t, cv[q * kTileM]);
         const float T1 = list_at<KM>(t, npast - 1);
