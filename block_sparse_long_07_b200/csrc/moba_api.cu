@@ -198,6 +198,9 @@ moba_status make_problem(const moba_params* p, bool varlen, const int32_t* cu, i
   pr.Hq = p->num_q_heads;
   pr.Hkv = p->num_kv_heads;
   pr.G = pr.Hq / pr.Hkv;
+  // q rows are addressed as one int32 index of q viewed as [T*Hq][D] (TMA
+  // row gathers); that q would be 512 GB at D = 128
+  if (pr.T * pr.Hq >= (int64_t)INT32_MAX) return MOBA_ERR_UNSUPPORTED;
   if (p->head_dim != 64 && p->head_dim != 128) return MOBA_ERR_UNSUPPORTED;
   pr.D = p->head_dim;
   if (need_blocks) {
@@ -281,7 +284,7 @@ bool make_tmap(CUtensorMap* m, const void* ptr, int H, int64_t T, int D) {
 
 // [T][H][D] bf16 viewed as rows (x = D, y = T*H), box 64 x 1, 128-B swizzle:
 // the routed kernel's four-row gathers of (token, head) rows.  Row indices
-// are int32, so T*H must stay below 2^31 (forward_setup checks).
+// are int32, so T*H must stay below 2^31 (make_problem checks).
 bool make_tmap_rows(CUtensorMap* m, const void* ptr, int64_t rows, int D) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
@@ -611,7 +614,6 @@ struct FwdCtx {
 template <int D>
 moba_status forward_setup(const Problem& pr, const void* q, const void* k, const void* v,
                           void* o, float* lse, const Ws& w, FwdCtx* c) {
-  if (pr.T * pr.Hq >= (int64_t)INT32_MAX) return MOBA_ERR_UNSUPPORTED;  // int32 q row index
   if (!make_tmap(&c->tq, q, pr.Hq, pr.T, D) || !make_tmap(&c->tk, k, pr.Hkv, pr.T, D) ||
       !make_tmap(&c->tv, v, pr.Hkv, pr.T, D) || !make_tmap_rows(&c->tq_rows, q, pr.T * pr.Hq, D))
     return MOBA_ERR_CUDA;

@@ -88,6 +88,8 @@ def test_workspace_size_grows_with_heads_per_pass(lib):
     (dict(Hkv=0), INVALID),
     (dict(batch=0), INVALID),
     (dict(seqlen=-1), INVALID),
+    # T * Hq = 2^31 (q rows take an int32 index)
+    (dict(seqlen=1 << 26, block_size=1 << 20), UNSUPPORTED),
 ])
 def test_bad_params_rejected(lib, kw, code):
     p = _p(**kw)
