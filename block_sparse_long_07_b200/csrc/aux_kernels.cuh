@@ -527,16 +527,17 @@ __global__ void __launch_bounds__(128) bucket_scatter_kernel(
 // and the own-block partial (fp32 O, log2 lse) -- are combined by the
 // online-softmax rule
 //   m = max lse_s, w_s = 2^(lse_s - m), O = sum w_s O_s / sum w_s,
-//   lse = m + log2(sum w_s)   (output converted to natural log).
+//   lse = m + log2(sum w_s)   (output converted to natural log),
+// with m the running maximum (sums rescaled when it grows).
 // A group of D/8 lanes owns one (token, head) row; each lane owns 8 of its
 // columns, so every partial row is read with one 16-byte load per lane and
-// four slots are loaded before any is used.  Rows whose selection is the own
-// block alone were finished by the own-block kernel and are skipped.  The
-// own-block partial is combined first, then the routed slots in ascending
-// order.  The routed partials were stored multiplied by 2^-S (S from
-// partial_scale_log2, 0 unless some |v| reaches 2^15); their weights carry
-// the 2^S back.  A merged row that is not finite (non-finite inputs) is
-// reported in the status word as MOBA_DEV_CAPACITY.
+// eight slots (O rows and lse) are loaded before any is used.  Rows whose
+// selection is the own block alone were finished by the own-block kernel and
+// are skipped.  The own-block partial is combined first, then the routed
+// slots in ascending order.  The routed partials were stored multiplied by
+// 2^-S (S from partial_scale_log2, 0 unless some |v| reaches 2^15); their
+// weights carry the 2^S back.  A merged row that is not finite (non-finite
+// inputs) is reported in the status word as MOBA_DEV_CAPACITY.
 template <int D>
 __global__ void __launch_bounds__(256) merge_kernel(
     const __half* __restrict__ part_O, const float* __restrict__ part_lse,
@@ -564,39 +565,50 @@ __global__ void __launch_bounds__(256) merge_kernel(
   const int64_t prow = ((int64_t)u * L.T + t) * G + hh;  // partial row
   const int64_t pbase = prow * (topk - 1);
   const float* lrow = part_lse + pbase;
-  const float lown = own_lse[prow];
-  float m = lown;
-  for (int sl = 0; sl < npast; ++sl) m = fmaxf(m, lrow[sl]);
+  // One pass with a running maximum: each batch's lse and O rows are loaded
+  // together, 8 slots in flight, instead of every lse before any O row.
+  float m = own_lse[prow];
+  float den = 1.f;  // the own partial's weight, relative to m
   float acc[8];
-  float den;
   {
-    const float w = ex2_approx(lown - m);
-    den = w;
     const float4* src = reinterpret_cast<const float4*>(own_O + prow * D + sub * 8);
     const float4 a = src[0], b = src[1];
-    acc[0] = w * a.x;
-    acc[1] = w * a.y;
-    acc[2] = w * a.z;
-    acc[3] = w * a.w;
-    acc[4] = w * b.x;
-    acc[5] = w * b.y;
-    acc[6] = w * b.z;
-    acc[7] = w * b.w;
+    acc[0] = a.x;
+    acc[1] = a.y;
+    acc[2] = a.z;
+    acc[3] = a.w;
+    acc[4] = b.x;
+    acc[5] = b.y;
+    acc[6] = b.z;
+    acc[7] = b.w;
   }
   const uint4* orow = reinterpret_cast<const uint4*>(part_O + pbase * D) + sub;
   constexpr int kStride = D / 8;  // uint4 per partial row
-  int sl = 0;
-  for (; sl + 4 <= npast; sl += 4) {
-    uint4 v[4];
-    float w[4];
+  constexpr int kBatch = 8;
+  for (int sl = 0; sl < npast; sl += kBatch) {
+    uint4 v[kBatch];
+    float l[kBatch];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) v[q] = orow[(sl + q) * kStride];
+    for (int q = 0; q < kBatch; ++q) {
+      const bool in = sl + q < npast;
+      v[q] = in ? orow[(sl + q) * kStride] : make_uint4(0u, 0u, 0u, 0u);
+      l[q] = in ? lrow[sl + q] : -INFINITY;
+    }
+    float mb = l[0];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) w[q] = ex2_approx(lrow[sl + q] - m);
+    for (int q = 1; q < kBatch; ++q) mb = fmaxf(mb, l[q]);
+    if (mb > m) {  // rescale what is summed so far to the new maximum
+      const float sc = ex2_approx(m - mb);
+      den *= sc;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      den += w[q];
-      const float wo = w[q] * unscale;
+      for (int e = 0; e < 8; ++e) acc[e] *= sc;
+      m = mb;
+    }
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const float w = ex2_approx(l[q] - m);  // 0 past the row's slots
+      den += w;
+      const float wo = w * unscale;
       const __half2* h2 = reinterpret_cast<const __half2*>(&v[q]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -604,19 +616,6 @@ __global__ void __launch_bounds__(256) merge_kernel(
         acc[2 * e] = fmaf(wo, f.x, acc[2 * e]);
         acc[2 * e + 1] = fmaf(wo, f.y, acc[2 * e + 1]);
       }
-    }
-  }
-  for (; sl < npast; ++sl) {
-    const uint4 v = orow[sl * kStride];
-    const float w = ex2_approx(lrow[sl] - m);
-    den += w;
-    const float wo = w * unscale;
-    const __half2* h2 = reinterpret_cast<const __half2*>(&v);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __half22float2(h2[e]);
-      acc[2 * e] = fmaf(wo, f.x, acc[2 * e]);
-      acc[2 * e + 1] = fmaf(wo, f.y, acc[2 * e + 1]);
     }
   }
   bool finite = true;
