@@ -22,6 +22,10 @@
 //   warp  8     TMA producer: Q tiles (own/dense) and the K/V ring
 //   warp  9     TMEM allocation and MMA issue (one elected lane per MMA)
 //   warp 10     Q row gather for routed items (TMA four-row gathers)
+// Each Q buffer carries its item's descriptor in shared memory, written by
+// whoever fills the buffer and released by the softmax warps once read.  The
+// buffer itself is released when the item's last S MMAs complete, one KV step
+// before its last PV MMAs.
 // TMEM (512 columns): S_X at 128*X (fp32 scores; after the softmax the first
 // 64 columns hold P_X as packed bf16, and on the first tile of an own/dense
 // block columns 64..95 hold the residual weights of rows 0..63), O_X at
