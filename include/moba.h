@@ -63,7 +63,9 @@ typedef enum moba_status {
   MOBA_OK = 0,
   MOBA_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad size or shape */
   MOBA_ERR_UNSUPPORTED = 2,  /* head_dim not 64/128, block_size not a multiple of 128,
-                                top_k beyond 65, too many blocks per sequence */
+                                top_k beyond 65, too many blocks per sequence,
+                                tokens x num_q_heads >= 2^31 (q rows take an int32
+                                index) */
   MOBA_ERR_WORKSPACE = 3,    /* ws null, misaligned (256 B) or smaller than required */
   MOBA_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, attribute, device) */
   MOBA_ERR_TIMEOUT = 5,      /* device: a pipeline wait ran out of time */
