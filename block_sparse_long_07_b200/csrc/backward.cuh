@@ -18,9 +18,9 @@
 //                 TMEM A operands of dV += P^T dO and dK += dS^T Q, accumulated
 //                 in TMEM; the elementwise pass of a tile overlaps the MMAs
 //                 of its neighbours
-//   bw_q_kernel   one CTA per tile of 128 rows (gathered or own): loops over
-//                 the block's key tiles; dS packed as bf16 into TMEM is the A
-//                 operand of dQ += dS K
+//   bw_q2_kernel  one CTA per tile of 128 rows (gathered or own), warp
+//                 roles: walks the block's key tiles in halves of 64 keys; dS
+//                 packed as bf16 into TMEM is the A operand of dQ += dS K
 // The Q / dO tiles ([rows][d], 128-byte swizzled) serve both as K-major
 // operands (S, dP and their transposes) and as MN-major B operands (dK, dV);
 // K / V tiles likewise.
@@ -134,7 +134,7 @@ __device__ __forceinline__ void bw_load_row(const BwArgs& a, BwRow x, int r, int
 }
 
 // ---------------------------------------------------------------- dK / dV, warp-specialised
-// One CTA per (bucket or own block, 128-key tile), as bw_kv_kernel, with the
+// One CTA per (bucket or own block, 128-key tile), with the
 // rows in 64-row tiles so that TMEM holds two tiles' S^T / dP^T next to the
 // dV / dK accumulators: the elementwise pass of tile n runs while the tensor
 // core computes dV / dK of tile n - 1 and S^T / dP^T of tile n + 1.
@@ -471,7 +471,7 @@ __global__ void __launch_bounds__(352, 1)
 }
 
 // ---------------------------------------------------------------- dQ, warp-specialised
-// One CTA per 128-row tile, as bw_q_kernel, with each 128-key K / V tile taken
+// One CTA per 128-row tile, with each 128-key K / V tile taken
 // in two halves of 64 keys so that TMEM holds two halves' S / dP next to the
 // dQ accumulator: the elementwise pass of half m runs while the tensor core
 // computes dQ of half m - 1 and S / dP of half m + 1.
